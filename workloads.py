@@ -1,0 +1,200 @@
+"""Seeded synthetic inputs for the varlen attention forward.
+
+This module only draws random numbers and lays them out; it holds none of the
+attention arithmetic.  It is the one module that both the oracle side (tests,
+CPU baseline) and the CUDA side (tests, bench) use, so both see identical
+inputs.
+
+Workloads (sequence lengths, head counts, head dim, dtype, mask) follow the
+five benchmark configurations of the varlen attention forward:
+
+  tiny      3 packed sequences {17, 64, 1}, H=Hkv=4, D=64, bf16, causal
+  gqa       8 sequences, q_len=k_len uniform-int [128, 2048], H=32, Hkv=8,
+            D=128, bf16, causal
+  long      16 sequences, log-uniform lengths in [64, 16384] rescaled to a
+            total of exactly 65536 tokens, H=64, Hkv=8, D=128, bf16, causal
+  shortq    32 sequences, q_len uniform-int [1, 64], k_len uniform-int
+            [512, 8192], H=32, Hkv=4, D=128, bf16, non-causal
+  wide      4 sequences of 4096, H=Hkv=16, D=256, fp16, Q/K ~ N(0, 3^2),
+            V ~ N(0, 1), causal
+
+Length recipe: numpy ``default_rng(seed)`` (PCG64).  Tensor recipe:
+``torch.Generator('cpu').manual_seed(seed)``, fp32 ``randn`` drawn in the
+order Q [Tq,H,D], K [Tk,Hkv,D], V [Tk,Hkv,D], multiplied by sigma, then cast
+to the storage dtype (round to nearest even).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import List, Optional, Sequence
+
+import numpy as np
+import torch
+
+DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    seed: int
+    H: int
+    Hkv: int
+    D: int
+    dtype: str
+    causal: bool
+    sigma_q: float = 1.0
+    sigma_k: float = 1.0
+    sigma_v: float = 1.0
+    description: str = ""
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 4, 4, 64, "bf16", True,
+                     description="3 packed sequences {17,64,1}, H=Hkv=4, D=64, bf16, causal"),
+    "gqa": Workload("gqa", 2, 32, 8, 128, "bf16", True,
+                    description="GQA prefill: 8 sequences in [128,2048], H=32, Hkv=8, D=128, bf16, causal"),
+    "long": Workload("long", 3, 64, 8, 128, "bf16", True,
+                     description="long ragged prefill: 16 log-uniform sequences totalling 65536 tokens, "
+                                 "H=64, Hkv=8, D=128, bf16, causal"),
+    "shortq": Workload("shortq", 4, 32, 4, 128, "bf16", False,
+                       description="short-query/long-KV: 32 sequences q in [1,64], k in [512,8192], "
+                                   "H=32, Hkv=4, D=128, bf16, non-causal"),
+    "wide": Workload("wide", 5, 16, 16, 256, "fp16", True, sigma_q=3.0, sigma_k=3.0, sigma_v=1.0,
+                     description="wide-head MHA: 4x4096, H=Hkv=16, D=256, fp16, Q/K sigma 3, causal"),
+}
+
+
+def _long_lengths(seed: int, n: int = 16, total: int = 65536,
+                  lo: int = 64, hi: int = 16384) -> List[int]:
+    rng = np.random.default_rng(seed)
+    u = rng.uniform(math.log(lo), math.log(hi), n)
+    raw = np.exp(u)
+    raw = raw * (total / raw.sum())
+    base = np.maximum(1, np.floor(raw)).astype(np.int64)
+    remainder = total - int(base.sum())
+    frac = raw - np.floor(raw)
+    # remainder goes to the largest fractional parts; ties go to the lower index
+    order = sorted(range(n), key=lambda i: (-frac[i], i))
+    for i in order[:remainder]:
+        base[i] += 1
+    return [int(x) for x in base]
+
+
+def seqlens(name: str):
+    """Per-sequence (q_lens, k_lens) of a named workload."""
+    w = WORKLOADS[name]
+    if name == "tiny":
+        q = [17, 64, 1]
+        return q, list(q)
+    if name == "gqa":
+        rng = np.random.default_rng(w.seed)
+        q = [int(x) for x in rng.integers(128, 2049, 8)]
+        return q, list(q)
+    if name == "long":
+        q = _long_lengths(w.seed)
+        return q, list(q)
+    if name == "shortq":
+        rng = np.random.default_rng(w.seed)
+        q = [int(x) for x in rng.integers(1, 65, 32)]
+        k = [int(x) for x in rng.integers(512, 8193, 32)]
+        return q, k
+    if name == "wide":
+        q = [4096] * 4
+        return q, list(q)
+    raise KeyError(name)
+
+
+def cu_seqlens(lens: Sequence[int]) -> torch.Tensor:
+    """Exclusive prefix sums [0, l0, l0+l1, ...] as int32."""
+    out = [0]
+    for x in lens:
+        out.append(out[-1] + int(x))
+    return torch.tensor(out, dtype=torch.int32)
+
+
+@dataclass
+class Case:
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    cu_q: torch.Tensor
+    cu_k: torch.Tensor
+    lens_q: List[int]
+    lens_k: List[int]
+    H: int
+    Hkv: int
+    D: int
+    causal: bool
+    dtype: str
+    scale: float
+    name: str = "custom"
+    seed: int = 0
+
+    @property
+    def B(self) -> int:
+        return len(self.lens_q)
+
+    @property
+    def max_q(self) -> int:
+        return max(self.lens_q) if self.lens_q else 0
+
+    @property
+    def max_k(self) -> int:
+        return max(self.lens_k) if self.lens_k else 0
+
+    @property
+    def Tq(self) -> int:
+        return int(self.cu_q[-1])
+
+    @property
+    def Tk(self) -> int:
+        return int(self.cu_k[-1])
+
+
+def make_case(lens_q: Sequence[int], lens_k: Optional[Sequence[int]], H: int, Hkv: int, D: int,
+              dtype: str = "bf16", causal: bool = True, seed: int = 0,
+              sigma_q: float = 1.0, sigma_k: float = 1.0, sigma_v: float = 1.0,
+              scale: Optional[float] = None, name: str = "custom") -> Case:
+    """Seeded random packed inputs for arbitrary lengths and head shapes."""
+    lens_q = [int(x) for x in lens_q]
+    lens_k = [int(x) for x in (lens_k if lens_k is not None else lens_q)]
+    assert len(lens_q) == len(lens_k)
+    Tq, Tk = sum(lens_q), sum(lens_k)
+    g = torch.Generator("cpu").manual_seed(seed)
+    tdt = DTYPES[dtype]
+    q = (torch.randn((Tq, H, D), generator=g, dtype=torch.float32) * sigma_q).to(tdt)
+    k = (torch.randn((Tk, Hkv, D), generator=g, dtype=torch.float32) * sigma_k).to(tdt)
+    v = (torch.randn((Tk, Hkv, D), generator=g, dtype=torch.float32) * sigma_v).to(tdt)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    return Case(q, k, v, cu_seqlens(lens_q), cu_seqlens(lens_k), lens_q, lens_k,
+                H, Hkv, D, causal, dtype, float(scale), name=name, seed=seed)
+
+
+def make_workload(name: str) -> Case:
+    """Full-size inputs of a named workload (CPU tensors)."""
+    w = WORKLOADS[name]
+    lq, lk = seqlens(name)
+    return make_case(lq, lk, w.H, w.Hkv, w.D, w.dtype, w.causal, w.seed,
+                     w.sigma_q, w.sigma_k, w.sigma_v, name=name)
+
+
+def sample_rows(case: Case, n: int, seed: int = 1234) -> np.ndarray:
+    """A seeded sample of (token, head) output rows that always includes the
+    first and last row of every sequence (ragged edges) plus random rows."""
+    rng = np.random.default_rng(seed)
+    rows = set()
+    cu = case.cu_q.tolist()
+    for b in range(case.B):
+        if cu[b + 1] > cu[b]:
+            for tok in (cu[b], cu[b + 1] - 1, min(cu[b] + 127, cu[b + 1] - 1),
+                        min(cu[b] + 128, cu[b + 1] - 1)):
+                rows.add((tok, int(rng.integers(0, case.H))))
+    if case.Tq > 0:
+        toks = rng.integers(0, case.Tq, n)
+        hs = rng.integers(0, case.H, n)
+        rows.update(zip(toks.tolist(), hs.tolist()))
+    arr = np.array(sorted(rows), dtype=np.int64).reshape(-1, 2)
+    return arr
