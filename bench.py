@@ -1,0 +1,438 @@
+"""Benchmark of the B200 varlen attention forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long]
+    python bench.py --impl reference ...     # the fp64 CPU oracle arm
+
+One step = one call of the C-ABI entry point ``varlen_attn_fwd`` over one
+batch of the workload (inputs resident in HBM).  The default workload is the
+long ragged prefill (16 causal sequences, 65536 tokens, H=64, Hkv=8, D=128,
+bf16), the configuration the throughput target is stated on.  The metric is
+TFLOP/s with FLOPs = 4 * D * (unmasked query-key pairs summed over heads).
+
+Prints ONE JSON line on rank 0.  With N > 1 (launched by torchrun) every rank
+runs its own batch of the workload (weak scaling, no collective on the data
+path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "varlen attn fwd TFLOP/s (unmasked FLOPs) and % of B200 dense bf16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["flash_attention_fwd_b200/csrc/varlen_attn_fwd.cu",
+                  "flash_attention_fwd_b200/csrc/sm100_ptx.cuh"]
+
+
+# ----------------------------------------------------------------------------- counting
+
+def visible_keys(lq: int, lk: int, causal: bool) -> int:
+    """Unmasked (query, key) pairs of one sequence and one head."""
+    if not causal:
+        return lq * lk
+    # query qi sees keys 0..min(qi, lk-1): min(qi+1, lk) keys
+    n = min(lq, lk)
+    full = n * (n + 1) // 2
+    return full + max(0, lq - lk) * lk
+
+
+def unmasked_pairs(lens_q, lens_k, H: int, causal: bool) -> int:
+    return H * sum(visible_keys(a, b, causal) for a, b in zip(lens_q, lens_k))
+
+
+def step_flops(case) -> int:
+    return 4 * case.D * unmasked_pairs(case.lens_q, case.lens_k, case.H, case.causal)
+
+
+def algorithmic_bytes(case) -> int:
+    e = 2
+    return (case.Tq * case.H * case.D * e * 2 + 2 * case.Tk * case.Hkv * case.D * e
+            + 4 * case.Tq * case.H + 8 * (case.B + 1))
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, only if it was
+    taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d.get(workload)
+        if ent and ent.get("kernel_hash") == kernel_hash():
+            return ent.get("bytes_per_launch")
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons, taken while
+    the timed region runs."""
+    FIELDS = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = bus_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.bus_id:
+                cmd += ["-i", self.bus_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        try:
+            rows = [l.strip().split(", ") for l in open(self.path) if l.strip()]
+            os.unlink(self.path)
+        except Exception:
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 10:
+                continue
+            try:
+                sm.append(float(r[2]))
+                mx.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[6:10]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def gpu_bus_id(dev_index: int):
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev_index)
+        return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample_rows(case, n_rows: int, seed: int = 99):
+    rows = workloads.sample_rows(case, n_rows, seed=seed)
+    G = case.H // case.Hkv
+    cu = case.cu_q.numpy()
+    b = np.searchsorted(cu, rows[:, 0], side="right") - 1
+    order = np.lexsort((rows[:, 0], rows[:, 1], rows[:, 1] // G, b))
+    rows = rows[order]
+    b = b[order]
+    qi = rows[:, 0] - cu[b]
+    lk = np.asarray(case.lens_k)[b]
+    vis = np.minimum(qi + 1, lk) if case.causal else lk
+    flops = int(4 * case.D * int(vis.sum()))
+    return rows, flops
+
+
+def time_oracle(case, seconds: float, nthreads: int | None = None):
+    """Times the fp64 oracle (as it stands) on a seeded row sample sized for
+    about ``seconds`` of CPU work.  Returns (TFLOP/s, rows, flops, secs)."""
+    import oracle
+    nthreads = nthreads or oracle.default_threads()
+    rows, fl = oracle_sample_rows(case, 256, seed=98)
+    t0 = time.perf_counter()
+    oracle.run_case_rows(case, rows, nthreads=nthreads)
+    rate = fl / max(time.perf_counter() - t0, 1e-6)
+    avg_row = fl / max(len(rows), 1)
+    n = int(max(64, min(2_000_000, seconds * rate / max(avg_row, 1))))
+    rows, fl = oracle_sample_rows(case, n, seed=99)
+    t0 = time.perf_counter()
+    oracle.run_case_rows(case, rows, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    return fl / dt / 1e12, len(rows), fl, dt, nthreads
+
+
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of per-rank timings (every rank calls it)."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: int, ms_per_step: float) -> float:
+    """Aggregate throughput: every rank processes one batch per step."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank: int, world: int):
+    import torch
+    import flash_attention_fwd_b200 as fa
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    case = workloads.make_workload(args.workload)
+    flops = step_flops(case)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    cq, ck = case.cu_q.to(dev), case.cu_k.to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((case.Tq, case.H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fa.load_library()
+    fa.device_status(clear=True)
+
+    def step():
+        fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, case.causal, case.scale,
+                           out=out, lse=lse, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(gpu_bus_id(local))
+    clocks.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    status = fa.device_status(clear=True)
+    if status != 0:
+        raise RuntimeError("device status word set: %d" % status)
+
+    # ---- end to end: pinned host inputs -> device -> kernel -> host results
+    if args.no_e2e:
+        e2e_ms, h2d, d2h = float("nan"), 0, 0
+    else:
+        e2e_ms, h2d, d2h = run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist)
+
+    if dist:
+        total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
+        dist.barrier()
+    emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk)
+    if dist:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist):
+    import torch
+    hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+    hcq, hck = case.cu_q.pin_memory(), case.cu_k.pin_memory()
+    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        cq.copy_(hcq, non_blocking=True)
+        ck.copy_(hck, non_blocking=True)
+        step()
+        ho.copy_(out, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    return e2e_ms, h2d, d2h
+
+
+def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk):
+    if rank == 0:
+        ms = total_ms / args.steps
+        value = whole_job_tflops(world, flops, ms)
+        peaks, peak_src = load_peaks()
+        peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        avg_launch_ms = sum(per_launch) / len(per_launch)
+        achieved = flops / (avg_launch_ms * 1e-3) / 1e12
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            tfs, nrows, fl, dt, thr = time_oracle(case, args.cpu_seconds)
+            cpu = {"value": tfs, "unit": UNIT, "cores": thr, "kind": "oracle",
+                   "sample": "%d seeded random (token, head) rows of the %s workload, "
+                             "%.2f GFLOP of its %.2f TFLOP step, %.1f s on %d threads"
+                             % (nrows, args.workload, fl / 1e9, flops / 1e12, dt, thr)}
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": case.dtype, "data": "synthetic (seeded N(0,1) Q/K/V, seeded lengths)",
+            "config": {
+                "workload": workloads.WORKLOADS[args.workload].description,
+                "name": args.workload, "batch_sequences": case.B, "total_q": case.Tq,
+                "total_k": case.Tk, "max_seqlen": case.max_q, "H": case.H, "Hkv": case.Hkv,
+                "D": case.D, "causal": case.causal, "flops_per_step": flops,
+                "l2": "no flush: inputs (%.0f MB) exceed the 126 MB L2"
+                      % (algorithmic_bytes(case) / 1e6),
+                "parallelism": "dp%d (one independent batch per GPU)" % world},
+            "pct_of_peak": round(100.0 * achieved / peak, 2),
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "traffic": traffic_for(args.workload),
+                         "peak_source": "%s burst bf16 (sustained %.1f -> frac %.4f)"
+                                        % (peak_src, peak_sus, achieved / peak_sus)},
+            "launch_ms": {"min": round(min(per_launch), 4),
+                          "median": round(statistics.median(per_launch), 4),
+                          "max": round(max(per_launch), 4)},
+            "e2e": {"value": round(whole_job_tflops(world, flops, e2e_ms), 3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 3)},
+            "gpu_launches": args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        if args.no_e2e:
+            line["e2e"] = None
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank: int, world: int):
+    """The fp64 CPU oracle as it stands, on the host cores, one bounded row
+    sample of the workload per step."""
+    if rank != 0:
+        return
+    import oracle
+    case = workloads.make_workload(args.workload)
+    nthreads = oracle.default_threads()
+    budget = max(0.5, min(30.0, args.reference_seconds / max(1, args.steps + args.warmup)))
+    rows0, fl0 = oracle_sample_rows(case, 256, seed=98)
+    t0 = time.perf_counter()
+    oracle.run_case_rows(case, rows0, nthreads=nthreads)
+    rate = fl0 / max(time.perf_counter() - t0, 1e-6)
+    n = int(max(64, budget * rate / max(fl0 / len(rows0), 1)))
+    rows, fl = oracle_sample_rows(case, n, seed=99)
+    for _ in range(args.warmup):
+        oracle.run_case_rows(case, rows, nthreads=nthreads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.run_case_rows(case, rows, nthreads=nthreads)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = fl / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) Q/K/V, seeded lengths)",
+        "config": {"workload": workloads.WORKLOADS[args.workload].description,
+                   "name": args.workload, "sample_rows": len(rows), "sample_flops": fl},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": "%d seeded random (token, head) rows per step, %.2f GFLOP"
+                                   % (len(rows), fl / 1e9)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="long", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=120.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_gpu(args, rank, world)
+
+
+if __name__ == "__main__":
+    main()

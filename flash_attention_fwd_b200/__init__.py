@@ -1,0 +1,171 @@
+"""B200-native (sm_100a) packed variable-length attention forward.
+
+Python binding of the C ABI declared in ``include/varlen_attn.h``.  This
+module only marshals arguments: every step of the attention forward runs in
+the CUDA kernels of ``libvarlen_attn.so``.  There is no CPU or PyTorch
+fallback; if the library cannot be loaded, calls raise.
+
+The operation is the varlen attention forward of boostr 0.2.0,
+src/ops/cpu/attention/varlen_attention.rs (``varlen_attention_fwd``), with
+the out-variant calling convention of PyTorch pull request #176015
+(``_flash_attention_forward_no_dropout_inplace``: output written into a
+caller buffer, log-sum-exp returned).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libvarlen_attn.so")
+
+VARLEN_BF16 = 0
+VARLEN_FP16 = 1
+DTYPE_CODES = {torch.bfloat16: VARLEN_BF16, torch.float16: VARLEN_FP16}
+
+VARLEN_OK = 0
+STATUS_NAMES = {
+    0: "VARLEN_OK", -1: "VARLEN_ERR_NULL", -2: "VARLEN_ERR_SHAPE", -3: "VARLEN_ERR_DTYPE",
+    -4: "VARLEN_ERR_ALIGN", -5: "VARLEN_ERR_LAUNCH", -6: "VARLEN_ERR_DEVICE",
+    -7: "VARLEN_ERR_ARCH",
+}
+
+# Every symbol include/varlen_attn.h declares.
+EXPORTED_SYMBOLS = (
+    "varlen_attn_fwd_v1",
+    "varlen_attn_fwd",
+    "varlen_attn_strerror",
+    "varlen_attn_device_status",
+    "varlen_attn_abi_version",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+
+class VarlenAttnError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("%s (%d): %s" % (STATUS_NAMES.get(code, "?"), code, msg))
+        self.code = code
+
+
+def _bind(lib):
+    P = ctypes.c_void_p
+    i32, i64, f32 = ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    fwd_args = [P, P, P, P, P, i32, i64, i64, i32, i32, i32, i32, i32, i32, f32, i32, P, P, P]
+    for name in ("varlen_attn_fwd_v1", "varlen_attn_fwd"):
+        fn = getattr(lib, name)
+        fn.argtypes = fwd_args
+        fn.restype = i32
+    lib.varlen_attn_strerror.argtypes = [i32]
+    lib.varlen_attn_strerror.restype = ctypes.c_char_p
+    lib.varlen_attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i32]
+    lib.varlen_attn_device_status.restype = i32
+    lib.varlen_attn_abi_version.argtypes = []
+    lib.varlen_attn_abi_version.restype = i32
+    return lib
+
+
+def load_library(build_if_missing: bool = True):
+    """Load (building first if it is missing or stale) the CUDA library."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if build_if_missing:
+                from . import build as _build
+                _build.build()
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError("CUDA extension %s is missing; run "
+                                   "`python -m flash_attention_fwd_b200.build`" % LIB_PATH)
+            _lib = _bind(ctypes.CDLL(LIB_PATH))
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return load_library().varlen_attn_strerror(int(code)).decode()
+
+
+def device_status(clear: bool = True) -> int:
+    """Device-side status word (bit 1 = a bounded pipeline wait timed out)."""
+    val = ctypes.c_uint(0)
+    rc = load_library().varlen_attn_device_status(ctypes.byref(val), int(clear))
+    if rc != VARLEN_OK:
+        raise VarlenAttnError(rc, strerror(rc))
+    return int(val.value)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return ctypes.c_void_p(t.data_ptr() if t is not None and t.numel() > 0 else 0)
+
+
+def varlen_attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, cu_q_ptr: int, cu_k_ptr: int,
+                        batch: int, total_q: int, total_k: int, max_seqlen_q: int,
+                        max_seqlen_k: int, num_heads: int, num_kv_heads: int, head_dim: int,
+                        causal: bool, scale: float, dtype_code: int, out_ptr: int,
+                        lse_ptr: int, stream: int) -> int:
+    """Direct call of the C entry point with integer addresses; returns the
+    status code unchanged."""
+    lib = load_library()
+    V = ctypes.c_void_p
+    return lib.varlen_attn_fwd(V(q_ptr), V(k_ptr), V(v_ptr), V(cu_q_ptr), V(cu_k_ptr),
+                               int(batch), int(total_q), int(total_k), int(max_seqlen_q),
+                               int(max_seqlen_k), int(num_heads), int(num_kv_heads),
+                               int(head_dim), int(bool(causal)), float(scale), int(dtype_code),
+                               V(out_ptr), V(lse_ptr), V(stream))
+
+
+def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                    max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,
+                    scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                    lse: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Packed attention forward on the GPU.
+
+    q [Tq, H, D], k/v [Tk, Hkv, D] (bf16 or fp16, contiguous, on one CUDA
+    device); cu_seqlens_q/k int32 [B+1] on the same device.  Writes ``out``
+    ([Tq, H, D], q's dtype) and ``lse`` ([Tq, H], float32) — allocated here
+    when not given — and returns them.  ``scale=None`` selects 1/sqrt(D).
+    """
+    if q.dtype not in DTYPE_CODES or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share dtype bfloat16 or float16")
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("expected q [Tq,H,D] and k, v [Tk,Hkv,D]")
+    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens_q", cu_seqlens_q),
+                    ("cu_seqlens_k", cu_seqlens_k)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise TypeError("cu_seqlens must be int32")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B+1 >= 1 entries")
+    total_q, H, D = q.shape
+    total_k, Hkv, Dk = k.shape
+    if Dk != D:
+        raise ValueError("head dims of q and k differ")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((total_q, H), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor shaped and typed like q")
+    if lse.shape != (total_q, H) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [Tq, H]")
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = varlen_attn_fwd_raw(
+            q.data_ptr(), k.data_ptr() if k.numel() else 0, v.data_ptr() if v.numel() else 0,
+            cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), cu_seqlens_q.numel() - 1,
+            total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), H, Hkv, D, causal,
+            0.0 if scale is None else float(scale), DTYPE_CODES[q.dtype],
+            out.data_ptr() if out.numel() else 0, lse.data_ptr() if lse.numel() else 0,
+            stream.cuda_stream)
+    if rc != VARLEN_OK:
+        raise VarlenAttnError(rc, strerror(rc))
+    return out, lse

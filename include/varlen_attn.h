@@ -1,0 +1,136 @@
+/*
+ * varlen_attn.h — C ABI of the B200 (sm_100a) variable-length attention
+ * forward.
+ *
+ * The operation is the packed ("varlen") scaled-dot-product attention
+ * forward of boostr 0.2.0, src/ops/cpu/attention/varlen_attention.rs
+ * (VarLenAttentionOps::varlen_attention_fwd): for every sequence b, query
+ * head h and sequence-local query index qi,
+ *
+ *   kv_h = h / (H / Hkv)                                   (GQA head map)
+ *   s_ki = scale * <Q[cu_q[b]+qi, h, :], K[cu_k[b]+ki, kv_h, :]>
+ *          for the keys ki in [0, Lk_b) that are visible: with causal != 0
+ *          key ki is hidden from query qi when qi < ki (sequence-local
+ *          indices, i.e. the mask is aligned at the top-left corner)
+ *   O[cu_q[b]+qi, h, :] = sum_ki softmax(s)_ki * V[cu_k[b]+ki, kv_h, :]
+ *   LSE[cu_q[b]+qi, h]  = max_ki s_ki + ln(sum_ki exp(s_ki - max))
+ *
+ * The calling convention follows the out-variant of PyTorch pull request
+ * #176015 "[varlen_attn for inference] add out variant"
+ * (_flash_attention_forward_no_dropout_inplace): the attention output is
+ * written into a caller-provided buffer, the softmax log-sum-exp is returned
+ * too, and there is no dropout, debug mask or RNG state.  That discussion
+ * also sets the rule that a stable C ABI is never changed in place: a new
+ * signature gets a new, versioned symbol.  varlen_attn_fwd is therefore an
+ * alias of varlen_attn_fwd_v1, whose signature will not change.
+ *
+ * All pointers passed to varlen_attn_fwd are DEVICE pointers that the caller
+ * allocates and owns.  The library allocates no memory per call, keeps no
+ * reference to any buffer after the call returns, and the call is
+ * asynchronous on `stream` (no host synchronisation, no host read of
+ * cu_seqlens).
+ */
+#ifndef VARLEN_ATTN_H_
+#define VARLEN_ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as the CUDA runtime's cudaStream_t. */
+struct CUstream_st;
+typedef struct CUstream_st *varlen_stream_t;
+
+typedef enum {
+    VARLEN_BF16 = 0, /* q, k, v and out hold bfloat16 */
+    VARLEN_FP16 = 1  /* q, k, v and out hold IEEE binary16 */
+} varlen_dtype_t;
+
+/* Status codes (0 = success, negative = error).  Every error except
+ * VARLEN_ERR_LAUNCH is detected on the host before anything is launched,
+ * and then no memory has been touched. */
+#define VARLEN_OK 0
+#define VARLEN_ERR_NULL (-1)        /* a required pointer is NULL */
+#define VARLEN_ERR_SHAPE (-2)       /* H % Hkv != 0, unsupported D, negative size, ... */
+#define VARLEN_ERR_DTYPE (-3)       /* dtype not VARLEN_BF16 / VARLEN_FP16 */
+#define VARLEN_ERR_ALIGN (-4)       /* q, k, v or out not 16-byte aligned; lse or cu_seqlens not 4-byte aligned */
+#define VARLEN_ERR_LAUNCH (-5)      /* the CUDA launch itself failed (see varlen_attn_strerror) */
+#define VARLEN_ERR_DEVICE (-6)      /* device-side status word set (see varlen_attn_device_status) */
+#define VARLEN_ERR_ARCH (-7)        /* current device is not compute capability 10.0 (B200/B100 class) */
+
+/*
+ * varlen_attn_fwd_v1 — packed attention forward, output written in place.
+ *
+ *   q            [total_q, H, D]   row-major, dtype, 16-byte aligned
+ *   k, v         [total_k, Hkv, D] row-major, dtype, 16-byte aligned
+ *   cu_seqlens_q [batch + 1] int32, device: cu_seqlens_q[0] = 0, non-decreasing,
+ *                cu_seqlens_q[batch] <= total_q.  Sequence b owns query rows
+ *                [cu_seqlens_q[b], cu_seqlens_q[b+1]).
+ *   cu_seqlens_k [batch + 1] int32, device, same rules against total_k.
+ *   batch        number of sequences B (>= 0; 0 is a no-op)
+ *   total_q, total_k   number of token rows allocated in q/out/lse and in k/v.
+ *                Every TMA read is bounded by these extents, so a sequence
+ *                table that runs past them cannot make the kernel read or
+ *                write outside the buffers.
+ *   max_seqlen_q, max_seqlen_k   upper bounds of the per-sequence lengths
+ *                (>= 0).  They only size the launch; the kernel walks the
+ *                actual lengths from cu_seqlens, so an understated bound
+ *                costs occupancy, never correctness.
+ *   num_heads H, num_kv_heads Hkv   H % Hkv == 0; query head h reads
+ *                key/value head h / (H / Hkv).
+ *   head_dim D   64, 128 or 256.
+ *   causal       0: every key of the sequence is visible; 1: key ki is hidden
+ *                from query qi when qi < ki (sequence-local indices).
+ *   scale        softmax scale; a value <= 0 or NaN selects 1/sqrt(D).
+ *   dtype        element type of q, k, v and out.
+ *   out          [total_q, H, D] dtype, written for rows [0, cu_seqlens_q[batch]).
+ *                Rows outside the packed extents are not touched.
+ *   lse          [total_q, H] float32, natural-log log-sum-exp of the scaled
+ *                scores of each row; a query with no visible key (Lk_b = 0)
+ *                gets out = 0 and lse = -inf.
+ *   stream       CUDA stream of the launch (NULL = legacy default stream).
+ *
+ * Returns VARLEN_OK or one of the negative codes above.
+ */
+int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       int batch, int64_t total_q, int64_t total_k,
+                       int max_seqlen_q, int max_seqlen_k,
+                       int num_heads, int num_kv_heads, int head_dim,
+                       int causal, float scale, varlen_dtype_t dtype,
+                       void *out, float *lse, varlen_stream_t stream);
+
+/* Unversioned name of the current stable entry point (same arguments and
+ * behaviour as varlen_attn_fwd_v1). */
+int varlen_attn_fwd(const void *q, const void *k, const void *v,
+                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                    int batch, int64_t total_q, int64_t total_k,
+                    int max_seqlen_q, int max_seqlen_k,
+                    int num_heads, int num_kv_heads, int head_dim,
+                    int causal, float scale, varlen_dtype_t dtype,
+                    void *out, float *lse, varlen_stream_t stream);
+
+/* Static, human-readable description of a status code.  Never NULL. */
+const char *varlen_attn_strerror(int code);
+
+/*
+ * Device-side status word of the current device.  Every wait inside the
+ * kernels is bounded; a wait that runs out (which does not happen in a
+ * correct launch) ORs a bit into this word, the kernel drains its own
+ * in-flight copies and returns instead of hanging.  Bits: 1 = pipeline wait
+ * timed out.  Reads the word synchronously into *status (device-wide,
+ * shared by all launches of this library on the device); clears it when
+ * clear != 0.  Returns VARLEN_OK or VARLEN_ERR_LAUNCH / VARLEN_ERR_NULL.
+ */
+int varlen_attn_device_status(unsigned int *status, int clear);
+
+/* Library ABI version (1 for this header). */
+int varlen_attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VARLEN_ATTN_H_ */

@@ -1,0 +1,93 @@
+"""CPU-only checks of the C-ABI library: it builds for sm_100a, loads, exports
+every symbol the header declares, and rejects invalid arguments on the host
+before touching any device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import flash_attention_fwd_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "varlen_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(varlen_attn_[a-z_0-9]+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_declares_exported_symbols():
+    assert header_functions() == sorted(fa.EXPORTED_SYMBOLS)
+
+
+def test_library_loads_and_exports_every_symbol():
+    lib = fa.load_library()
+    raw = ctypes.CDLL(fa.LIB_PATH)
+    for name in header_functions():
+        assert hasattr(raw, name), name
+    assert lib.varlen_attn_abi_version() == 1
+
+
+def test_library_is_built_for_sm100a():
+    data = open(fa.LIB_PATH, "rb").read()
+    # the fatbin names its target architecture; only sm_100a is built
+    assert b"sm_100a" in data
+
+
+def test_strerror_covers_codes():
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -99):
+        msg = fa.strerror(code)
+        assert isinstance(msg, str) and msg
+
+
+BASE = dict(q_ptr=0x10000, k_ptr=0x20000, v_ptr=0x30000, cu_q_ptr=0x40000, cu_k_ptr=0x50000,
+            batch=2, total_q=10, total_k=10, max_seqlen_q=5, max_seqlen_k=5, num_heads=4,
+            num_kv_heads=2, head_dim=128, causal=True, scale=0.0, dtype_code=0,
+            out_ptr=0x60000, lse_ptr=0x70000, stream=0)
+
+
+@pytest.mark.parametrize("change,code", [
+    (dict(num_heads=5), -2),                 # H % Hkv != 0
+    (dict(head_dim=96), -2),                 # unsupported D
+    (dict(head_dim=32), -2),
+    (dict(batch=-1), -2),
+    (dict(total_q=-3), -2),
+    (dict(total_q=1 << 31), -2),
+    (dict(max_seqlen_k=-1), -2),
+    (dict(num_kv_heads=0), -2),
+    (dict(dtype_code=2), -3),
+    (dict(q_ptr=0), -1),
+    (dict(out_ptr=0), -1),
+    (dict(lse_ptr=0), -1),
+    (dict(k_ptr=0), -1),
+    (dict(cu_q_ptr=0), -1),
+    (dict(q_ptr=0x10008), -4),               # 8-byte aligned only
+    (dict(out_ptr=0x60002), -4),
+    (dict(lse_ptr=0x70002), -4),
+    (dict(cu_k_ptr=0x50001), -4),
+])
+def test_host_validation_rejects(change, code):
+    args = dict(BASE)
+    args.update(change)
+    assert fa.varlen_attn_fwd_raw(**args) == code
+
+
+def test_empty_problems_are_noops_without_device():
+    args = dict(BASE)
+    args.update(batch=0)
+    assert fa.varlen_attn_fwd_raw(**args) == 0
+    args = dict(BASE)
+    args.update(total_q=0, q_ptr=0, out_ptr=0, lse_ptr=0)
+    assert fa.varlen_attn_fwd_raw(**args) == 0
+
+
+def test_product_module_does_not_import_oracle():
+    import sys
+    pkg_dir = os.path.dirname(fa.__file__)
+    for fn in os.listdir(pkg_dir):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg_dir, fn)).read()
+            assert "oracle" not in re.sub(r'""".*?"""', "", src, flags=re.S), fn

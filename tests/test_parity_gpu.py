@@ -1,0 +1,200 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.
+
+Tolerances (bf16/fp16 output against fp64): O max abs err <= 1.5e-2, O mean
+abs err <= 2e-3, LSE max abs err <= 5e-3.  Indexing is checked exactly: the
+output buffers carry guard rows before and after the packed extents, filled
+with a canary, and must come back with every packed row written (no NaN
+pre-fill left) and every guard row untouched.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+O_MAX, O_MEAN, LSE_MAX = 1.5e-2, 2e-3, 5e-3
+GUARD = 3
+
+
+def run_gpu(case, scale=None, guard=GUARD, max_q=None, max_k=None):
+    """Runs the CUDA forward with NaN-filled outputs inside guard rows.
+    Returns (out float64 [Tq,H,D], lse float64 [Tq,H], raw out, raw lse)."""
+    import flash_attention_fwd_b200 as fa
+    dev = torch.device("cuda", 0)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    cq, ck = case.cu_q.to(dev), case.cu_k.to(dev)
+    Tq, H, D = case.q.shape
+    tdt = case.q.dtype
+    out_buf = torch.full((Tq + 2 * guard, H, D), float("nan"), dtype=tdt, device=dev)
+    lse_buf = torch.full((Tq + 2 * guard, H), float("nan"), dtype=torch.float32, device=dev)
+    canary = torch.tensor(-12345.0, dtype=tdt)
+    out_buf[:guard] = canary
+    out_buf[guard + Tq:] = canary
+    lse_buf[:guard] = -777.0
+    lse_buf[guard + Tq:] = -777.0
+    out = out_buf[guard:guard + Tq]
+    lse = lse_buf[guard:guard + Tq]
+    fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q if max_q is None else max_q,
+                       case.max_k if max_k is None else max_k, case.causal,
+                       scale if scale is not None else case.scale, out=out, lse=lse)
+    torch.cuda.synchronize()
+    ob, lb = out_buf.cpu(), lse_buf.cpu()
+    assert torch.all(ob[:guard] == canary) and torch.all(ob[guard + Tq:] == canary), "guard rows of out written"
+    assert torch.all(lb[:guard] == -777.0) and torch.all(lb[guard + Tq:] == -777.0), "guard rows of lse written"
+    return (ob[guard:guard + Tq].to(torch.float64).numpy(), lb[guard:guard + Tq].to(torch.float64).numpy(),
+            ob[guard:guard + Tq], lb[guard:guard + Tq])
+
+
+def check_close(out, lse, ref_out, ref_lse, what=""):
+    assert not np.isnan(out).any(), "%s: NaN left in out (row not written)" % what
+    assert not np.isnan(lse).any(), "%s: NaN left in lse (row not written)" % what
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(np.isfinite(lse), fin), "%s: -inf pattern of lse differs" % what
+    err = np.abs(out - ref_out)
+    assert err.max() <= O_MAX, "%s: O max abs err %.3e" % (what, err.max())
+    assert err.mean() <= O_MEAN, "%s: O mean abs err %.3e" % (what, err.mean())
+    if fin.any():
+        lerr = np.abs(lse[fin] - ref_lse[fin]).max()
+        assert lerr <= LSE_MAX, "%s: LSE max abs err %.3e" % (what, lerr)
+
+
+def full_check(case, **kw):
+    out, lse, _, _ = run_gpu(case, **kw)
+    ref_out, ref_lse = oracle.run_case(case)
+    check_close(out, lse, ref_out, ref_lse, case.name)
+    return out, lse
+
+
+def sampled_check(case, n=2000, seed=7, **kw):
+    out, lse, _, _ = run_gpu(case, **kw)
+    assert not np.isnan(out).any() and not np.isnan(lse).any(), "a packed row was not written"
+    rows = workloads.sample_rows(case, n, seed=seed)
+    ref_out, ref_lse = oracle.run_case_rows(case, rows)
+    check_close(out[rows[:, 0], rows[:, 1]], lse[rows[:, 0], rows[:, 1]], ref_out, ref_lse,
+                case.name)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _require_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import flash_attention_fwd_b200 as fa
+    fa.load_library()
+    fa.device_status(clear=True)
+    yield
+    assert fa.device_status(clear=True) == 0, "a bounded pipeline wait timed out on the device"
+
+
+# --- the benchmark configurations ----------------------------------------------------
+
+def test_tiny_full():
+    full_check(workloads.make_workload("tiny"))
+
+
+def test_gqa_prefill_full():
+    full_check(workloads.make_workload("gqa"))
+
+
+def test_long_ragged_sampled():
+    sampled_check(workloads.make_workload("long"), n=600)
+
+
+def test_short_query_long_kv_sampled():
+    sampled_check(workloads.make_workload("shortq"), n=1500)
+
+
+def test_wide_head_fp16_sampled():
+    sampled_check(workloads.make_workload("wide"), n=1000)
+
+
+# --- several tiles plus ragged tails, every head dim and dtype ------------------------
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ragged_tiles(D, dtype, causal):
+    lens = [300, 1, 129, 128, 77, 513]
+    case = workloads.make_case(lens, None, 4, 2, D, dtype, causal, seed=D + len(dtype) + causal)
+    full_check(case)
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_q_and_k_lengths_differ(D):
+    # causal with Lq != Lk uses the top-left (sequence-local) rule
+    case = workloads.make_case([70, 200, 5, 131], [250, 64, 1, 300], 6, 3, D, "bf16", True,
+                               seed=40 + D)
+    full_check(case)
+    case2 = workloads.make_case([70, 200, 5, 131], [250, 64, 1, 300], 6, 3, D, "bf16", False,
+                                seed=41 + D)
+    full_check(case2)
+
+
+def test_empty_sequences_and_empty_keys():
+    # Lq=0 sequences write nothing; Lk=0 sequences give O = 0, LSE = -inf
+    case = workloads.make_case([0, 50, 3, 0, 140], [10, 0, 7, 0, 140], 4, 4, 128, "bf16", False,
+                               seed=50)
+    out, lse = full_check(case)
+    cu = case.cu_q.tolist()
+    assert np.all(out[cu[1]:cu[2]] == 0.0) and np.all(np.isneginf(lse[cu[1]:cu[2]]))
+
+
+def test_single_kv_head_and_many_sequences():
+    rng = np.random.default_rng(60)
+    lens = [int(x) for x in rng.integers(1, 300, 97)]
+    case = workloads.make_case(lens, None, 16, 1, 128, "bf16", True, seed=60)
+    full_check(case)
+
+
+def test_explicit_scale_and_default_scale():
+    case = workloads.make_case([200, 31], None, 4, 4, 64, "bf16", True, seed=61, scale=0.05)
+    full_check(case)
+    case.scale = 1.0 / math.sqrt(64)
+    out_a, lse_a, _, _ = run_gpu(case, scale=0.0)
+    out_b, lse_b, _, _ = run_gpu(case, scale=1.0 / math.sqrt(64))
+    assert np.array_equal(out_a, out_b) and np.array_equal(lse_a, lse_b)
+
+
+def test_understated_max_seqlen_still_covers_all_rows():
+    case = workloads.make_case([700, 20], None, 2, 2, 128, "bf16", True, seed=62)
+    out, lse, _, _ = run_gpu(case, max_q=1, max_k=1)
+    ref_out, ref_lse = oracle.run_case(case)
+    check_close(out, lse, ref_out, ref_lse, "understated max_seqlen")
+
+
+def test_deterministic():
+    case = workloads.make_workload("gqa")
+    _, _, o1, l1 = run_gpu(case)
+    _, _, o2, l2 = run_gpu(case)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(l1, l2)
+
+
+def test_large_logit_stability_fp16():
+    case = workloads.make_case([1024, 333], None, 4, 4, 256, "fp16", True, seed=63,
+                               sigma_q=3.0, sigma_k=3.0)
+    out, lse = full_check(case)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_running_max_growth_rescales(D):
+    """Scores that grow along the key axis force many in-place rescales of O."""
+    case = workloads.make_case([900, 300], None, 4, 2, D, "bf16", True, seed=70 + D,
+                               sigma_q=2.0, sigma_k=2.0)
+    Tk = case.k.shape[0]
+    ramp = (1.0 + torch.arange(Tk, dtype=torch.float32) / 150.0).view(Tk, 1, 1)
+    case.k = (case.k.float() * ramp).to(case.k.dtype)
+    full_check(case)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_large_logits_bf16(D):
+    case = workloads.make_case([700, 129, 64], None, 8, 2, D, "bf16", True, seed=80 + D,
+                               sigma_q=3.0, sigma_k=3.0)
+    full_check(case)

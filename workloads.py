@@ -63,6 +63,12 @@ WORKLOADS = {
                                    "H=32, Hkv=4, D=128, bf16, non-causal"),
     "wide": Workload("wide", 5, 16, 16, 256, "fp16", True, sigma_q=3.0, sigma_k=3.0, sigma_v=1.0,
                      description="wide-head MHA: 4x4096, H=Hkv=16, D=256, fp16, Q/K sigma 3, causal"),
+    # Profiling case only (not a benchmark configuration): the long ragged
+    # prefill lengths with a quarter of its heads, so that a many-pass profiler
+    # capture stays small while its inputs still exceed the L2 cache.
+    "long_h16": Workload("long_h16", 3, 16, 2, 128, "bf16", True,
+                         description="profiling case: long ragged prefill lengths, H=16, Hkv=2, "
+                                     "D=128, bf16, causal"),
 }
 
 
@@ -92,7 +98,7 @@ def seqlens(name: str):
         rng = np.random.default_rng(w.seed)
         q = [int(x) for x in rng.integers(128, 2049, 8)]
         return q, list(q)
-    if name == "long":
+    if name in ("long", "long_h16"):
         q = _long_lengths(w.seed)
         return q, list(q)
     if name == "shortq":
