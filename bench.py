@@ -37,6 +37,9 @@ METRIC = "varlen attn fwd TFLOP/s (unmasked FLOPs) and % of B200 dense bf16 peak
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["flash_attention_fwd_b200/csrc/varlen_attn_fwd.cu",
+                  "flash_attention_fwd_b200/csrc/fwd_common.cuh",
+                  "flash_attention_fwd_b200/csrc/fwd_pair.cuh",
+                  "flash_attention_fwd_b200/csrc/fwd_single.cuh",
                   "flash_attention_fwd_b200/csrc/sm100_ptx.cuh"]
 
 

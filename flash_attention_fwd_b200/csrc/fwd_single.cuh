@@ -1,0 +1,326 @@
+/*
+ * fwd_single.cuh — attention forward, one 128-row query tile per work item.
+ *
+ * Used for head dim 256 (TMEM holds one tile's O of 256 columns plus two S
+ * buffers of 64 key columns) and for head layouts without query-head pairs
+ * sharing a key/value head (H / Hkv odd, e.g. plain multi-head attention).
+ *
+ * One persistent CTA per SM, 192 threads:
+ *   warps 0-3  softmax warpgroup (thread t = query row t = TMEM lane t)
+ *   warp 4     TMA producer: Q tile, K/V tiles through a shared-memory ring
+ *   warp 5     TMEM owner and MMA issuer
+ * S is double-buffered in TMEM so that S(j+1) = Q K(j+1)^T runs on the tensor
+ * cores while the softmax warps work on S(j); the MMA order per key tile is
+ * S(0), S(1), then PV(j), S(j+2) for j = 0, 1, ...
+ */
+#pragma once
+#include "fwd_common.cuh"
+
+namespace vattn {
+namespace single {
+
+constexpr int NUM_THREADS = 192;
+constexpr int PRODUCER_WARP = 4;
+constexpr int MMA_WARP = 5;
+
+template <int D>
+struct Cfg;
+// BN = keys per tile, NSLOT = K/V shared-memory ring depth.
+template <>
+struct Cfg<64> {
+  static constexpr int BN = 128, NSLOT = 8;
+};
+template <>
+struct Cfg<128> {
+  static constexpr int BN = 128, NSLOT = 6;
+};
+template <>
+struct Cfg<256> {
+  static constexpr int BN = 64, NSLOT = 4;
+};
+
+struct Barriers {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t q_full, q_empty;
+  uint64_t s_full[2], p_full[2];
+  uint64_t pv_done, o_ready, o_free, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int D>
+constexpr size_t smem_bytes() {
+  return (size_t)BM * D * 2 + (size_t)Cfg<D>::NSLOT * Cfg<D>::BN * D * 2 + sizeof(Barriers) +
+         1024;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const KParams p) {
+  constexpr int BN = Cfg<D>::BN;
+  constexpr int NSLOT = Cfg<D>::NSLOT;
+  constexpr int DB = D / 64;  // 128-byte swizzle blocks along D
+  constexpr uint32_t Q_BYTES = BM * D * 2;
+  constexpr uint32_t KV_BYTES = BN * D * 2;
+  // TMEM columns: S buffer b at [b*BN, (b+1)*BN), P aliases its first BN/2
+  // columns, O accumulator at [2*BN, 2*BN + D).
+  constexpr uint32_t O_COL = 2 * BN;
+  static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
+  constexpr uint32_t IDESC_S = ptx::idesc_f16(BM, BN, BF16, false);
+  constexpr uint32_t IDESC_PV = ptx::idesc_f16(BM, D, BF16, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = smem;
+  uint8_t *sKV = smem + Q_BYTES;
+  Barriers *bars = reinterpret_cast<Barriers *>(sKV + NSLOT * KV_BYTES);
+  volatile int *abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSLOT; ++s) {
+      ptx::mbar_init(&bars->full[s], 1);
+      ptx::mbar_init(&bars->empty[s], 1);
+    }
+    ptx::mbar_init(&bars->q_full, 1);
+    ptx::mbar_init(&bars->q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars->s_full[i], 1);
+      ptx::mbar_init(&bars->p_full[i], 4);
+    }
+    ptx::mbar_init(&bars->pv_done, 1);
+    ptx::mbar_init(&bars->o_ready, 1);
+    ptx::mbar_init(&bars->o_free, 4);
+    ptx::mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    ptx::mbar_init_fence();
+  }
+  if (warp == PRODUCER_WARP && lane == 0) {
+    ptx::tma_prefetch_desc(&tm_q);
+    ptx::tma_prefetch_desc(&tm_k);
+    ptx::tma_prefetch_desc(&tm_v);
+  }
+  if (warp == MMA_WARP) {
+    ptx::tmem_alloc(&bars->tmem_base, TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      Scheduler<BN> sched;
+      sched.init(p);
+      WorkItem w;
+      uint32_t slot = 0, phase = 0, q_count = 0;
+      uint32_t slot_fills[NSLOT];
+      for (int s = 0; s < NSLOT; ++s) slot_fills[s] = 0;
+      bool ok = true;
+      const uint64_t pol_kv = ptx::policy_evict_last();
+      auto load_kv = [&](const CUtensorMap *tm, int kv_h, int row) -> bool {
+        if (!wait_bar(&bars->empty[slot], phase ^ 1u, abort_flag)) return false;
+        uint8_t *dst = sKV + slot * KV_BYTES;
+        ptx::mbar_arrive_expect_tx(&bars->full[slot], KV_BYTES);
+#pragma unroll
+        for (int db = 0; db < DB; ++db)
+          ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &bars->full[slot], db * 64, kv_h, row,
+                                pol_kv);
+        ++slot_fills[slot];
+        if (++slot == NSLOT) {
+          slot = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
+      // Ring order per item: K0, K1, V0, K2, V1, K3, ..., V(n-1) — the order
+      // in which the MMA warp consumes them.
+      while (ok && sched.next(w)) {
+        const int n = w.n_kv;
+        if (n == 0) continue;
+        const int kv_h = w.hu / p.group;
+        ok = load_kv(&tm_k, kv_h, w.k0);
+        if (!ok) break;
+        if (!wait_bar(&bars->q_empty, (q_count & 1u) ^ 1u, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(&bars->q_full, Q_BYTES);
+#pragma unroll
+        for (int db = 0; db < DB; ++db)
+          ptx::tma_load_3d(sQ + db * (BM * 128), &tm_q, &bars->q_full, db * 64, w.hu, w.q0);
+        ++q_count;
+        if (n >= 2) ok = load_kv(&tm_k, kv_h, w.k0 + BN);
+        for (int j = 0; ok && j < n; ++j) {
+          ok = load_kv(&tm_v, kv_h, w.k0 + j * BN);
+          if (ok && j + 2 < n) ok = load_kv(&tm_k, kv_h, w.k0 + (j + 2) * BN);
+        }
+      }
+      // Drain: every copy this thread issued has landed before the CTA exits.
+      for (int s = 0; s < NSLOT; ++s)
+        if (slot_fills[s] > 0) wait_bar(&bars->full[s], (slot_fills[s] - 1) & 1u, abort_flag);
+      if (q_count > 0) wait_bar(&bars->q_full, (q_count - 1) & 1u, abort_flag);
+    }
+  } else if (warp == MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      Scheduler<BN> sched;
+      sched.init(p);
+      WorkItem w;
+      uint32_t slot = 0, phase = 0, g = 0, items = 0;
+      bool ok = true;
+      const uint32_t sQ_addr = ptx::smem_u32(sQ);
+      const uint32_t sKV_addr = ptx::smem_u32(sKV);
+      auto take_slot = [&](uint32_t &s_out) -> bool {
+        s_out = slot;
+        if (!wait_bar(&bars->full[slot], phase, abort_flag)) return false;
+        ptx::tc_fence_after();
+        if (++slot == NSLOT) {
+          slot = 0;
+          phase ^= 1u;
+        }
+        return true;
+      };
+      // S[buf] = Q K^T over D in steps of 16 (K-major A and B, 128B swizzle)
+      auto issue_s = [&](uint32_t buf, uint32_t kslot) {
+        const uint32_t kbase = sKV_addr + kslot * KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk % 4) * 32u;  // 16 elements = 32 bytes inside a swizzle row
+          uint64_t a = ptx::sdesc_sw128(sQ_addr + (kk / 4) * (BM * 128) + off, 16, 1024);
+          uint64_t bdesc = ptx::sdesc_sw128(kbase + (kk / 4) * (BN * 128) + off, 16, 1024);
+          ptx::mma_ss(tmem + buf * BN, a, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O += P V over the BN keys in steps of 16 (P from TMEM, V MN-major)
+      auto issue_pv = [&](uint32_t buf, uint32_t vslot, bool acc) {
+        const uint32_t vbase = sKV_addr + vslot * KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
+          ptx::mma_ts(tmem + O_COL, tmem + buf * BN + kk * 8, bdesc, IDESC_PV,
+                      (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      while (ok && sched.next(w)) {
+        const int n = w.n_kv;
+        if (n == 0) continue;
+        if (!wait_bar(&bars->q_full, items & 1u, abort_flag)) break;
+        ptx::tc_fence_after();
+        for (int jj = 0; ok && jj < 2 && jj < n; ++jj) {
+          uint32_t ks;
+          if (!(ok = take_slot(ks))) break;
+          const uint32_t buf = (g + jj) & 1u;
+          issue_s(buf, ks);
+          ptx::mma_commit(&bars->s_full[buf]);
+          ptx::mma_commit(&bars->empty[ks]);
+          if (jj == n - 1) ptx::mma_commit(&bars->q_empty);
+        }
+        for (int j = 0; ok && j < n; ++j) {
+          const uint32_t gj = g + j;
+          const uint32_t buf = gj & 1u;
+          if (!(ok = wait_bar(&bars->p_full[buf], (gj >> 1) & 1u, abort_flag))) break;
+          ptx::tc_fence_after();
+          if (j == 0 && items > 0) {
+            if (!(ok = wait_bar(&bars->o_free, (items - 1) & 1u, abort_flag))) break;
+            ptx::tc_fence_after();
+          }
+          uint32_t vs;
+          if (!(ok = take_slot(vs))) break;
+          issue_pv(buf, vs, j > 0);
+          ptx::mma_commit(&bars->empty[vs]);
+          ptx::mma_commit(&bars->pv_done);
+          if (j == n - 1) ptx::mma_commit(&bars->o_ready);
+          if (j + 2 < n) {
+            uint32_t ks;
+            if (!(ok = take_slot(ks))) break;
+            issue_s(buf, ks);
+            ptx::mma_commit(&bars->s_full[buf]);
+            ptx::mma_commit(&bars->empty[ks]);
+            if (j + 2 == n - 1) ptx::mma_commit(&bars->q_empty);
+          }
+        }
+        g += n;
+        ++items;
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      ptx::mma_commit(&bars->drain);
+      wait_bar(&bars->drain, 0, abort_flag);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax WG
+    const int r = threadIdx.x;  // row in the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t tS0 = tmem + lane_base;
+    const uint32_t tO = tmem + lane_base + O_COL;
+    const float sl2 = p.scale_log2;
+    Scheduler<BN> sched;
+    sched.init(p);
+    WorkItem w;
+    uint32_t g = 0, items = 0;
+    bool ok = true;
+    while (ok && sched.next(w)) {
+      const int n = w.n_kv;
+      const int qi = w.qi0 + r;
+      const bool row_valid = r < w.q_rows;
+      const size_t orow = (size_t)(w.q0 + r) * p.H + w.hu;  // row index into [total_q, H]
+      uint16_t *orow_ptr = reinterpret_cast<uint16_t *>(p.out) + orow * D;
+      if (n == 0) {
+        if (row_valid) empty_row<D>(orow_ptr, p.lse + orow);
+        continue;
+      }
+      const int key_lim = p.causal ? min(w.Lk, qi + 1) : w.Lk;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t gj = g + j;
+        const uint32_t buf = gj & 1u;
+        bool got = wait_bar(&bars->s_full[buf], (gj >> 1) & 1u, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        // O must hold PV(gj-1) before it is rescaled in place.  The wait by
+        // parity is exact: S(gj) completing implies PV(gj-2) did, and PV(gj)
+        // cannot be issued before this iteration's P, so the barrier is in
+        // phase gj-1 or gj.
+        auto wait_o = [&]() { return wait_bar(&bars->pv_done, (gj - 1) & 1u, abort_flag); };
+        if (!softmax_tile<BN, D, BF16>(tS0 + buf * BN, tO, j, sl2, (j + 1) * BN > w.min_lim,
+                                       key_lim - j * BN, m, l, wait_o)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->p_full[buf]);
+      }
+      if (!ok) break;
+      g += n;
+      // o_ready completes once per item, after the item's last PV; the next
+      // item's first PV waits for o_free, so it is never a phase ahead.
+      bool got = wait_bar(&bars->o_ready, items & 1u, abort_flag);
+      ++items;
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      epilogue_row<D, BF16>(tO, m, l, row_valid, orow_ptr, p.lse + orow, &bars->o_free, lane);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == MMA_WARP) {
+    __syncwarp();
+    ptx::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace single
+}  // namespace vattn
