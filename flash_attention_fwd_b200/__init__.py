@@ -71,17 +71,21 @@ def _bind(lib):
 
 
 def load_library(build_if_missing: bool = True):
-    """Load (building first if it is missing or stale) the CUDA library."""
+    """Load (building first if it is missing or stale) the CUDA library.
+
+    The environment variable VARLEN_ATTN_LIB may name another build of the
+    same library (same ABI) to load instead."""
     global _lib
     with _lock:
         if _lib is None:
-            if build_if_missing:
+            path = os.environ.get("VARLEN_ATTN_LIB") or LIB_PATH
+            if path == LIB_PATH and build_if_missing:
                 from . import build as _build
                 _build.build()
-            if not os.path.exists(LIB_PATH):
+            if not os.path.exists(path):
                 raise RuntimeError("CUDA extension %s is missing; run "
-                                   "`python -m flash_attention_fwd_b200.build`" % LIB_PATH)
-            _lib = _bind(ctypes.CDLL(LIB_PATH))
+                                   "`python -m flash_attention_fwd_b200.build`" % path)
+            _lib = _bind(ctypes.CDLL(path))
     return _lib
 
 

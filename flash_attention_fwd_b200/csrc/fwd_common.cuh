@@ -54,19 +54,76 @@ struct WorkItem {
   int min_lim;  // smallest per-row visible-key bound in the tile
 };
 
-// Walks the work list (sequence ascending, query tile descending, head unit
-// ascending) and deals item idx to CTA round-robin with the direction
-// reversed every round.  Every role of a CTA runs its own copy and sees the
-// same sequence of items.  Lengths are clamped into the buffers' extents so
-// that an inconsistent sequence table cannot address memory outside them.
+// ---------------------------------------------------------------------------
+// Work scheduler.  A work item is (sequence b, query tile qt of BM rows, head
+// unit hu).  Its cost is measured in 128-key tiles: with the causal rule a
+// query tile needs the keys [0, min(Lk, min(Lq, (qt+1) * BM))), i.e.
+// min(nk, qt + 1) tiles where nk = ceil(Lk / BM); without it, nk tiles.  Items
+// are listed by cost level, highest first ("longest processing time first"),
+// and within a level by sequence, query tile, head unit (the head units that
+// share K/V tiles are adjacent, so they run at the same time on neighbouring
+// CTAs and the K/V tiles are served from L2).  Item i goes to CTA i mod G, the
+// direction reversed every round, so each CTA gets a near-equal sum of costs.
+//
+// The walk is warp-cooperative (all 32 lanes of the calling warp call
+// init/next together): sequences are examined 32 at a time.  Lengths are
+// clamped into the buffers' extents, so an inconsistent sequence table can
+// never address memory outside them.
 template <int BN>
 struct Scheduler {
   const int *cu_q, *cu_k;
   int B, HU, causal, total_q, total_k;
-  int cta, grid, round;
-  int b;
-  long long base;
-  int q_start, q_len, k_start, k_len, nq;
+  int cta, grid, lane;
+  long long round;
+  int level;              // current cost level; -1 once the list is exhausted
+  long long level_base;   // index of the first item of the level
+  long long level_items;  // items in the level
+  int cur_b;              // cursor inside the level: first sequence not passed yet
+  long long cur_units;    // (sequence, query tile) units before cur_b in this level
+
+  __device__ void extents(int b, int &qs, int &lq, int &ks, int &lk) const {
+    qs = __ldg(cu_q + b);
+    int qe = __ldg(cu_q + b + 1);
+    ks = __ldg(cu_k + b);
+    int ke = __ldg(cu_k + b + 1);
+    qs = min(max(qs, 0), total_q);
+    qe = min(max(qe, qs), total_q);
+    ks = min(max(ks, 0), total_k);
+    ke = min(max(ke, ks), total_k);
+    lq = qe - qs;
+    lk = ke - ks;
+  }
+  // (sequence, query tile) units of a sequence at cost level c
+  __device__ int units_at(int nq, int nk, int c) const {
+    if (!causal || nk == 0) return (c == nk) ? nq : 0;
+    if (c >= 1 && c < nk) return (c <= nq) ? 1 : 0;
+    if (c == nk) return (nq >= nk) ? nq - nk + 1 : 0;
+    return 0;
+  }
+  // query tile of the k-th unit of a sequence at level c
+  __device__ int tile_of(int nk, int c, int k) const {
+    if (causal && nk > 0) return (c < nk) ? c - 1 : nk - 1 + k;
+    return k;
+  }
+  __device__ int top_level(int nq, int nk) const {
+    if (nq == 0) return -1;
+    return (causal && nk > 0) ? min(nk, nq) : nk;
+  }
+  __device__ long long count_level(int c) const {
+    long long u = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      int b = b0 + lane, v = 0;
+      if (b < B) {
+        int qs, lq, ks, lk;
+        extents(b, qs, lq, ks, lk);
+        v = units_at((lq + BM - 1) / BM, (lk + BM - 1) / BM, c);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      u += v;
+    }
+    return u * HU;
+  }
 
   __device__ void init(const KParams &p) {
     cu_q = p.cu_q;
@@ -78,48 +135,91 @@ struct Scheduler {
     total_k = p.total_k;
     cta = blockIdx.x;
     grid = gridDim.x;
+    lane = threadIdx.x & 31;
     round = 0;
-    b = 0;
-    base = 0;
-    if (B > 0) load(0);
-  }
-
-  __device__ void load(int bb) {
-    int qs = __ldg(cu_q + bb), qe = __ldg(cu_q + bb + 1);
-    int ks = __ldg(cu_k + bb), ke = __ldg(cu_k + bb + 1);
-    qs = min(max(qs, 0), total_q);
-    qe = min(max(qe, qs), total_q);
-    ks = min(max(ks, 0), total_k);
-    ke = min(max(ke, ks), total_k);
-    q_start = qs;
-    q_len = qe - qs;
-    k_start = ks;
-    k_len = ke - ks;
-    nq = (q_len + BM - 1) / BM;
+    int top = -1;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      int b = b0 + lane;
+      if (b < B) {
+        int qs, lq, ks, lk;
+        extents(b, qs, lq, ks, lk);
+        top = max(top, top_level((lq + BM - 1) / BM, (lk + BM - 1) / BM));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) top = max(top, __shfl_xor_sync(0xffffffffu, top, o));
+    level = top;
+    level_base = 0;
+    level_items = (level >= 0) ? count_level(level) : 0;
+    cur_b = 0;
+    cur_units = 0;
   }
 
   __device__ bool next(WorkItem &w) {
-    long long idx = (long long)round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
+    const long long idx = round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
     ++round;
-    while (b < B && idx >= base + (long long)nq * HU) {
-      base += (long long)nq * HU;
-      ++b;
-      if (b < B) load(b);
+    while (level >= 0 && idx >= level_base + level_items) {
+      level_base += level_items;
+      --level;
+      if (level >= 0) {
+        level_items = count_level(level);
+        cur_b = 0;
+        cur_units = 0;
+      }
     }
-    if (b >= B) return false;
-    long long local = idx - base;
-    int qt = nq - 1 - (int)(local / HU);
+    if (level < 0) return false;
+    const long long local = idx - level_base;
+    const long long unit = local / HU;
     w.hu = (int)(local % HU);
-    w.qi0 = qt * BM;
-    w.q0 = q_start + w.qi0;
-    w.q_rows = min(BM, q_len - w.qi0);
-    w.k0 = k_start;
-    w.Lk = k_len;
-    int kv_end = causal ? min(k_len, min(q_len, w.qi0 + BM)) : k_len;
-    w.n_kv = (kv_end + BN - 1) / BN;
-    w.min_lim = causal ? min(k_len, w.qi0 + 1) : k_len;
-    return true;
+    for (;;) {
+      const int b = cur_b + lane;
+      int qs = 0, lq = 0, ks = 0, lk = 0, u = 0;
+      if (b < B) {
+        extents(b, qs, lq, ks, lk);
+        u = units_at((lq + BM - 1) / BM, (lk + BM - 1) / BM, level);
+      }
+      int incl = u;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (cur_units + total > unit) {
+        const unsigned hit = __ballot_sync(0xffffffffu, cur_units + incl > unit);
+        const int src = __ffs(hit) - 1;
+        const int before = __shfl_sync(0xffffffffu, incl - u, src);
+        qs = __shfl_sync(0xffffffffu, qs, src);
+        lq = __shfl_sync(0xffffffffu, lq, src);
+        ks = __shfl_sync(0xffffffffu, ks, src);
+        lk = __shfl_sync(0xffffffffu, lk, src);
+        cur_b += src;
+        cur_units += before;
+        const int k = (int)(unit - cur_units);
+        const int qt = tile_of((lk + BM - 1) / BM, level, k);
+        w.qi0 = qt * BM;
+        w.q0 = qs + w.qi0;
+        w.q_rows = min(BM, lq - w.qi0);
+        w.k0 = ks;
+        w.Lk = lk;
+        const int kv_end = causal ? min(lk, min(lq, w.qi0 + BM)) : lk;
+        w.n_kv = (kv_end + BN - 1) / BN;
+        w.min_lim = causal ? min(lk, w.qi0 + 1) : lk;
+        return true;
+      }
+      cur_b += 32;
+      cur_units += total;
+    }
   }
+};
+
+// Work items travel from the scheduling (producer) warp to the other roles
+// through a small ring in shared memory.  An item with hu < 0 ends the list.
+constexpr int ITEM_RING = 4;
+struct ItemRing {
+  WorkItem items[ITEM_RING];
+  uint64_t full[ITEM_RING];
+  uint64_t empty[ITEM_RING];
 };
 
 // Bounded wait; on timeout raises the CTA abort flag and the device status.
@@ -177,6 +277,51 @@ __device__ __forceinline__ void tmem_st<64>(uint32_t taddr, const uint32_t (&r)[
 }
 
 // ---------------------------------------------------------------------------
+// Software 2^x for the two lanes of a packed pair, used for a share of the
+// softmax exponentials so that the MUFU pipe is not the only unit computing
+// them.  Range reduction in the manner of Cody and Waite: x = n + f with
+// n = rint(x) (adding 1.5 * 2^23 rounds to the nearest integer) and
+// f in [-1/2, 1/2]; 2^f from a polynomial whose coefficients were fitted by a
+// Remez exchange on the relative error over [-1/2, 1/2] (degree 3: max
+// relative error 7.5e-5, below half a bf16 ulp; degree 4: 2.6e-6, below half
+// an fp16 ulp); 2^n is then added into the exponent field.  Inputs are
+// clamped below at -126 so that the exponent stays in range; the result there
+// (about 1e-38) stands in for exp of a masked (-inf) score.
+template <int DEG>
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  ptx::f2_unpack(x2, x0, x1);
+  const uint64_t x = ptx::f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t magic = ptx::f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = ptx::f2_add(x, magic);
+  const uint64_t f = ptx::f2_sub(x, ptx::f2_sub(t, magic));
+  uint64_t p;
+  if constexpr (DEG == 3) {
+    p = ptx::f2_fma(f, ptx::f2_pack(0.0551716685295105f, 0.0551716685295105f),
+                    ptx::f2_pack(0.2426111251115799f, 0.2426111251115799f));
+    p = ptx::f2_fma(p, f, ptx::f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    p = ptx::f2_fma(p, f, ptx::f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  } else {
+    p = ptx::f2_fma(f, ptx::f2_pack(0.009570102207362652f, 0.009570102207362652f),
+                    ptx::f2_pack(0.05591785907745361f, 0.05591785907745361f));
+    p = ptx::f2_fma(p, f, ptx::f2_pack(0.240247443318367f, 0.240247443318367f));
+    p = ptx::f2_fma(p, f, ptx::f2_pack(0.6931217908859253f, 0.6931217908859253f));
+    p = ptx::f2_fma(p, f, ptx::f2_pack(0.9999992847442627f, 0.9999992847442627f));
+  }
+  uint32_t t0 = (uint32_t)t, t1 = (uint32_t)(t >> 32);
+  uint32_t p0 = (uint32_t)p, p1 = (uint32_t)(p >> 32);
+  p0 += t0 << 23;  // the low bits of t hold n (two's complement)
+  p1 += t1 << 23;
+  return (uint64_t)p0 | ((uint64_t)p1 << 32);
+}
+
+// Share of the exponential pairs computed by exp2_poly2: one pair in every
+// SOFTMAX_POLY_EVERY (0 = all on the MUFU).
+#ifndef SOFTMAX_POLY_EVERY
+#define SOFTMAX_POLY_EVERY 0
+#endif
+
+// ---------------------------------------------------------------------------
 // Softmax of one S tile held in TMEM (one row per thread), written back as P
 // (bf16/fp16) over the first BN/2 columns of the same TMEM region.
 //
@@ -187,11 +332,15 @@ __device__ __forceinline__ void tmem_st<64>(uint32_t taddr, const uint32_t (&r)[
 // called by the whole warp and must guarantee that no PV MMA into O is in
 // flight.  P is written in 32-column chunks and O is rescaled after P, so
 // that the full S row, the packed P and an O chunk are never live together.
+// The row sum adds the rounded P values (what the PV MMA sees), so the
+// numerator and the denominator of O / l carry the same rounding.
 // Returns false when that wait gave up.
 template <int BN, int D, bool BF16, class WaitO>
 __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, float sl2,
                                              bool need_mask, int lim, float &m, float &l,
                                              WaitO &&wait_o) {
+  constexpr int POLY = SOFTMAX_POLY_EVERY;
+  constexpr int DEG = BF16 ? 3 : 4;
   uint32_t sr[BN];
   tmem_ld_wait<BN>(tS, sr);
   float s[BN];
@@ -202,15 +351,18 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, fl
     for (int c = 0; c < BN; ++c)
       if (c >= lim) s[c] = -INFINITY;
   }
+  // Row max: four independent chains of three-input maxima.
   float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-  for (int c = 4; c < BN; c += 4) {
-    mx0 = fmaxf(mx0, s[c]);
-    mx1 = fmaxf(mx1, s[c + 1]);
-    mx2 = fmaxf(mx2, s[c + 2]);
-    mx3 = fmaxf(mx3, s[c + 3]);
+  for (int c = 4; c + 8 <= BN; c += 8) {
+    mx0 = ptx::fmax3(mx0, s[c], s[c + 1]);
+    mx1 = ptx::fmax3(mx1, s[c + 2], s[c + 3]);
+    mx2 = ptx::fmax3(mx2, s[c + 4], s[c + 5]);
+    mx3 = ptx::fmax3(mx3, s[c + 6], s[c + 7]);
   }
-  const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+  mx0 = ptx::fmax3(mx0, s[BN - 4], s[BN - 3]);
+  mx1 = ptx::fmax3(mx1, s[BN - 2], s[BN - 1]);
+  const float mx = fmaxf(ptx::fmax3(mx0, mx1, mx2), mx3) * sl2;
   float alpha = 1.f;
   bool need = false;
   if (j == 0) {
@@ -220,39 +372,53 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, fl
     m = mx;
     need = true;
   }
-  const float neg_m = -m;
-  float sum0 = 0.f, sum1 = 0.f;
+  const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+  const uint64_t negm_2 = ptx::f2_pack(-m, -m);
+  float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
 #pragma unroll
   for (int c0 = 0; c0 < BN; c0 += 32) {
     uint32_t pk[16];
 #pragma unroll
-    for (int c = 0; c < 32; c += 2) {
-      const float p0 = ptx::ex2_approx(fmaf(s[c0 + c], sl2, neg_m));
-      const float p1 = ptx::ex2_approx(fmaf(s[c0 + c + 1], sl2, neg_m));
-      const uint32_t pp = pack2<BF16>(p0, p1);
-      pk[c / 2] = pp;
-      if constexpr (BF16) {
-        // Sum the values the PV MMA actually sees (bf16-rounded), so the
-        // numerator and the denominator of O / l carry the same rounding.
-        sum0 += __uint_as_float(pp << 16);
-        sum1 += __uint_as_float(pp & 0xFFFF0000u);
+    for (int i = 0; i < 16; ++i) {
+      const int c = c0 + 2 * i;
+      const uint64_t x2 = ptx::f2_fma(ptx::f2_pack(s[c], s[c + 1]), sl2_2, negm_2);
+      float p0, p1;
+      if (POLY > 0 && (i % (POLY > 0 ? POLY : 1)) == POLY - 1) {
+        ptx::f2_unpack(exp2_poly2<DEG>(x2), p0, p1);
       } else {
-        sum0 += p0;
-        sum1 += p1;
+        float x0, x1;
+        ptx::f2_unpack(x2, x0, x1);
+        p0 = ptx::ex2_approx(x0);
+        p1 = ptx::ex2_approx(x1);
+      }
+      pk[i] = pack2<BF16>(p0, p1);
+      if (i & 1) {
+        sc = ptx::add_lo16<BF16>(pk[i], sc);
+        sd = ptx::add_hi16<BF16>(pk[i], sd);
+      } else {
+        sa = ptx::add_lo16<BF16>(pk[i], sa);
+        sb = ptx::add_hi16<BF16>(pk[i], sb);
       }
     }
     ptx::tmem_st_x16(tS + c0 / 2, pk);
   }
-  l = l * alpha + (sum0 + sum1);
+  l = l * alpha + ((sa + sb) + (sc + sd));
   if (__any_sync(0xffffffffu, need)) {
     if (!__all_sync(0xffffffffu, wait_o())) return false;
     ptx::tc_fence_after();
+    const uint64_t a2 = ptx::f2_pack(alpha, alpha);
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t o[32];
       tmem_ld_wait<32>(tO + c0, o);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+      for (int c = 0; c < 32; c += 2) {
+        float o0, o1;
+        ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), a2),
+                       o0, o1);
+        o[c] = __float_as_uint(o0);
+        o[c + 1] = __float_as_uint(o1);
+      }
       tmem_st<32>(tO + c0, o);
     }
   }

@@ -35,10 +35,11 @@ namespace pair {
 
 constexpr int NUM_THREADS = 384;
 constexpr int PRODUCER_WARP = 8;
+constexpr int RING_CONSUMERS = 1 + 8;  // MMA thread + one arrival per softmax warp
 constexpr int MMA_WARP = 9;
 constexpr uint32_t REG_LAUNCH = 168;  // 65536 / 384 rounded down to a multiple of 8
-constexpr uint32_t REG_LOW = 104;
-constexpr uint32_t REG_HIGH = 200;
+constexpr uint32_t REG_LOW = 120;
+constexpr uint32_t REG_HIGH = 192;
 static_assert(128 * REG_LOW + 256 * REG_HIGH == NUM_THREADS * REG_LAUNCH, "register split");
 constexpr int BN = 128;
 
@@ -60,6 +61,7 @@ struct Barriers {
   uint64_t s_full[2], p_full[2];  // per query tile (A, B)
   uint64_t o_ready[2], o_free[2];
   uint64_t drain;
+  ItemRing ring;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -108,6 +110,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&bars->o_free[i], 4);
     }
     ptx::mbar_init(&bars->drain, 1);
+    for (int i = 0; i < ITEM_RING; ++i) {
+      ptx::mbar_init(&bars->ring.full[i], 1);
+      ptx::mbar_init(&bars->ring.empty[i], RING_CONSUMERS);
+    }
     bars->abort_flag = 0;
     ptx::mbar_init_fence();
   }
@@ -136,10 +142,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   ptx::setmaxnreg_dec<REG_LOW>();
   if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // The whole warp runs the scheduler and publishes items on the ring;
+    // lane 0 issues the TMA copies.
+    {
       Scheduler<BN> sched;
       sched.init(p);
-      WorkItem w;
+      uint32_t rs = 0, rph = 0;
       uint32_t slot = 0, phase = 0, q_count = 0;
       uint32_t slot_fills[NSLOT];
       for (int s = 0; s < NSLOT; ++s) slot_fills[s] = 0;
@@ -161,14 +169,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         return true;
       };
       // Ring order per item: K0, V0, K1, V1, ..., K(n-1), V(n-1).
-      while (ok && sched.next(w)) {
+      // Loads of one item, issued by lane 0; false when a bounded wait gave up.
+      auto load_item = [&](const WorkItem &w) -> bool {
         const int n = w.n_kv;
-        if (n == 0) continue;
+        bool ok = true;
         const int h0 = 2 * w.hu;
         const int kv_h = h0 / p.group;
-        ok = load_kv(&tm_k, kv_h, w.k0);
-        if (!ok) break;
-        if (!wait_bar(&bars->q_empty, (q_count & 1u) ^ 1u, abort_flag)) break;
+        if (!load_kv(&tm_k, kv_h, w.k0)) return false;
+        if (!wait_bar(&bars->q_empty, (q_count & 1u) ^ 1u, abort_flag)) return false;
         ptx::mbar_arrive_expect_tx(&bars->q_full, 2 * Q_BYTES);
 #pragma unroll
         for (int t = 0; t < 2; ++t)
@@ -181,17 +189,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = load_kv(&tm_v, kv_h, w.k0 + j * BN);
           if (ok && j + 1 < n) ok = load_kv(&tm_k, kv_h, w.k0 + (j + 1) * BN);
         }
+        return ok;
+      };
+      for (;;) {
+        WorkItem w;
+        const bool have = sched.next(w);
+        if (!have) w.hu = -1;
+        if (lane == 0) {
+          ok = wait_bar(&bars->ring.empty[rs], rph ^ 1u, abort_flag);
+          if (ok) {
+            bars->ring.items[rs] = w;
+            ptx::mbar_arrive(&bars->ring.full[rs]);
+          }
+        }
+        if (++rs == ITEM_RING) {
+          rs = 0;
+          rph ^= 1u;
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!have || !ok) break;
+        if (lane == 0 && w.n_kv > 0) ok = load_item(w);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
       }
-      for (int s = 0; s < NSLOT; ++s)
-        if (slot_fills[s] > 0) wait_bar(&bars->full[s], (slot_fills[s] - 1) & 1u, abort_flag);
-      if (q_count > 0) wait_bar(&bars->q_full, (q_count - 1) & 1u, abort_flag);
+      if (lane == 0) {
+        // Drain: every copy this thread issued has landed before the CTA exits.
+        for (int s = 0; s < NSLOT; ++s)
+          if (slot_fills[s] > 0) wait_bar(&bars->full[s], (slot_fills[s] - 1) & 1u, abort_flag);
+        if (q_count > 0) wait_bar(&bars->q_full, (q_count - 1) & 1u, abort_flag);
+      }
     }
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      Scheduler<BN> sched;
-      sched.init(p);
-      WorkItem w;
+      uint32_t rs = 0, rph = 0;
       uint32_t slot = 0, phase = 0, g = 0, items = 0;
       bool ok = true;
       const uint32_t sQ_addr = ptx::smem_u32(sQ);
@@ -226,7 +257,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                       (acc || kk > 0) ? 1u : 0u);
         }
       };
-      while (ok && sched.next(w)) {
+      while (ok) {
+        if (!(ok = wait_bar(&bars->ring.full[rs], rph, abort_flag))) break;
+        const WorkItem w = bars->ring.items[rs];
+        ptx::mbar_arrive(&bars->ring.empty[rs]);
+        if (++rs == ITEM_RING) {
+          rs = 0;
+          rph ^= 1u;
+        }
+        if (w.hu < 0) break;
         const int n = w.n_kv;
         if (n == 0) continue;
         if (!wait_bar(&bars->q_full, items & 1u, abort_flag)) break;
@@ -288,13 +327,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tS = tmem + lane_base + t * BN;
     const uint32_t tO = tmem + lane_base + O_COL0 + t * D;
     const float sl2 = p.scale_log2;
-    Scheduler<BN> sched;
-    sched.init(p);
-    WorkItem w;
+    uint32_t rs = 0, rph = 0;
     uint32_t g = 0, items = 0;
     bool ok = true;
     auto no_wait = []() { return true; };
-    while (ok && sched.next(w)) {
+    while (ok) {
+      bool have = wait_bar(&bars->ring.full[rs], rph, abort_flag);
+      if (!__all_sync(0xffffffffu, have)) break;
+      const WorkItem w = bars->ring.items[rs];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->ring.empty[rs]);
+      if (++rs == ITEM_RING) {
+        rs = 0;
+        rph ^= 1u;
+      }
+      if (w.hu < 0) break;
       const int n = w.n_kv;
       const int h = 2 * w.hu + t;
       const int qi = w.qi0 + r;

@@ -16,8 +16,10 @@
  *
  * Kernels (all persistent, one CTA per SM, warp-specialised, tcgen05 MMAs
  * into TMEM fed by TMA):
- *   fwd_pair.cuh    two query heads of one GQA group per work item (ping-pong
- *                   softmax warpgroups), D = 64 / 128, H / Hkv even
+ *   fwd_pair_db.cuh two query heads of one GQA group per work item, 64-key
+ *                   tiles, double-buffered S per tile, D = 64 / 128, H / Hkv even
+ *   fwd_pair.cuh    the same pairing with 128-key tiles and one S buffer per
+ *                   tile (ping-pong), selected at build time
  *   fwd_single.cuh  one query tile per work item, every other case
  */
 #include <cuda.h>
@@ -30,8 +32,15 @@
 
 #include "fwd_common.cuh"
 #include "fwd_pair.cuh"
+#include "fwd_pair_db.cuh"
 #include "fwd_single.cuh"
 #include "varlen_attn.h"
+
+// Pair kernel selection: 1 = 64-key tiles with double-buffered S
+// (fwd_pair_db.cuh), 0 = 128-key tiles with one S buffer (fwd_pair.cuh).
+#ifndef PAIR_DOUBLE_BUFFERED
+#define PAIR_DOUBLE_BUFFERED 0
+#endif
 
 namespace vattn {
 
@@ -112,6 +121,15 @@ static int launch_single(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
 }
 
 template <int D, bool BF16>
+static int launch_pairdb(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                         const KParams &kp, int grid, cudaStream_t s, DeviceInfo &dev, int slot) {
+  constexpr size_t smem = pairdb::smem_bytes<D>();
+  static_assert(smem <= 232448, "shared memory budget");
+  return launch_kernel(pairdb::fwd_kernel<D, BF16>, smem, pairdb::NUM_THREADS, tq, tk, tv, kp,
+                       grid, s, dev.attr_set[slot], (int)pairdb::REG_LAUNCH);
+}
+
+template <int D, bool BF16>
 static int launch_pair(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                        const KParams &kp, int grid, cudaStream_t s, DeviceInfo &dev, int slot) {
   constexpr size_t smem = pair::smem_bytes<D>();
@@ -174,7 +192,8 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
   // Query-head pairs share a key/value head when the group size is even;
   // the pair kernel then covers D = 64 and 128 (TMEM holds 2 x (S + O)).
   const bool use_pair = (group % 2 == 0) && (D == 64 || D == 128);
-  const int BN = use_pair ? pair::BN : (D == 256 ? single::Cfg<256>::BN : single::Cfg<128>::BN);
+  const int pair_bn = PAIR_DOUBLE_BUFFERED ? pairdb::BN : pair::BN;
+  const int BN = use_pair ? pair_bn : (D == 256 ? single::Cfg<256>::BN : single::Cfg<128>::BN);
   alignas(64) CUtensorMap tq, tk, tv;
   memset(&tk, 0, sizeof tk);
   memset(&tv, 0, sizeof tv);
@@ -209,6 +228,13 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
   if (grid < 1) grid = 1;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (use_pair && PAIR_DOUBLE_BUFFERED) {
+    if (D == 64)
+      return bf16 ? launch_pairdb<64, true>(tq, tk, tv, kp, grid, s, dev, 10)
+                  : launch_pairdb<64, false>(tq, tk, tv, kp, grid, s, dev, 11);
+    return bf16 ? launch_pairdb<128, true>(tq, tk, tv, kp, grid, s, dev, 12)
+                : launch_pairdb<128, false>(tq, tk, tv, kp, grid, s, dev, 13);
+  }
   if (use_pair) {
     if (D == 64)
       return bf16 ? launch_pair<64, true>(tq, tk, tv, kp, grid, s, dev, 0)
