@@ -36,11 +36,7 @@ import workloads  # noqa: E402
 METRIC = "varlen attn fwd TFLOP/s (unmasked FLOPs) and % of B200 dense bf16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["flash_attention_fwd_b200/csrc/varlen_attn_fwd.cu",
-                  "flash_attention_fwd_b200/csrc/fwd_common.cuh",
-                  "flash_attention_fwd_b200/csrc/fwd_pair.cuh",
-                  "flash_attention_fwd_b200/csrc/fwd_single.cuh",
-                  "flash_attention_fwd_b200/csrc/sm100_ptx.cuh"]
+KERNEL_DIR = "flash_attention_fwd_b200/csrc"
 
 
 # ----------------------------------------------------------------------------- counting
@@ -81,11 +77,14 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_hash() -> str:
+def kernel_hash(read=None) -> str:
+    """Hash of every CUDA source of the library (file names sorted)."""
+    d = os.path.join(ROOT, KERNEL_DIR)
+    names = sorted(n for n in os.listdir(d) if n.endswith((".cu", ".cuh")))
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+    for n in names:
+        h.update(n.encode())
+        h.update(read(n) if read else open(os.path.join(d, n), "rb").read())
     return h.hexdigest()[:16]
 
 

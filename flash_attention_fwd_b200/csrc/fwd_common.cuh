@@ -37,17 +37,20 @@ struct KParams {
   void *out;
   float *lse;
   int B, H, Hkv, group;  // group = H / Hkv
-  int head_units;        // heads per work item row: H (one tile) or H/2 (head pairs)
+  int head_units;        // head units per (sequence, token range): H, H/2 (head pairs) or Hkv (packed)
+  int unit_tokens;       // query tokens per work item (divides BM)
+  int pack_log2;         // 0: a tile's rows are BM tokens of one head; k > 0: a tile's rows are
+                         // BM >> k tokens x the 2^k query heads of one key/value head
   int total_q, total_k;
   int causal;
   float scale_log2;  // scale * log2(e)
 };
 
 struct WorkItem {
-  int hu;       // head unit (a head, or a pair of heads 2hu, 2hu+1)
-  int q0;       // packed index of the tile's first query token
-  int q_rows;   // valid rows in the tile (<= BM)
-  int qi0;      // sequence-local index of the tile's first query
+  int hu;       // head unit (a head, a pair of heads 2hu, 2hu+1, or a key/value head)
+  int q0;       // packed index of the item's first query token
+  int q_rows;   // valid query tokens in the item (<= unit_tokens)
+  int qi0;      // sequence-local index of the item's first query
   int k0;       // packed index of the sequence's first key
   int Lk;       // keys in the sequence
   int n_kv;     // key tiles to visit
@@ -55,10 +58,11 @@ struct WorkItem {
 };
 
 // ---------------------------------------------------------------------------
-// Work scheduler.  A work item is (sequence b, query tile qt of BM rows, head
-// unit hu).  Its cost is measured in 128-key tiles: with the causal rule a
-// query tile needs the keys [0, min(Lk, min(Lq, (qt+1) * BM))), i.e.
-// min(nk, qt + 1) tiles where nk = ceil(Lk / BM); without it, nk tiles.  Items
+// Work scheduler.  A work item is (sequence b, query range qt of U tokens,
+// head unit hu), U = unit_tokens dividing BM.  Its cost is measured in 128-key
+// tiles: with the causal rule the range needs the keys
+// [0, min(Lk, min(Lq, (qt+1) * U))), i.e. min(nk, ceil((qt+1) / R)) tiles
+// where nk = ceil(Lk / BM) and R = BM / U; without it, nk tiles.  Items
 // are listed by cost level, highest first ("longest processing time first"),
 // and within a level by sequence, query tile, head unit (the head units that
 // share K/V tiles are adjacent, so they run at the same time on neighbouring
@@ -72,7 +76,7 @@ struct WorkItem {
 template <int BN>
 struct Scheduler {
   const int *cu_q, *cu_k;
-  int B, HU, causal, total_q, total_k;
+  int B, HU, U, R, causal, total_q, total_k;
   int cta, grid, lane;
   long long round;
   int level;              // current cost level; -1 once the list is exhausted
@@ -93,21 +97,22 @@ struct Scheduler {
     lq = qe - qs;
     lk = ke - ks;
   }
-  // (sequence, query tile) units of a sequence at cost level c
+  // (sequence, query range) units of a sequence at cost level c; nq ranges of
+  // U tokens, nk tiles of BM keys
   __device__ int units_at(int nq, int nk, int c) const {
     if (!causal || nk == 0) return (c == nk) ? nq : 0;
-    if (c >= 1 && c < nk) return (c <= nq) ? 1 : 0;
-    if (c == nk) return (nq >= nk) ? nq - nk + 1 : 0;
+    if (c >= 1 && c < nk) return max(0, min(c * R, nq) - (c - 1) * R);
+    if (c == nk) return max(0, nq - (nk - 1) * R);
     return 0;
   }
-  // query tile of the k-th unit of a sequence at level c
+  // query range of the k-th unit of a sequence at level c
   __device__ int tile_of(int nk, int c, int k) const {
-    if (causal && nk > 0) return (c < nk) ? c - 1 : nk - 1 + k;
+    if (causal && nk > 0) return (min(c, nk) - 1) * R + k;
     return k;
   }
   __device__ int top_level(int nq, int nk) const {
     if (nq == 0) return -1;
-    return (causal && nk > 0) ? min(nk, nq) : nk;
+    return (causal && nk > 0) ? min(nk, (nq + R - 1) / R) : nk;
   }
   __device__ long long count_level(int c) const {
     long long u = 0;
@@ -116,7 +121,7 @@ struct Scheduler {
       if (b < B) {
         int qs, lq, ks, lk;
         extents(b, qs, lq, ks, lk);
-        v = units_at((lq + BM - 1) / BM, (lk + BM - 1) / BM, c);
+        v = units_at((lq + U - 1) / U, (lk + BM - 1) / BM, c);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -130,6 +135,8 @@ struct Scheduler {
     cu_k = p.cu_k;
     B = p.B;
     HU = p.head_units;
+    U = p.unit_tokens;
+    R = BM / U;
     causal = p.causal;
     total_q = p.total_q;
     total_k = p.total_k;
@@ -143,7 +150,7 @@ struct Scheduler {
       if (b < B) {
         int qs, lq, ks, lk;
         extents(b, qs, lq, ks, lk);
-        top = max(top, top_level((lq + BM - 1) / BM, (lk + BM - 1) / BM));
+        top = max(top, top_level((lq + U - 1) / U, (lk + BM - 1) / BM));
       }
     }
 #pragma unroll
@@ -176,7 +183,7 @@ struct Scheduler {
       int qs = 0, lq = 0, ks = 0, lk = 0, u = 0;
       if (b < B) {
         extents(b, qs, lq, ks, lk);
-        u = units_at((lq + BM - 1) / BM, (lk + BM - 1) / BM, level);
+        u = units_at((lq + U - 1) / U, (lk + BM - 1) / BM, level);
       }
       int incl = u;
 #pragma unroll
@@ -197,12 +204,12 @@ struct Scheduler {
         cur_units += before;
         const int k = (int)(unit - cur_units);
         const int qt = tile_of((lk + BM - 1) / BM, level, k);
-        w.qi0 = qt * BM;
+        w.qi0 = qt * U;
         w.q0 = qs + w.qi0;
-        w.q_rows = min(BM, lq - w.qi0);
+        w.q_rows = min(U, lq - w.qi0);
         w.k0 = ks;
         w.Lk = lk;
-        const int kv_end = causal ? min(lk, min(lq, w.qi0 + BM)) : lk;
+        const int kv_end = causal ? min(lk, min(lq, w.qi0 + U)) : lk;
         w.n_kv = (kv_end + BN - 1) / BN;
         w.min_lim = causal ? min(lk, w.qi0 + 1) : lk;
         return true;
@@ -253,6 +260,10 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 template <int N>
 __device__ __forceinline__ void tmem_ld_wait(uint32_t taddr, uint32_t (&r)[N]);
 template <>
+__device__ __forceinline__ void tmem_ld_wait<16>(uint32_t taddr, uint32_t (&r)[16]) {
+  ptx::tmem_ld_x16_wait(taddr, r);
+}
+template <>
 __device__ __forceinline__ void tmem_ld_wait<32>(uint32_t taddr, uint32_t (&r)[32]) {
   ptx::tmem_ld_x32_wait(taddr, r);
 }
@@ -267,6 +278,10 @@ __device__ __forceinline__ void tmem_ld_wait<128>(uint32_t taddr, uint32_t (&r)[
 
 template <int N>
 __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&r)[N]);
+template <>
+__device__ __forceinline__ void tmem_st<16>(uint32_t taddr, const uint32_t (&r)[16]) {
+  ptx::tmem_st_x16(taddr, r);
+}
 template <>
 __device__ __forceinline__ void tmem_st<32>(uint32_t taddr, const uint32_t (&r)[32]) {
   ptx::tmem_st_x32(taddr, r);

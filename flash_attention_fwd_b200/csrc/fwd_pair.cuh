@@ -1,31 +1,40 @@
 /*
- * fwd_pair.cuh — attention forward, two query tiles per work item that share
- * every K/V tile: the same 128 query rows of the two query heads 2u and 2u+1,
- * which map to the same key/value head whenever H / Hkv is even (GQA head map
- * kv_h = h / (H / Hkv)).  Head dims 64 and 128.
+ * fwd_pair.cuh — attention forward with two 128-row query tiles per work item
+ * that share every K/V tile (D = 64 and 128, H / Hkv even).
+ *
+ * Two row layouts (KParams::pack_log2):
+ *   0      tile A = 128 tokens of query head 2u, tile B = the same tokens of
+ *          head 2u+1 (both map to one key/value head because H / Hkv is even:
+ *          GQA head map kv_h = h / (H / Hkv));
+ *   k > 0  "GQA-packed": a tile holds 128 >> k tokens x the 2^k = H / Hkv query
+ *          heads of key/value head u (row r = token r >> k, head r & (2^k - 1));
+ *          tile B holds the next 128 >> k tokens.  Short query sequences then
+ *          fill the 128 MMA rows, and each K/V tile is read once per key/value
+ *          head.
  *
  * One persistent CTA per SM, 384 threads (three warpgroups):
- *   warps 0-3  softmax warpgroup A (query head 2u; thread t = row t = TMEM lane t)
- *   warps 4-7  softmax warpgroup B (query head 2u+1)
- *   warp 8     TMA producer: both Q tiles, K/V tiles through a shared-memory ring
- *   warp 9     TMEM owner and MMA issuer
+ *   warps 0-3   softmax warpgroup A (thread t = row t of tile A = TMEM lane t)
+ *   warps 4-7   softmax warpgroup B
+ *   warp 8      scheduler + TMA producer (both Q tiles, K/V ring)
+ *   warp 9      TMEM owner and MMA issuer
  *   warps 10-11 idle
  * The kernel is compiled for REG_LAUNCH registers per thread; the third
  * warpgroup gives registers back (REG_LOW) and the softmax warpgroups take
  * them (REG_HIGH): 128 * REG_LOW + 256 * REG_HIGH == 384 * REG_LAUNCH.  The
  * host refuses to launch a build whose register count is not REG_LAUNCH.
- * TMEM: S_A, S_B (BN columns each, P aliases their first BN/2 columns), O_A,
- * O_B (D columns each).  The MMA warp alternates between the tiles:
- *   S_A(0), S_B(0), then for each key tile j:
- *     PV_A(j), S_A(j+1), PV_B(j), S_B(j+1)
- * so softmax A of tile j runs while the tensor cores do PV_B(j-1), S_B(j),
- * and softmax B while they do PV_A(j), S_A(j+1) ("ping-pong").  Each K/V tile
- * crosses L2 -> shared memory once for both query tiles.
  *
- * Because S_T(j) is issued after PV_T(j-1) and its tcgen05.commit tracks all
- * earlier MMAs of the issuing thread, the arrival of S_T(j) implies that
- * PV_T(j-1) has completed: the softmax may rescale O_T in place without a
- * further wait.
+ * TMEM: S_A, S_B (128 columns each; P aliases their first 64 columns), O_A,
+ * O_B (D columns each).  The MMA warp alternates between the tiles: after
+ * S_A(0), S_B(0), for each key tile j it issues PV_A(j), S_A(j+1), PV_B(j),
+ * S_B(j+1), so softmax A runs while the tensor cores work for tile B and vice
+ * versa.  P_T(j) is handed over in PAIR_P_CHUNKS pieces and PV_T(j) is issued
+ * piece by piece.  (A build option, PAIR_S_SPLIT, also computes the upper half
+ * of S_T(j+1) — keys 64..127 into columns 64..127, which P does not use — as
+ * soon as the softmax has read S_T(j); it measured slower and is off.)
+ * Because S_T(j) (its lower half with the split) is issued after PV_T(j-1)
+ * and its tcgen05.commit tracks every earlier MMA of the issuing thread, the
+ * arrival of S_T(j) proves that PV_T(j-1) completed: the softmax may rescale
+ * O_T in place, before its first P piece, without a further wait.
  */
 #pragma once
 #include "fwd_common.cuh"
@@ -42,6 +51,18 @@ constexpr uint32_t REG_LOW = 120;
 constexpr uint32_t REG_HIGH = 192;
 static_assert(128 * REG_LOW + 256 * REG_HIGH == NUM_THREADS * REG_LAUNCH, "register split");
 constexpr int BN = 128;
+// P is handed to the MMA warp in NCHUNK pieces of BN / NCHUNK keys; with
+// S_SPLIT the upper half of S(j+1) is computed while the softmax runs.
+#ifndef PAIR_P_CHUNKS
+#define PAIR_P_CHUNKS 2
+#endif
+#ifndef PAIR_S_SPLIT
+#define PAIR_S_SPLIT 0
+#endif
+constexpr int NCHUNK = PAIR_P_CHUNKS;
+constexpr int CHUNK_KEYS = BN / NCHUNK;
+constexpr bool S_SPLIT = PAIR_S_SPLIT != 0;
+static_assert(NCHUNK == 1 || NCHUNK == 2 || NCHUNK == 4, "P chunks");
 
 template <int D>
 struct Cfg;
@@ -58,7 +79,8 @@ struct Barriers {
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t q_full, q_empty;
-  uint64_t s_full[2], p_full[2];  // per query tile (A, B)
+  uint64_t s_full[2], s_loaded[2];  // per query tile (A, B)
+  uint64_t p_chunk[2][NCHUNK];
   uint64_t o_ready[2], o_free[2];
   uint64_t drain;
   ItemRing ring;
@@ -69,6 +91,95 @@ struct Barriers {
 template <int D>
 constexpr size_t smem_bytes() {
   return (size_t)2 * BM * D * 2 + (size_t)Cfg<D>::NSLOT * BN * D * 2 + sizeof(Barriers) + 1024;
+}
+
+// Softmax of one 128-key S tile with fine-grained hand-offs: `loaded()` once
+// S is in registers, `chunk_ready(c)` once P columns [16c, 16c+16) (keys
+// 32c..32c+31) are in TMEM.  O is rescaled (when the running max jumps) before
+// the first chunk is signalled.
+template <int D, bool BF16, class Loaded, class ChunkReady>
+__device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, int j, float sl2,
+                                                     bool need_mask, int lim, float &m, float &l,
+                                                     Loaded &&loaded, ChunkReady &&chunk_ready) {
+  uint32_t sr[BN];
+  tmem_ld_wait<BN>(tS, sr);
+  loaded();
+  float s[BN];
+#pragma unroll
+  for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
+  if (need_mask) {
+#pragma unroll
+    for (int c = 0; c < BN; ++c)
+      if (c >= lim) s[c] = -INFINITY;
+  }
+  float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+  for (int c = 4; c + 8 <= BN; c += 8) {
+    mx0 = ptx::fmax3(mx0, s[c], s[c + 1]);
+    mx1 = ptx::fmax3(mx1, s[c + 2], s[c + 3]);
+    mx2 = ptx::fmax3(mx2, s[c + 4], s[c + 5]);
+    mx3 = ptx::fmax3(mx3, s[c + 6], s[c + 7]);
+  }
+  mx0 = ptx::fmax3(mx0, s[BN - 4], s[BN - 3]);
+  mx1 = ptx::fmax3(mx1, s[BN - 2], s[BN - 1]);
+  const float mx = fmaxf(ptx::fmax3(mx0, mx1, mx2), mx3) * sl2;
+  float alpha = 1.f;
+  bool need = false;
+  if (j == 0) {
+    m = (mx == -INFINITY) ? 0.f : mx;
+  } else if (mx > m + RESCALE_THRESHOLD) {
+    alpha = ptx::ex2_approx(m - mx);
+    m = mx;
+    need = true;
+  }
+  if (__any_sync(0xffffffffu, need)) {
+    // 16-column pieces: the whole S row is still live here
+    const uint64_t a2 = ptx::f2_pack(alpha, alpha);
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 16) {
+      uint32_t o[16];
+      tmem_ld_wait<16>(tO + c0, o);
+#pragma unroll
+      for (int c = 0; c < 16; c += 2) {
+        float o0, o1;
+        ptx::f2_unpack(
+            ptx::f2_mul(ptx::f2_pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), a2), o0,
+            o1);
+        o[c] = __float_as_uint(o0);
+        o[c + 1] = __float_as_uint(o1);
+      }
+      tmem_st<16>(tO + c0, o);
+    }
+  }
+  const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+  const uint64_t negm_2 = ptx::f2_pack(-m, -m);
+  float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
+#pragma unroll
+  for (int c0 = 0; c0 < BN; c0 += 32) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = c0 + 2 * i;
+      const uint64_t x2 = ptx::f2_fma(ptx::f2_pack(s[c], s[c + 1]), sl2_2, negm_2);
+      float x0, x1;
+      ptx::f2_unpack(x2, x0, x1);
+      pk[i] = pack2<BF16>(ptx::ex2_approx(x0), ptx::ex2_approx(x1));
+      // the rounded P values (what the PV MMA sees) go into the row sum
+      if (i & 1) {
+        sc = ptx::add_lo16<BF16>(pk[i], sc);
+        sd = ptx::add_hi16<BF16>(pk[i], sd);
+      } else {
+        sa = ptx::add_lo16<BF16>(pk[i], sa);
+        sb = ptx::add_hi16<BF16>(pk[i], sb);
+      }
+    }
+    ptx::tmem_st_x16(tS + c0 / 2, pk);
+    if ((c0 + 32) % CHUNK_KEYS == 0) {
+      ptx::tmem_st_wait();
+      chunk_ready(c0 / CHUNK_KEYS);
+    }
+  }
+  l = l * alpha + ((sa + sb) + (sc + sd));
 }
 
 template <int D, bool BF16>
@@ -82,7 +193,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // TMEM columns: S_t at [t*BN, (t+1)*BN), O_t at [2*BN + t*D, 2*BN + (t+1)*D)
   constexpr uint32_t O_COL0 = 2 * BN;
   static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
-  constexpr uint32_t IDESC_S = ptx::idesc_f16(BM, BN, BF16, false);
+  constexpr uint32_t IDESC_S_FULL = ptx::idesc_f16(BM, BN, BF16, false);
+  constexpr uint32_t IDESC_S_HALF = ptx::idesc_f16(BM, BN / 2, BF16, false);
   constexpr uint32_t IDESC_PV = ptx::idesc_f16(BM, D, BF16, true);
 
   extern __shared__ uint8_t smem_raw[];
@@ -95,6 +207,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  const int pack = p.pack_log2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -105,7 +218,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::mbar_init(&bars->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars->s_full[i], 1);
-      ptx::mbar_init(&bars->p_full[i], 4);
+      ptx::mbar_init(&bars->s_loaded[i], 4);
+      for (int c = 0; c < NCHUNK; ++c) ptx::mbar_init(&bars->p_chunk[i][c], 4);
       ptx::mbar_init(&bars->o_ready[i], 1);
       ptx::mbar_init(&bars->o_free[i], 4);
     }
@@ -139,12 +253,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tc_fence_after();
   };
   if (warp >= 8) {
-  ptx::setmaxnreg_dec<REG_LOW>();
-  if (warp == PRODUCER_WARP) {
-    // ------------------------------------------------------------ producer
-    // The whole warp runs the scheduler and publishes items on the ring;
-    // lane 0 issues the TMA copies.
-    {
+    ptx::setmaxnreg_dec<REG_LOW>();
+    if (warp == PRODUCER_WARP) {
+      // ---------------------------------------------------------- producer
+      // The whole warp runs the scheduler and publishes items on the ring;
+      // lane 0 issues the TMA copies.
       Scheduler<BN> sched;
       sched.init(p);
       uint32_t rs = 0, rph = 0;
@@ -168,26 +281,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         return true;
       };
-      // Ring order per item: K0, V0, K1, V1, ..., K(n-1), V(n-1).
-      // Loads of one item, issued by lane 0; false when a bounded wait gave up.
+      // Ring order per item: K0, K1, V0, K2, V1, K3, ..., V(n-1) — the order
+      // in which the MMA warp consumes them.  Loads of one item, issued by
+      // lane 0; false when a bounded wait gave up.
       auto load_item = [&](const WorkItem &w) -> bool {
         const int n = w.n_kv;
-        bool ok = true;
-        const int h0 = 2 * w.hu;
-        const int kv_h = h0 / p.group;
+        const int kv_h = pack ? w.hu : (2 * w.hu) / p.group;
         if (!load_kv(&tm_k, kv_h, w.k0)) return false;
         if (!wait_bar(&bars->q_empty, (q_count & 1u) ^ 1u, abort_flag)) return false;
         ptx::mbar_arrive_expect_tx(&bars->q_full, 2 * Q_BYTES);
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t) {
+          // packed: tile t = next (BM >> pack) tokens, all heads of kv_h;
+          // otherwise: tile t = head 2u + t
+          const int head = pack ? (w.hu << pack) : (2 * w.hu + t);
+          const int tok = pack ? (w.q0 + t * (BM >> pack)) : w.q0;
 #pragma unroll
           for (int db = 0; db < DB; ++db)
             ptx::tma_load_3d(sQ + t * Q_BYTES + db * (BM * 128), &tm_q, &bars->q_full, db * 64,
-                             h0 + t, w.q0);
+                             head, tok);
+        }
         ++q_count;
+        bool ok = true;
+        if (n >= 2) ok = load_kv(&tm_k, kv_h, w.k0 + BN);
         for (int j = 0; ok && j < n; ++j) {
           ok = load_kv(&tm_v, kv_h, w.k0 + j * BN);
-          if (ok && j + 1 < n) ok = load_kv(&tm_k, kv_h, w.k0 + (j + 1) * BN);
+          if (ok && j + 2 < n) ok = load_kv(&tm_k, kv_h, w.k0 + (j + 2) * BN);
         }
         return ok;
       };
@@ -218,10 +337,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (slot_fills[s] > 0) wait_bar(&bars->full[s], (slot_fills[s] - 1) & 1u, abort_flag);
         if (q_count > 0) wait_bar(&bars->q_full, (q_count - 1) & 1u, abort_flag);
       }
-    }
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == MMA_WARP && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       uint32_t rs = 0, rph = 0;
       uint32_t slot = 0, phase = 0, g = 0, items = 0;
       bool ok = true;
@@ -237,24 +354,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         return true;
       };
-      auto issue_s = [&](int t, uint32_t kslot) {
+      // S_t columns [row0, row0 + N) = Q_t K^T for key rows [row0, row0 + N)
+      // of the K tile, over D in steps of 16 (K-major, 128-byte swizzle).
+      auto issue_s = [&](int t, uint32_t kslot, uint32_t row0, uint32_t idesc) {
         const uint32_t qbase = sQ_addr + t * Q_BYTES;
-        const uint32_t kbase = sKV_addr + kslot * KV_BYTES;
+        const uint32_t kbase = sKV_addr + kslot * KV_BYTES + row0 * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk % 4) * 32u;
           uint64_t a = ptx::sdesc_sw128(qbase + (kk / 4) * (BM * 128) + off, 16, 1024);
           uint64_t bdesc = ptx::sdesc_sw128(kbase + (kk / 4) * (BN * 128) + off, 16, 1024);
-          ptx::mma_ss(tmem + t * BN, a, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+          ptx::mma_ss(tmem + t * BN + row0, a, bdesc, idesc, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, uint32_t vslot, bool acc) {
+      // O_t += P_t V for keys [c * CHUNK_KEYS, (c + 1) * CHUNK_KEYS) (P from
+      // TMEM, V MN-major), in steps of 16 keys
+      auto issue_pv_chunk = [&](int t, uint32_t vslot, int c, bool acc) {
         const uint32_t vbase = sKV_addr + vslot * KV_BYTES;
+        constexpr int KS = CHUNK_KEYS / 16;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
+        for (int kk = KS * c; kk < KS * c + KS; ++kk) {
           uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
           ptx::mma_ts(tmem + O_COL0 + t * D, tmem + t * BN + kk * 8, bdesc, IDESC_PV,
-                      (acc || kk > 0) ? 1u : 0u);
+                      (acc || kk > KS * c) ? 1u : 0u);
         }
       };
       while (ok) {
@@ -268,36 +390,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (w.hu < 0) break;
         const int n = w.n_kv;
         if (n == 0) continue;
-        if (!wait_bar(&bars->q_full, items & 1u, abort_flag)) break;
+        if (!(ok = wait_bar(&bars->q_full, items & 1u, abort_flag))) break;
         ptx::tc_fence_after();
         uint32_t ks;
         if (!(ok = take_slot(ks))) break;
-        issue_s(0, ks);
+        issue_s(0, ks, 0, IDESC_S_FULL);
         ptx::mma_commit(&bars->s_full[0]);
-        issue_s(1, ks);
+        issue_s(1, ks, 0, IDESC_S_FULL);
         ptx::mma_commit(&bars->s_full[1]);
         ptx::mma_commit(&bars->empty[ks]);
         if (n == 1) ptx::mma_commit(&bars->q_empty);
         for (int j = 0; ok && j < n; ++j) {
-          const uint32_t gj = g + j;
-          uint32_t vs;
-          if (!(ok = take_slot(vs))) break;
+          const uint32_t par = (g + j) & 1u;
           const bool more = j + 1 < n;
-          uint32_t ks_next = 0;
+          uint32_t ks_next = 0, vs = 0;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            if (!(ok = wait_bar(&bars->p_full[t], gj & 1u, abort_flag))) break;
-            ptx::tc_fence_after();
+            if (S_SPLIT) {
+              // upper half of S_t(j+1) while the softmax works on S_t(j)
+              if (!(ok = wait_bar(&bars->s_loaded[t], par, abort_flag))) break;
+              ptx::tc_fence_after();
+              if (more) {
+                if (t == 0 && !(ok = take_slot(ks_next))) break;
+                issue_s(t, ks_next, BN / 2, IDESC_S_HALF);
+              }
+            } else if (more && t == 0 && !(ok = take_slot(ks_next))) {
+              break;
+            }
+            if (t == 0 && !(ok = take_slot(vs))) break;
             if (j == 0 && items > 0) {
               if (!(ok = wait_bar(&bars->o_free[t], (items - 1) & 1u, abort_flag))) break;
               ptx::tc_fence_after();
             }
-            issue_pv(t, vs, j > 0);
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c) {
+              if (!(ok = wait_bar(&bars->p_chunk[t][c], par, abort_flag))) break;
+              ptx::tc_fence_after();
+              issue_pv_chunk(t, vs, c, j > 0 || c > 0);
+            }
+            if (!ok) break;
             if (j == n - 1) ptx::mma_commit(&bars->o_ready[t]);
             if (t == 1) ptx::mma_commit(&bars->empty[vs]);
             if (more) {
-              if (t == 0 && !(ok = take_slot(ks_next))) break;
-              issue_s(t, ks_next);
+              // lower half of S_t(j+1): columns 0..63 that P_t(j) occupied
+              // (the whole of S_t(j+1) without the split)
+              issue_s(t, ks_next, 0, S_SPLIT ? IDESC_S_HALF : IDESC_S_FULL);
               ptx::mma_commit(&bars->s_full[t]);
               if (t == 1) {
                 ptx::mma_commit(&bars->empty[ks_next]);
@@ -309,28 +446,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         g += n;
         ++items;
       }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
       ptx::mma_commit(&bars->drain);
       wait_bar(&bars->drain, 0, abort_flag);
     }
-  }
-  end_of_kernel();
-  if (warp == MMA_WARP) {
-    __syncwarp();
-    ptx::tmem_dealloc(tmem, TMEM_COLS);
-  }
+    end_of_kernel();
+    if (warp == MMA_WARP) {
+      __syncwarp();
+      ptx::tmem_dealloc(tmem, TMEM_COLS);
+    }
   } else {
     ptx::setmaxnreg_inc<REG_HIGH>();
     // ------------------------------------------------------------ softmax WGs
-    const int t = warp / 4;              // query tile A (0) or B (1)
-    const int r = threadIdx.x - t * 128; // row in the tile == TMEM lane
+    const int t = warp / 4;               // query tile A (0) or B (1)
+    const int r = threadIdx.x - t * 128;  // row in the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * BN;
     const uint32_t tO = tmem + lane_base + O_COL0 + t * D;
     const float sl2 = p.scale_log2;
+    // row -> (token offset in the item, query head offset)
+    const int tok_off = pack ? t * (BM >> pack) + (r >> pack) : r;
+    const int head_off = pack ? (r & ((1 << pack) - 1)) : t;
     uint32_t rs = 0, rph = 0;
     uint32_t g = 0, items = 0;
     bool ok = true;
-    auto no_wait = []() { return true; };
+    auto arrive = [&](uint64_t *bar) {
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar);
+    };
     while (ok) {
       bool have = wait_bar(&bars->ring.full[rs], rph, abort_flag);
       if (!__all_sync(0xffffffffu, have)) break;
@@ -343,10 +487,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (w.hu < 0) break;
       const int n = w.n_kv;
-      const int h = 2 * w.hu + t;
-      const int qi = w.qi0 + r;
-      const bool row_valid = r < w.q_rows;
-      const size_t orow = (size_t)(w.q0 + r) * p.H + h;
+      const int h = (pack ? (w.hu << pack) : 2 * w.hu) + head_off;
+      const int qi = w.qi0 + tok_off;
+      const bool row_valid = tok_off < w.q_rows;
+      const size_t orow = (size_t)(w.q0 + tok_off) * p.H + h;
       uint16_t *orow_ptr = reinterpret_cast<uint16_t *>(p.out) + orow * D;
       if (n == 0) {
         if (row_valid) empty_row<D>(orow_ptr, p.lse + orow);
@@ -355,18 +499,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int key_lim = p.causal ? min(w.Lk, qi + 1) : w.Lk;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
-        const uint32_t gj = g + j;
-        bool got = wait_bar(&bars->s_full[t], gj & 1u, abort_flag);
+        const uint32_t par = (g + j) & 1u;
+        bool got = wait_bar(&bars->s_full[t], par, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        softmax_tile<BN, D, BF16>(tS, tO, j, sl2, (j + 1) * BN > w.min_lim, key_lim - j * BN, m,
-                                  l, no_wait);
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->p_full[t]);
+        softmax_tile_chunked<D, BF16>(
+            tS, tO, j, sl2, (j + 1) * BN > w.min_lim, key_lim - j * BN, m, l,
+            [&]() {
+              if (S_SPLIT) arrive(&bars->s_loaded[t]);
+            },
+            [&](int c) { arrive(&bars->p_chunk[t][c]); });
       }
       if (!ok) break;
       g += n;

@@ -16,10 +16,9 @@
  *
  * Kernels (all persistent, one CTA per SM, warp-specialised, tcgen05 MMAs
  * into TMEM fed by TMA):
- *   fwd_pair_db.cuh two query heads of one GQA group per work item, 64-key
- *                   tiles, double-buffered S per tile, D = 64 / 128, H / Hkv even
- *   fwd_pair.cuh    the same pairing with 128-key tiles and one S buffer per
- *                   tile (ping-pong), selected at build time
+ *   fwd_pair.cuh    two 128-row query tiles per work item sharing every K/V
+ *                   tile (two query heads of one GQA group, or GQA-packed rows
+ *                   for short queries), D = 64 / 128, H / Hkv even
  *   fwd_single.cuh  one query tile per work item, every other case
  */
 #include <cuda.h>
@@ -32,14 +31,13 @@
 
 #include "fwd_common.cuh"
 #include "fwd_pair.cuh"
-#include "fwd_pair_db.cuh"
 #include "fwd_single.cuh"
 #include "varlen_attn.h"
 
-// Pair kernel selection: 1 = 64-key tiles with double-buffered S
-// (fwd_pair_db.cuh), 0 = 128-key tiles with one S buffer (fwd_pair.cuh).
-#ifndef PAIR_DOUBLE_BUFFERED
-#define PAIR_DOUBLE_BUFFERED 0
+// GQA packing in the pair kernel: 0 = never, 1 = whenever H / Hkv is a power
+// of two, 2 = when the query sequences are short (see use_packing below).
+#ifndef PAIR_PACK_POLICY
+#define PAIR_PACK_POLICY 2
 #endif
 
 namespace vattn {
@@ -66,13 +64,14 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [rows, heads, D] row-major 16-bit tensor; box = 64 elements x 1 head x box_rows,
-// written to shared memory with the 128-byte swizzle the MMA descriptors expect.
+// [rows, heads, D] row-major 16-bit tensor; box = 64 elements x box_heads
+// heads x box_rows rows, written to shared memory (row-major over rows, then
+// heads) with the 128-byte swizzle the MMA descriptors expect.
 static bool encode_qkv_map(EncodeTiledFn enc, CUtensorMap *map, const void *base, bool bf16,
-                           int64_t rows, int heads, int D, int box_rows) {
+                           int64_t rows, int heads, int D, int box_rows, int box_heads = 1) {
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)heads, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)heads * D * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                    3, const_cast<void *>(base), dims, strides, box, estr,
@@ -118,15 +117,6 @@ static int launch_single(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
   static_assert(smem <= 232448, "shared memory budget");
   return launch_kernel(single::fwd_kernel<D, BF16>, smem, single::NUM_THREADS, tq, tk, tv, kp,
                        grid, s, dev.attr_set[slot]);
-}
-
-template <int D, bool BF16>
-static int launch_pairdb(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                         const KParams &kp, int grid, cudaStream_t s, DeviceInfo &dev, int slot) {
-  constexpr size_t smem = pairdb::smem_bytes<D>();
-  static_assert(smem <= 232448, "shared memory budget");
-  return launch_kernel(pairdb::fwd_kernel<D, BF16>, smem, pairdb::NUM_THREADS, tq, tk, tv, kp,
-                       grid, s, dev.attr_set[slot], (int)pairdb::REG_LAUNCH);
 }
 
 template <int D, bool BF16>
@@ -192,12 +182,23 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
   // Query-head pairs share a key/value head when the group size is even;
   // the pair kernel then covers D = 64 and 128 (TMEM holds 2 x (S + O)).
   const bool use_pair = (group % 2 == 0) && (D == 64 || D == 128);
-  const int pair_bn = PAIR_DOUBLE_BUFFERED ? pairdb::BN : pair::BN;
-  const int BN = use_pair ? pair_bn : (D == 256 ? single::Cfg<256>::BN : single::Cfg<128>::BN);
+  // GQA packing: a tile's 128 rows = (128 / group) tokens x the group's query
+  // heads.  It pays when query sequences are short next to a 128-row tile
+  // (most rows of a per-head tile would be empty); group must be a power of
+  // two dividing 128.
+  int pack_log2 = 0;
+  if (use_pair && (group & (group - 1)) == 0 && group <= BM) {
+    const bool short_q = (long long)max_seqlen_q * 2 <= BM;
+    if (PAIR_PACK_POLICY == 1 || (PAIR_PACK_POLICY == 2 && short_q))
+      while ((1 << pack_log2) < group) ++pack_log2;
+  }
+  const int BN = use_pair ? pair::BN : (D == 256 ? single::Cfg<256>::BN : single::Cfg<128>::BN);
   alignas(64) CUtensorMap tq, tk, tv;
   memset(&tk, 0, sizeof tk);
   memset(&tv, 0, sizeof tv);
-  if (!encode_qkv_map(enc, &tq, q, bf16, total_q, num_heads, D, BM)) return VARLEN_ERR_LAUNCH;
+  if (!encode_qkv_map(enc, &tq, q, bf16, total_q, num_heads, D, BM >> pack_log2,
+                      1 << pack_log2))
+    return VARLEN_ERR_LAUNCH;
   if (total_k > 0) {
     if (!encode_qkv_map(enc, &tk, k, bf16, total_k, num_kv_heads, D, BN) ||
         !encode_qkv_map(enc, &tv, v, bf16, total_k, num_kv_heads, D, BN))
@@ -213,7 +214,9 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
   kp.H = num_heads;
   kp.Hkv = num_kv_heads;
   kp.group = group;
-  kp.head_units = use_pair ? num_heads / 2 : num_heads;
+  kp.head_units = pack_log2 ? num_kv_heads : (use_pair ? num_heads / 2 : num_heads);
+  kp.unit_tokens = pack_log2 ? 2 * (BM >> pack_log2) : BM;
+  kp.pack_log2 = pack_log2;
   kp.total_q = (int)total_q;
   kp.total_k = (int)total_k;
   kp.causal = causal ? 1 : 0;
@@ -222,19 +225,13 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
 
   // Upper bound of work items from max_seqlen_q; at least one CTA so that an
   // understated bound never drops work (the CTAs loop over all items).
-  long long max_items = (long long)batch * ((max_seqlen_q + BM - 1) / BM) * kp.head_units;
+  long long max_items =
+      (long long)batch * ((max_seqlen_q + kp.unit_tokens - 1) / kp.unit_tokens) * kp.head_units;
   int grid = dev.sms;
   if (max_items >= 1 && max_items < grid) grid = (int)max_items;
   if (grid < 1) grid = 1;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (use_pair && PAIR_DOUBLE_BUFFERED) {
-    if (D == 64)
-      return bf16 ? launch_pairdb<64, true>(tq, tk, tv, kp, grid, s, dev, 10)
-                  : launch_pairdb<64, false>(tq, tk, tv, kp, grid, s, dev, 11);
-    return bf16 ? launch_pairdb<128, true>(tq, tk, tv, kp, grid, s, dev, 12)
-                : launch_pairdb<128, false>(tq, tk, tv, kp, grid, s, dev, 13);
-  }
   if (use_pair) {
     if (D == 64)
       return bf16 ? launch_pair<64, true>(tq, tk, tv, kp, grid, s, dev, 0)

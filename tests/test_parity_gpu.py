@@ -218,3 +218,24 @@ def test_large_logits_fp16(D):
     case = workloads.make_case([700, 129, 64], None, 8, 2, D, "fp16", True, seed=80 + D,
                                sigma_q=3.0, sigma_k=3.0)
     full_check(case)
+
+
+# --- short queries: GQA-packed tiles (query heads of one key/value head share a tile) ----
+
+@pytest.mark.parametrize("G", [2, 4, 8, 16])
+@pytest.mark.parametrize("causal", [False, True])
+def test_short_queries_gqa_packed(G, causal):
+    rng = np.random.default_rng(100 + G + 10 * causal)
+    lq = [int(x) for x in rng.integers(1, 65, 9)]
+    lk = [int(x) for x in rng.integers(1, 700, 9)]
+    Hkv = 2
+    case = workloads.make_case(lq, lk, Hkv * G, Hkv, 128, "bf16", causal, seed=110 + G)
+    full_check(case)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_short_queries_gqa_packed_fp16(D):
+    lq = [64, 1, 33, 17, 2]
+    lk = [900, 129, 64, 1, 300]
+    case = workloads.make_case(lq, lk, 16, 2, D, "fp16", True, seed=120 + D)
+    full_check(case)
