@@ -57,6 +57,12 @@ def _bind(lib):
     lib.oracle_varlen_attn_rows.restype = i32
     lib.oracle_decode16.argtypes = [ctypes.c_uint16, i32]
     lib.oracle_decode16.restype = f64
+    lib.oracle_varlen_attn_fwd_ext.argtypes = [P, P, P, i32, P, P, P, i32, i32, i32, i32,
+                                               i32, i32, i32, f64, P, P, i32]
+    lib.oracle_varlen_attn_fwd_ext.restype = i32
+    lib.oracle_varlen_attn_rows_ext.argtypes = [P, P, P, i32, P, P, P, i32, i32, i32, i32,
+                                                i32, i32, i32, f64, P, P, i64, P, P, i32]
+    lib.oracle_varlen_attn_rows_ext.restype = i32
     return lib
 
 
@@ -95,9 +101,18 @@ def decode16(bits: int, dtype: str) -> float:
     return _load().oracle_decode16(bits, DTYPE_CODE[dtype])
 
 
+def _seqused(seqused_k):
+    if seqused_k is None:
+        return None, ctypes.c_void_p(0)
+    a = np.ascontiguousarray(np.asarray(seqused_k, dtype=np.int32))
+    return a, _ptr(a)
+
+
 def varlen_attn_fwd(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, nthreads=None,
-                    lib=None):
-    """Full fp64 forward.  Returns (out [Tq,H,D] float64, lse [Tq,H] float64)."""
+                    lib=None, window_left=-1, window_right=-1, seqused_k=None):
+    """Full fp64 forward.  Returns (out [Tq,H,D] float64, lse [Tq,H] float64).
+    window_left/right < 0 mean unbounded; seqused_k (length B) caps the keys
+    of each sequence."""
     lib = lib or _load()
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
@@ -106,17 +121,26 @@ def varlen_attn_fwd(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, nthrea
     Tq = int(cq[-1]) if B >= 0 else 0
     out = np.zeros((Tq, H, D), dtype=np.float64)
     lse = np.zeros((Tq, H), dtype=np.float64)
-    rc = lib.oracle_varlen_attn_fwd(_ptr(qb), _ptr(kb), _ptr(vb), DTYPE_CODE[dtype],
-                                    _ptr(cq), _ptr(ck), B, H, Hkv, D, int(bool(causal)),
-                                    float(scale), _ptr(out), _ptr(lse),
-                                    nthreads or default_threads())
+    keep, su = _seqused(seqused_k)
+    if window_left < 0 and window_right < 0 and seqused_k is None:
+        rc = lib.oracle_varlen_attn_fwd(_ptr(qb), _ptr(kb), _ptr(vb), DTYPE_CODE[dtype],
+                                        _ptr(cq), _ptr(ck), B, H, Hkv, D, int(bool(causal)),
+                                        float(scale), _ptr(out), _ptr(lse),
+                                        nthreads or default_threads())
+    else:
+        rc = lib.oracle_varlen_attn_fwd_ext(_ptr(qb), _ptr(kb), _ptr(vb), DTYPE_CODE[dtype],
+                                            _ptr(cq), _ptr(ck), su, B, H, Hkv, D,
+                                            int(bool(causal)), int(window_left),
+                                            int(window_right), float(scale), _ptr(out),
+                                            _ptr(lse), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError("oracle_varlen_attn_fwd failed with code %d" % rc)
     return out, lse
 
 
 def varlen_attn_rows(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, rows,
-                     nthreads=None, lib=None):
+                     nthreads=None, lib=None, window_left=-1, window_right=-1,
+                     seqused_k=None):
     """fp64 forward of selected rows.  rows: int array [n, 2] of (token, head).
     Returns (out [n, D], lse [n])."""
     lib = lib or _load()
@@ -129,23 +153,26 @@ def varlen_attn_rows(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, rows,
     n = rows.shape[0]
     out = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
-    rc = lib.oracle_varlen_attn_rows(_ptr(qb), _ptr(kb), _ptr(vb), DTYPE_CODE[dtype],
-                                     _ptr(cq), _ptr(ck), len(cq) - 1, H, Hkv, D,
-                                     int(bool(causal)), float(scale), _ptr(tok), _ptr(head),
-                                     n, _ptr(out), _ptr(lse), nthreads or default_threads())
+    keep, su = _seqused(seqused_k)
+    rc = lib.oracle_varlen_attn_rows_ext(_ptr(qb), _ptr(kb), _ptr(vb), DTYPE_CODE[dtype],
+                                         _ptr(cq), _ptr(ck), su, len(cq) - 1, H, Hkv, D,
+                                         int(bool(causal)), int(window_left), int(window_right),
+                                         float(scale), _ptr(tok), _ptr(head), n, _ptr(out),
+                                         _ptr(lse), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError("oracle_varlen_attn_rows failed with code %d" % rc)
     return out, lse
 
 
-def run_case(case, nthreads=None, lib=None):
-    """Full oracle forward of a ``workloads.Case``."""
+def run_case(case, nthreads=None, lib=None, **mask):
+    """Full oracle forward of a ``workloads.Case`` (mask: window_left,
+    window_right, seqused_k)."""
     return varlen_attn_fwd(case.q, case.k, case.v, case.cu_q.numpy(), case.cu_k.numpy(),
                            case.H, case.Hkv, case.D, case.causal, case.scale, case.dtype,
-                           nthreads, lib=lib)
+                           nthreads, lib=lib, **mask)
 
 
-def run_case_rows(case, rows, nthreads=None):
+def run_case_rows(case, rows, nthreads=None, **mask):
     return varlen_attn_rows(case.q, case.k, case.v, case.cu_q.numpy(), case.cu_k.numpy(),
                             case.H, case.Hkv, case.D, case.causal, case.scale, case.dtype,
-                            rows, nthreads)
+                            rows, nthreads, **mask)

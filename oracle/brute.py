@@ -26,8 +26,12 @@ def segment_ids(cu: np.ndarray) -> np.ndarray:
 
 
 def dense_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_q, cu_k, causal: bool,
-                  scale: float):
-    """q [Tq,H,D], k/v [Tk,Hkv,D] float64.  Returns (out [Tq,H,D], lse [Tq,H])."""
+                  scale: float, window_left: int = -1, window_right: int = -1,
+                  seqused_k=None):
+    """q [Tq,H,D], k/v [Tk,Hkv,D] float64.  Returns (out [Tq,H,D], lse [Tq,H]).
+    Optional sliding window (sequence-local: key ki visible to query qi only
+    if qi - left <= ki <= qi + right, negative = unbounded) and per-sequence
+    used-key counts; rows without a visible key give O = 0, LSE = -inf."""
     Tq, H, D = q.shape
     Tk, Hkv, _ = k.shape
     G = H // Hkv
@@ -36,6 +40,13 @@ def dense_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_q, cu_k, causa
     visible = sq[:, None] == sk[None, :]
     if causal:
         visible &= ~(pq[:, None] < pk[None, :])
+    if window_left >= 0:
+        visible &= pk[None, :] >= pq[:, None] - window_left
+    if window_right >= 0:
+        visible &= pk[None, :] <= pq[:, None] + window_right
+    if seqused_k is not None:
+        used = np.asarray(seqused_k, dtype=np.int64)[sk]
+        visible &= (pk < used)[None, :]
     out = np.zeros((Tq, H, D))
     lse = np.full((Tq, H), -np.inf)
     for h in range(H):

@@ -24,6 +24,14 @@
  * LSE [Tq, H], all row-major.  The scale is an explicit argument; a value
  * <= 0 or NaN selects the page's default 1/sqrt(D).
  *
+ * Extension (the `_ext` entry points): the sliding window and used-key count
+ * that PyTorch pull request #176015 lists in the varlen forward schema
+ * (window_size_left, window_size_right, seqused_k), read with the page's
+ * sequence-local indices: key ki is also hidden when ki >= seqused_k[b]
+ * (clipped to [0, Lk_b]), when left >= 0 and ki < qi - left, or when
+ * right >= 0 and ki > qi + right.  A row with no visible key gets O = 0 and
+ * LSE = -inf, what the page's loop gives for a sequence without keys.
+ *
  * Inputs are bf16 or fp16 bit patterns; they are widened exactly to double
  * before any arithmetic.  The widening of a key/value head of one sequence
  * is done once per (b, h) work item; that is a format conversion, not a
@@ -73,7 +81,9 @@ typedef struct {
     const uint16_t *q, *k, *v;
     int dtype;
     const int32_t *cu_q, *cu_k;
+    const int32_t *seqused_k; /* NULL: every key of the sequence */
     int B, H, Hkv, D, causal;
+    int win_left, win_right;  /* < 0: unbounded */
     double scale;
     /* full mode */
     double *out, *lse;
@@ -93,6 +103,25 @@ static double effective_scale(double scale, int D) {
     return scale;
 }
 
+/* Keys of sequence b that exist for attention: Lk_b, or seqused_k[b] when
+ * given (clipped to [0, Lk_b]). */
+static int used_keys(const OracleCtx *c, int b) {
+    int Lk = c->cu_k[b + 1] - c->cu_k[b];
+    if (c->seqused_k) {
+        int u = c->seqused_k[b];
+        if (u < 0) u = 0;
+        if (u < Lk) Lk = u;
+    }
+    return Lk;
+}
+
+static int key_hidden(const OracleCtx *c, int qi, int ki) {
+    if (c->causal && qi < ki) return 1;
+    if (c->win_left >= 0 && ki < qi - c->win_left) return 1;
+    if (c->win_right >= 0 && ki > qi + c->win_right) return 1;
+    return 0;
+}
+
 /* One query row: the page's two-pass softmax, in double precision.
  * kd/vd hold the widened keys/values of head kv_h of sequence b, [Lk][D]. */
 static void oracle_attend_row(const OracleCtx *c, const double *qrow, int qi, int Lk,
@@ -101,7 +130,7 @@ static void oracle_attend_row(const OracleCtx *c, const double *qrow, int qi, in
     const int D = c->D;
     double max_score = -INFINITY;
     for (int ki = 0; ki < Lk; ++ki) {
-        if (c->causal && qi < ki) {
+        if (key_hidden(c, qi, ki)) {
             scores[ki] = -INFINITY;
             continue;
         }
@@ -111,6 +140,11 @@ static void oracle_attend_row(const OracleCtx *c, const double *qrow, int qi, in
         double s = dot * c->scale;
         if (s > max_score) max_score = s;
         scores[ki] = s;
+    }
+    if (max_score == -INFINITY) { /* no visible key */
+        for (int d = 0; d < D; ++d) out_row[d] = 0.0;
+        *lse_out = -INFINITY;
+        return;
     }
     double sum_exp = 0.0;
     for (int ki = 0; ki < Lk; ++ki) {
@@ -174,7 +208,7 @@ static void *full_worker(void *arg) {
         int b = (int)(item / H), h = (int)(item % H);
         int kv_h = h / G;
         int q0 = c->cu_q[b], Lq = c->cu_q[b + 1] - c->cu_q[b];
-        int Lk = c->cu_k[b + 1] - c->cu_k[b];
+        int Lk = used_keys(c, b);
         if (Lq <= 0) continue;
         widen_kv(c, b, kv_h, kd, vd);
         for (int qi = 0; qi < Lq; ++qi) {
@@ -224,7 +258,7 @@ static void *rows_worker(void *arg) {
         int b = find_seq(c, tok);
         int kv_h = h / G;
         int qi = (int)(tok - c->cu_q[b]);
-        int Lk = c->cu_k[b + 1] - c->cu_k[b];
+        int Lk = used_keys(c, b);
         if (b != cached_b || kv_h != cached_kvh) {
             widen_kv(c, b, kv_h, kd, vd);
             cached_b = b;
@@ -261,38 +295,62 @@ static int check_args(int B, int H, int Hkv, int D, int dtype) {
 
 /* Full forward: writes out[Tq*H*D] and lse[Tq*H] (Tq = cu_q[B]).
  * Returns 0, or a negative code on bad arguments / allocation failure. */
-int oracle_varlen_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int dtype,
-                           const int32_t *cu_q, const int32_t *cu_k, int B, int H, int Hkv,
-                           int D, int causal, double scale, double *out, double *lse,
-                           int nthreads) {
+int oracle_varlen_attn_fwd_ext(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                               int dtype, const int32_t *cu_q, const int32_t *cu_k,
+                               const int32_t *seqused_k, int B, int H, int Hkv, int D, int causal,
+                               int win_left, int win_right, double scale, double *out,
+                               double *lse, int nthreads) {
     int rc = check_args(B, H, Hkv, D, dtype);
     if (rc) return rc;
     OracleCtx c;
     memset(&c, 0, sizeof c);
     c.q = q; c.k = k; c.v = v; c.dtype = dtype; c.cu_q = cu_q; c.cu_k = cu_k;
+    c.seqused_k = seqused_k;
     c.B = B; c.H = H; c.Hkv = Hkv; c.D = D; c.causal = causal != 0;
+    c.win_left = win_left; c.win_right = win_right;
     c.scale = effective_scale(scale, D);
     c.out = out; c.lse = lse;
     c.n_items = (int64_t)B * H;
     return run_threads(&c, full_worker, nthreads);
 }
 
+int oracle_varlen_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int dtype,
+                           const int32_t *cu_q, const int32_t *cu_k, int B, int H, int Hkv,
+                           int D, int causal, double scale, double *out, double *lse,
+                           int nthreads) {
+    return oracle_varlen_attn_fwd_ext(q, k, v, dtype, cu_q, cu_k, NULL, B, H, Hkv, D, causal,
+                                      -1, -1, scale, out, lse, nthreads);
+}
+
 /* Selected rows: for i in [0, nrows) computes the output row of packed query
  * token row_tok[i], head row_head[i] into out_rows[i*D..] and lse_rows[i]. */
-int oracle_varlen_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int dtype,
-                            const int32_t *cu_q, const int32_t *cu_k, int B, int H, int Hkv,
-                            int D, int causal, double scale, const int64_t *row_tok,
-                            const int32_t *row_head, int64_t nrows, double *out_rows,
-                            double *lse_rows, int nthreads) {
+int oracle_varlen_attn_rows_ext(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                int dtype, const int32_t *cu_q, const int32_t *cu_k,
+                                const int32_t *seqused_k, int B, int H, int Hkv, int D,
+                                int causal, int win_left, int win_right, double scale,
+                                const int64_t *row_tok, const int32_t *row_head, int64_t nrows,
+                                double *out_rows, double *lse_rows, int nthreads) {
     int rc = check_args(B, H, Hkv, D, dtype);
     if (rc) return rc;
     if (B < 1) return -2;
     OracleCtx c;
     memset(&c, 0, sizeof c);
     c.q = q; c.k = k; c.v = v; c.dtype = dtype; c.cu_q = cu_q; c.cu_k = cu_k;
+    c.seqused_k = seqused_k;
     c.B = B; c.H = H; c.Hkv = Hkv; c.D = D; c.causal = causal != 0;
+    c.win_left = win_left; c.win_right = win_right;
     c.scale = effective_scale(scale, D);
     c.row_tok = row_tok; c.row_head = row_head; c.nrows = nrows;
     c.out_rows = out_rows; c.lse_rows = lse_rows;
     return run_threads(&c, rows_worker, nthreads);
+}
+
+int oracle_varlen_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int dtype,
+                            const int32_t *cu_q, const int32_t *cu_k, int B, int H, int Hkv,
+                            int D, int causal, double scale, const int64_t *row_tok,
+                            const int32_t *row_head, int64_t nrows, double *out_rows,
+                            double *lse_rows, int nthreads) {
+    return oracle_varlen_attn_rows_ext(q, k, v, dtype, cu_q, cu_k, NULL, B, H, Hkv, D, causal,
+                                       -1, -1, scale, row_tok, row_head, nrows, out_rows,
+                                       lse_rows, nthreads);
 }

@@ -263,7 +263,7 @@ def test_empty_key_set_and_empty_query():
 # --- the pins catch planted mistakes ------------------------------------------------------
 
 MUTANTS = {
-    "causal_off_by_one": ("if (c->causal && qi < ki)", "if (c->causal && qi <= ki)"),
+    "causal_off_by_one": ("if (c->causal && qi < ki) return 1;", "if (c->causal && qi <= ki) return 1;"),
     "gqa_map_modulo": ("int kv_h = h / G;\n        int q0", "int kv_h = h % G;\n        int q0"),
     "dropped_scale": ("double s = dot * c->scale;", "double s = dot;"),
     "lse_without_max": ("*lse_out = max_score + log(sum_exp);", "*lse_out = log(sum_exp);"),
