@@ -41,8 +41,19 @@ KERNEL_DIR = "flash_attention_fwd_b200/csrc"
 
 # ----------------------------------------------------------------------------- counting
 
-def visible_keys(lq: int, lk: int, causal: bool) -> int:
-    """Unmasked (query, key) pairs of one sequence and one head."""
+def visible_keys(lq: int, lk: int, causal: bool, window_left: int = -1,
+                 window_right: int = -1, used=None) -> int:
+    """Unmasked (query, key) pairs of one sequence and one head: key ki is
+    visible to query qi iff ki < min(lk, used), qi - left <= ki (left >= 0),
+    ki <= qi + right (right >= 0) and not (causal and qi < ki)."""
+    if used is not None:
+        lk = min(lk, max(int(used), 0))
+    if window_left >= 0 or window_right >= 0:
+        qi = np.arange(lq, dtype=np.int64)
+        lo = np.maximum(0, qi - window_left) if window_left >= 0 else np.zeros_like(qi)
+        r = 0 if causal else window_right
+        hi = np.minimum(lk, qi + r + 1) if r >= 0 else np.full_like(qi, lk)
+        return int(np.maximum(0, hi - lo).sum())
     if not causal:
         return lq * lk
     # query qi sees keys 0..min(qi, lk-1): min(qi+1, lk) keys
@@ -51,18 +62,31 @@ def visible_keys(lq: int, lk: int, causal: bool) -> int:
     return full + max(0, lq - lk) * lk
 
 
-def unmasked_pairs(lens_q, lens_k, H: int, causal: bool) -> int:
-    return H * sum(visible_keys(a, b, causal) for a, b in zip(lens_q, lens_k))
+def unmasked_pairs(lens_q, lens_k, H: int, causal: bool, mask=None) -> int:
+    mask = mask or {}
+    used = mask.get("seqused_k") or [None] * len(lens_q)
+    return H * sum(visible_keys(a, b, causal, mask.get("window_left", -1),
+                                mask.get("window_right", -1), u)
+                   for a, b, u in zip(lens_q, lens_k, used))
 
 
 def step_flops(case) -> int:
-    return 4 * case.D * unmasked_pairs(case.lens_q, case.lens_k, case.H, case.causal)
+    return 4 * case.D * unmasked_pairs(case.lens_q, case.lens_k, case.H, case.causal, case.mask)
+
+
+def used_keys(case) -> int:
+    """Keys a step must read: all of them, or the used counts with seqused_k."""
+    used = case.mask.get("seqused_k")
+    if used is None:
+        return case.Tk
+    return sum(min(lk, max(u, 0)) for lk, u in zip(case.lens_k, used))
 
 
 def algorithmic_bytes(case) -> int:
     e = 2
-    return (case.Tq * case.H * case.D * e * 2 + 2 * case.Tk * case.Hkv * case.D * e
-            + 4 * case.Tq * case.H + 8 * (case.B + 1))
+    return (case.Tq * case.H * case.D * e * 2 + 2 * used_keys(case) * case.Hkv * case.D * e
+            + 4 * case.Tq * case.H + 8 * (case.B + 1)
+            + (4 * case.B if "seqused_k" in case.mask else 0))
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -182,7 +206,15 @@ def oracle_sample_rows(case, n_rows: int, seed: int = 99):
     b = b[order]
     qi = rows[:, 0] - cu[b]
     lk = np.asarray(case.lens_k)[b]
-    vis = np.minimum(qi + 1, lk) if case.causal else lk
+    m = case.mask
+    if m.get("seqused_k") is not None:
+        lk = np.minimum(lk, np.maximum(np.asarray(m["seqused_k"])[b], 0))
+    left, right = m.get("window_left", -1), m.get("window_right", -1)
+    if case.causal:
+        right = 0
+    lo = np.maximum(0, qi - left) if left >= 0 else np.zeros_like(qi)
+    hi = np.minimum(lk, qi + right + 1) if right >= 0 else lk
+    vis = np.maximum(0, hi - lo)
     flops = int(4 * case.D * int(vis.sum()))
     return rows, flops
 
@@ -194,13 +226,13 @@ def time_oracle(case, seconds: float, nthreads: int | None = None):
     nthreads = nthreads or oracle.default_threads()
     rows, fl = oracle_sample_rows(case, 256, seed=98)
     t0 = time.perf_counter()
-    oracle.run_case_rows(case, rows, nthreads=nthreads)
+    oracle.run_case_rows(case, rows, nthreads=nthreads, **case.mask)
     rate = fl / max(time.perf_counter() - t0, 1e-6)
     avg_row = fl / max(len(rows), 1)
     n = int(max(64, min(2_000_000, seconds * rate / max(avg_row, 1))))
     rows, fl = oracle_sample_rows(case, n, seed=99)
     t0 = time.perf_counter()
-    oracle.run_case_rows(case, rows, nthreads=nthreads)
+    oracle.run_case_rows(case, rows, nthreads=nthreads, **case.mask)
     dt = time.perf_counter() - t0
     return fl / dt / 1e12, len(rows), fl, dt, nthreads
 
@@ -246,9 +278,14 @@ def run_gpu(args, rank: int, world: int):
     fa.load_library()
     fa.device_status(clear=True)
 
+    used = case.mask.get("seqused_k")
+    used_t = None if used is None else torch.tensor(used, dtype=torch.int32, device=dev)
+    wl, wr = case.mask.get("window_left", -1), case.mask.get("window_right", -1)
+
     def step():
         fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, case.causal, case.scale,
-                           out=out, lse=lse, stream=stream)
+                           out=out, lse=lse, stream=stream, window_size_left=wl,
+                           window_size_right=wr, seqused_k=used_t)
 
     for _ in range(args.warmup):
         step()
@@ -279,7 +316,8 @@ def run_gpu(args, rank: int, world: int):
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
     else:
-        e2e_ms, h2d, d2h = run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist)
+        e2e_ms, h2d, d2h = run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist,
+                                   extra=[used_t] if used_t is not None else [])
 
     if dist:
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
@@ -289,13 +327,14 @@ def run_gpu(args, rank: int, world: int):
         dist.destroy_process_group()
 
 
-def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist):
+def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist, extra=()):
     import torch
     hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
     hcq, hck = case.cu_q.pin_memory(), case.cu_k.pin_memory()
     ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck))
+    hx = [t.cpu().pin_memory() for t in extra]  # further inputs (seqused_k)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck, *hx))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     def e2e_step():
@@ -304,6 +343,8 @@ def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist):
         v.copy_(hv, non_blocking=True)
         cq.copy_(hcq, non_blocking=True)
         ck.copy_(hck, non_blocking=True)
+        for d, h in zip(extra, hx):
+            d.copy_(h, non_blocking=True)
         step()
         ho.copy_(out, non_blocking=True)
         hl.copy_(lse, non_blocking=True)
@@ -350,6 +391,8 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
                 "name": args.workload, "batch_sequences": case.B, "total_q": case.Tq,
                 "total_k": case.Tk, "max_seqlen": case.max_q, "H": case.H, "Hkv": case.Hkv,
                 "D": case.D, "causal": case.causal, "flops_per_step": flops,
+                "window": [case.mask.get("window_left", -1), case.mask.get("window_right", -1)],
+                "seqused_k": "seqused_k" in case.mask,
                 "l2": "no flush: inputs (%.0f MB) exceed the 126 MB L2"
                       % (algorithmic_bytes(case) / 1e6),
                 "parallelism": "dp%d (one independent batch per GPU)" % world},
@@ -387,15 +430,15 @@ def run_reference(args, rank: int, world: int):
     budget = max(0.5, min(30.0, args.reference_seconds / max(1, args.steps + args.warmup)))
     rows0, fl0 = oracle_sample_rows(case, 256, seed=98)
     t0 = time.perf_counter()
-    oracle.run_case_rows(case, rows0, nthreads=nthreads)
+    oracle.run_case_rows(case, rows0, nthreads=nthreads, **case.mask)
     rate = fl0 / max(time.perf_counter() - t0, 1e-6)
     n = int(max(64, budget * rate / max(fl0 / len(rows0), 1)))
     rows, fl = oracle_sample_rows(case, n, seed=99)
     for _ in range(args.warmup):
-        oracle.run_case_rows(case, rows, nthreads=nthreads)
+        oracle.run_case_rows(case, rows, nthreads=nthreads, **case.mask)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.run_case_rows(case, rows, nthreads=nthreads)
+        oracle.run_case_rows(case, rows, nthreads=nthreads, **case.mask)
     dt = (time.perf_counter() - t0) / args.steps
     value = fl / dt / 1e12
     line = {

@@ -37,6 +37,7 @@ STATUS_NAMES = {
 # Every symbol include/varlen_attn.h declares.
 EXPORTED_SYMBOLS = (
     "varlen_attn_fwd_v1",
+    "varlen_attn_fwd_v2",
     "varlen_attn_fwd",
     "varlen_attn_strerror",
     "varlen_attn_device_status",
@@ -61,6 +62,9 @@ def _bind(lib):
         fn = getattr(lib, name)
         fn.argtypes = fwd_args
         fn.restype = i32
+    # v2: v1's arguments with window_left, window_right, seqused_k after scale
+    lib.varlen_attn_fwd_v2.argtypes = fwd_args[:15] + [i32, i32, P] + fwd_args[15:]
+    lib.varlen_attn_fwd_v2.restype = i32
     lib.varlen_attn_strerror.argtypes = [i32]
     lib.varlen_attn_strerror.restype = ctypes.c_char_p
     lib.varlen_attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i32]
@@ -110,16 +114,21 @@ def varlen_attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, cu_q_ptr: int, cu_k_
                         batch: int, total_q: int, total_k: int, max_seqlen_q: int,
                         max_seqlen_k: int, num_heads: int, num_kv_heads: int, head_dim: int,
                         causal: bool, scale: float, dtype_code: int, out_ptr: int,
-                        lse_ptr: int, stream: int) -> int:
+                        lse_ptr: int, stream: int, window_left: int = -1,
+                        window_right: int = -1, seqused_k_ptr: int = 0) -> int:
     """Direct call of the C entry point with integer addresses; returns the
-    status code unchanged."""
+    status code unchanged.  Calls varlen_attn_fwd (v1) unless a window bound
+    or a seqused_k array is given, varlen_attn_fwd_v2 otherwise."""
     lib = load_library()
     V = ctypes.c_void_p
-    return lib.varlen_attn_fwd(V(q_ptr), V(k_ptr), V(v_ptr), V(cu_q_ptr), V(cu_k_ptr),
-                               int(batch), int(total_q), int(total_k), int(max_seqlen_q),
-                               int(max_seqlen_k), int(num_heads), int(num_kv_heads),
-                               int(head_dim), int(bool(causal)), float(scale), int(dtype_code),
-                               V(out_ptr), V(lse_ptr), V(stream))
+    head = (V(q_ptr), V(k_ptr), V(v_ptr), V(cu_q_ptr), V(cu_k_ptr), int(batch), int(total_q),
+            int(total_k), int(max_seqlen_q), int(max_seqlen_k), int(num_heads),
+            int(num_kv_heads), int(head_dim), int(bool(causal)), float(scale))
+    tail = (int(dtype_code), V(out_ptr), V(lse_ptr), V(stream))
+    if window_left < 0 and window_right < 0 and not seqused_k_ptr:
+        return lib.varlen_attn_fwd(*head, *tail)
+    return lib.varlen_attn_fwd_v2(*head, int(window_left), int(window_right),
+                                  V(seqused_k_ptr), *tail)
 
 
 def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -127,7 +136,9 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,
                     scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                     lse: Optional[torch.Tensor] = None,
-                    stream: Optional[torch.cuda.Stream] = None
+                    stream: Optional[torch.cuda.Stream] = None,
+                    window_size_left: int = -1, window_size_right: int = -1,
+                    seqused_k: Optional[torch.Tensor] = None
                     ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Packed attention forward on the GPU.
 
@@ -135,6 +146,11 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     device); cu_seqlens_q/k int32 [B+1] on the same device.  Writes ``out``
     ([Tq, H, D], q's dtype) and ``lse`` ([Tq, H], float32) — allocated here
     when not given — and returns them.  ``scale=None`` selects 1/sqrt(D).
+    ``window_size_left/right`` (negative = unbounded) and ``seqused_k`` (int32
+    [B] on the device, or None) restrict the visible keys as in the varlen
+    forward schema of PyTorch pull request #176015: key ki is visible to query
+    qi iff ki < min(Lk, seqused_k[b]), qi - left <= ki <= qi + right, and
+    not (causal and qi < ki).
     """
     if q.dtype not in DTYPE_CODES or k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share dtype bfloat16 or float16")
@@ -160,6 +176,11 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         raise ValueError("out must be a contiguous tensor shaped and typed like q")
     if lse.shape != (total_q, H) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 tensor [Tq, H]")
+    if seqused_k is not None:
+        if (not seqused_k.is_cuda or not seqused_k.is_contiguous()
+                or seqused_k.dtype != torch.int32
+                or seqused_k.numel() != cu_seqlens_q.numel() - 1):
+            raise ValueError("seqused_k must be a contiguous int32 CUDA tensor [B]")
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     with torch.cuda.device(q.device):
@@ -169,7 +190,8 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), H, Hkv, D, causal,
             0.0 if scale is None else float(scale), DTYPE_CODES[q.dtype],
             out.data_ptr() if out.numel() else 0, lse.data_ptr() if lse.numel() else 0,
-            stream.cuda_stream)
+            stream.cuda_stream, int(window_size_left), int(window_size_right),
+            seqused_k.data_ptr() if seqused_k is not None and seqused_k.numel() else 0)
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return out, lse

@@ -43,18 +43,33 @@ struct KParams {
                          // BM >> k tokens x the 2^k query heads of one key/value head
   int total_q, total_k;
   int causal;
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;      // scale * log2(e)
+  const int *seqused_k;  // optional [B]: keys of sequence b used = min(Lk_b, seqused_k[b])
+  int win_left;          // key ki visible to query qi only if ki >= qi - win_left (-1: no bound)
+  int win_right;         // ... and ki <= qi + win_right (-1: no bound); the causal rule is
+                         // folded in by the host (causal => win_right = 0)
 };
+
+// Visible keys [key_lo, key_hi) of the sequence-local query qi in a sequence
+// with Lk used keys (empty when key_hi <= key_lo).
+__device__ __forceinline__ int key_lo(const KParams &p, int qi) {
+  return p.win_left >= 0 ? max(0, qi - p.win_left) : 0;
+}
+__device__ __forceinline__ int key_hi(const KParams &p, int qi, int Lk) {
+  return p.win_right >= 0 ? (int)min((long long)Lk, (long long)qi + p.win_right + 1) : Lk;
+}
 
 struct WorkItem {
   int hu;       // head unit (a head, a pair of heads 2hu, 2hu+1, or a key/value head)
   int q0;       // packed index of the item's first query token
   int q_rows;   // valid query tokens in the item (<= unit_tokens)
   int qi0;      // sequence-local index of the item's first query
-  int k0;       // packed index of the sequence's first key
-  int Lk;       // keys in the sequence
+  int k0;       // packed index of the first key of the first visited key tile
+  int kofs;     // sequence-local index of that key (a multiple of the key tile)
+  int Lk;       // used keys in the sequence
   int n_kv;     // key tiles to visit
-  int min_lim;  // smallest per-row visible-key bound in the tile
+  int min_hi;   // smallest per-row visible-key end, relative to kofs
+  int max_lo;   // largest per-row visible-key start, relative to kofs
 };
 
 // ---------------------------------------------------------------------------
@@ -69,13 +84,19 @@ struct WorkItem {
 // CTAs and the K/V tiles are served from L2).  Item i goes to CTA i mod G, the
 // direction reversed every round, so each CTA gets a near-equal sum of costs.
 //
+// With per-sequence used-key counts Lk means the used keys.  A sliding
+// window changes which key tiles an item visits (the range [lo, hi) spanned
+// by its rows' visible keys) but not the ordering, which stays the one above:
+// the windowed cost is nearly the same for all ranges of a sequence, so the
+// dealing still balances.
+//
 // The walk is warp-cooperative (all 32 lanes of the calling warp call
 // init/next together): sequences are examined 32 at a time.  Lengths are
 // clamped into the buffers' extents, so an inconsistent sequence table can
 // never address memory outside them.
 template <int BN>
 struct Scheduler {
-  const int *cu_q, *cu_k;
+  const int *cu_q, *cu_k, *seqused_k;
   int B, HU, U, R, causal, total_q, total_k;
   int cta, grid, lane;
   long long round;
@@ -96,6 +117,7 @@ struct Scheduler {
     ke = min(max(ke, ks), total_k);
     lq = qe - qs;
     lk = ke - ks;
+    if (seqused_k) lk = min(lk, max(__ldg(seqused_k + b), 0));
   }
   // (sequence, query range) units of a sequence at cost level c; nq ranges of
   // U tokens, nk tiles of BM keys
@@ -133,6 +155,7 @@ struct Scheduler {
   __device__ void init(const KParams &p) {
     cu_q = p.cu_q;
     cu_k = p.cu_k;
+    seqused_k = p.seqused_k;
     B = p.B;
     HU = p.head_units;
     U = p.unit_tokens;
@@ -162,7 +185,7 @@ struct Scheduler {
     cur_units = 0;
   }
 
-  __device__ bool next(WorkItem &w) {
+  __device__ bool next(WorkItem &w, const KParams &p) {
     const long long idx = round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
     ++round;
     while (level >= 0 && idx >= level_base + level_items) {
@@ -207,11 +230,15 @@ struct Scheduler {
         w.qi0 = qt * U;
         w.q0 = qs + w.qi0;
         w.q_rows = min(U, lq - w.qi0);
-        w.k0 = ks;
         w.Lk = lk;
-        const int kv_end = causal ? min(lk, min(lq, w.qi0 + U)) : lk;
-        w.n_kv = (kv_end + BN - 1) / BN;
-        w.min_lim = causal ? min(lk, w.qi0 + 1) : lk;
+        // key tiles spanned by the visible keys of the first and last query
+        const int qa = w.qi0, qb = w.qi0 + w.q_rows - 1;
+        const int lo_a = key_lo(p, qa), hi_b = key_hi(p, qb, lk);
+        w.kofs = (lo_a / BN) * BN;
+        w.k0 = ks + w.kofs;
+        w.n_kv = hi_b > lo_a ? (hi_b - w.kofs + BN - 1) / BN : 0;
+        w.min_hi = key_hi(p, qa, lk) - w.kofs;
+        w.max_lo = key_lo(p, qb) - w.kofs;
         return true;
       }
       cur_b += 32;
@@ -336,6 +363,23 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
 #define SOFTMAX_POLY_EVERY 0
 #endif
 
+// Running-max update of one row for key tile j, mx = the tile's row max in
+// log2 units (-inf when every key of the tile is hidden from the row).  m
+// stays -inf until the row has seen a visible key; the first finite max then
+// "rescales" O and l by exp2(-inf) = 0, which is exact because both are 0.
+__device__ __forceinline__ void update_max(int j, float mx, float &m, float &alpha, bool &need) {
+  if (j == 0) {
+    m = mx;
+  } else if (mx > m + RESCALE_THRESHOLD) {
+    alpha = ptx::ex2_approx(m - mx);
+    m = mx;
+    need = true;
+  }
+}
+// Offset added to the scaled scores before exp2: -m, or 0 while m = -inf (the
+// row has no visible key yet, every score is -inf and exp2 gives 0).
+__device__ __forceinline__ float exp_offset(float m) { return m == -INFINITY ? 0.f : -m; }
+
 // ---------------------------------------------------------------------------
 // Softmax of one S tile held in TMEM (one row per thread), written back as P
 // (bf16/fp16) over the first BN/2 columns of the same TMEM region.
@@ -352,7 +396,7 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
 // Returns false when that wait gave up.
 template <int BN, int D, bool BF16, class WaitO>
 __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, float sl2,
-                                             bool need_mask, int lim, float &m, float &l,
+                                             bool need_mask, int lo, int hi, float &m, float &l,
                                              WaitO &&wait_o) {
   constexpr int POLY = SOFTMAX_POLY_EVERY;
   constexpr int DEG = BF16 ? 3 : 4;
@@ -364,7 +408,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, fl
   if (need_mask) {
 #pragma unroll
     for (int c = 0; c < BN; ++c)
-      if (c >= lim) s[c] = -INFINITY;
+      if (c < lo || c >= hi) s[c] = -INFINITY;
   }
   // Row max: four independent chains of three-input maxima.
   float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
@@ -380,15 +424,10 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, fl
   const float mx = fmaxf(ptx::fmax3(mx0, mx1, mx2), mx3) * sl2;
   float alpha = 1.f;
   bool need = false;
-  if (j == 0) {
-    m = (mx == -INFINITY) ? 0.f : mx;
-  } else if (mx > m + RESCALE_THRESHOLD) {
-    alpha = ptx::ex2_approx(m - mx);
-    m = mx;
-    need = true;
-  }
+  update_max(j, mx, m, alpha, need);
   const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
-  const uint64_t negm_2 = ptx::f2_pack(-m, -m);
+  const float negm = exp_offset(m);
+  const uint64_t negm_2 = ptx::f2_pack(negm, negm);
   float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
 #pragma unroll
   for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -442,12 +481,15 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, fl
 }
 
 // Epilogue of one row: O / l -> out (bf16/fp16, 16-byte stores), LSE -> lse.
-// Arrives on o_free (one arrival per warp) as soon as O has been read.
+// A row that saw no visible key (l = 0; O is then 0 too) gets O = 0 and
+// LSE = -inf.  Arrives on o_free (one arrival per warp) as soon as O has been
+// read.
 template <int D, bool BF16>
 __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, bool row_valid,
                                              uint16_t *orow_ptr, float *lse_ptr,
                                              uint64_t *o_free, int lane) {
-  const float inv_l = 1.f / l;
+  const bool any = l > 0.f;
+  const float inv_l = any ? 1.f / l : 0.f;
 #pragma unroll
   for (int c0 = 0; c0 < D; c0 += 32) {
     uint32_t o[32];
@@ -468,7 +510,7 @@ __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, bool
         dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
     }
   }
-  if (row_valid) *lse_ptr = (m + log2f(l)) * 0.69314718055994530942f;
+  if (row_valid) *lse_ptr = any ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
 }
 
 // A query row whose sequence has no key: O = 0, LSE = -inf.

@@ -99,8 +99,9 @@ constexpr size_t smem_bytes() {
 // the first chunk is signalled.
 template <int D, bool BF16, class Loaded, class ChunkReady>
 __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, int j, float sl2,
-                                                     bool need_mask, int lim, float &m, float &l,
-                                                     Loaded &&loaded, ChunkReady &&chunk_ready) {
+                                                     bool need_mask, int lo, int hi, float &m,
+                                                     float &l, Loaded &&loaded,
+                                                     ChunkReady &&chunk_ready) {
   uint32_t sr[BN];
   tmem_ld_wait<BN>(tS, sr);
   loaded();
@@ -110,7 +111,7 @@ __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, i
   if (need_mask) {
 #pragma unroll
     for (int c = 0; c < BN; ++c)
-      if (c >= lim) s[c] = -INFINITY;
+      if (c < lo || c >= hi) s[c] = -INFINITY;
   }
   float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
@@ -125,13 +126,7 @@ __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, i
   const float mx = fmaxf(ptx::fmax3(mx0, mx1, mx2), mx3) * sl2;
   float alpha = 1.f;
   bool need = false;
-  if (j == 0) {
-    m = (mx == -INFINITY) ? 0.f : mx;
-  } else if (mx > m + RESCALE_THRESHOLD) {
-    alpha = ptx::ex2_approx(m - mx);
-    m = mx;
-    need = true;
-  }
+  update_max(j, mx, m, alpha, need);
   if (__any_sync(0xffffffffu, need)) {
     // 16-column pieces: the whole S row is still live here
     const uint64_t a2 = ptx::f2_pack(alpha, alpha);
@@ -152,7 +147,8 @@ __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, i
     }
   }
   const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
-  const uint64_t negm_2 = ptx::f2_pack(-m, -m);
+  const float negm = exp_offset(m);
+  const uint64_t negm_2 = ptx::f2_pack(negm, negm);
   float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
 #pragma unroll
   for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -312,7 +308,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       for (;;) {
         WorkItem w;
-        const bool have = sched.next(w);
+        const bool have = sched.next(w, p);
         if (!have) w.hu = -1;
         if (lane == 0) {
           ok = wait_bar(&bars->ring.empty[rs], rph ^ 1u, abort_flag);
@@ -496,7 +492,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (row_valid) empty_row<D>(orow_ptr, p.lse + orow);
         continue;
       }
-      const int key_lim = p.causal ? min(w.Lk, qi + 1) : w.Lk;
+      // visible keys of this row, relative to the first visited key tile
+      const int lo = key_lo(p, qi) - w.kofs;
+      const int hi = key_hi(p, qi, w.Lk) - w.kofs;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
         const uint32_t par = (g + j) & 1u;
@@ -507,7 +505,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ptx::tc_fence_after();
         softmax_tile_chunked<D, BF16>(
-            tS, tO, j, sl2, (j + 1) * BN > w.min_lim, key_lim - j * BN, m, l,
+            tS, tO, j, sl2, j * BN < w.max_lo || (j + 1) * BN > w.min_hi, lo - j * BN,
+            hi - j * BN, m, l,
             [&]() {
               if (S_SPLIT) arrive(&bars->s_loaded[t]);
             },

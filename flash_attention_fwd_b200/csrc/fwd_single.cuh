@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       for (;;) {
         WorkItem w;
-        const bool have = sched.next(w);
+        const bool have = sched.next(w, p);
         if (!have) w.hu = -1;
         if (lane == 0) {
           ok = wait_bar(&bars->ring.empty[rs], rph ^ 1u, abort_flag);
@@ -319,7 +319,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (row_valid) empty_row<D>(orow_ptr, p.lse + orow);
         continue;
       }
-      const int key_lim = p.causal ? min(w.Lk, qi + 1) : w.Lk;
+      // visible keys of this row, relative to the first visited key tile
+      const int lo = key_lo(p, qi) - w.kofs;
+      const int hi = key_hi(p, qi, w.Lk) - w.kofs;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
         const uint32_t gj = g + j;
@@ -335,8 +337,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // cannot be issued before this iteration's P, so the barrier is in
         // phase gj-1 or gj.
         auto wait_o = [&]() { return wait_bar(&bars->pv_done, (gj - 1) & 1u, abort_flag); };
-        if (!softmax_tile<BN, D, BF16>(tS0 + buf * BN, tO, j, sl2, (j + 1) * BN > w.min_lim,
-                                       key_lim - j * BN, m, l, wait_o)) {
+        const bool need_mask = j * BN < w.max_lo || (j + 1) * BN > w.min_hi;
+        if (!softmax_tile<BN, D, BF16>(tS0 + buf * BN, tO, j, sl2, need_mask, lo - j * BN,
+                                       hi - j * BN, m, l, wait_o)) {
           ok = false;
           break;
         }

@@ -134,12 +134,14 @@ static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_
 
 using namespace vattn;
 
-extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
-                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
-                                  int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
-                                  int max_seqlen_k, int num_heads, int num_kv_heads, int head_dim,
-                                  int causal, float scale, varlen_dtype_t dtype, void *out,
-                                  float *lse, varlen_stream_t stream) {
+// Common body of the entry points.  window_left / window_right < 0 mean "no
+// bound"; seqused_k may be NULL.
+static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *cu_seqlens_q,
+                    const int32_t *cu_seqlens_k, int batch, int64_t total_q, int64_t total_k,
+                    int max_seqlen_q, int max_seqlen_k, int num_heads, int num_kv_heads,
+                    int head_dim, int causal, float scale, int window_left, int window_right,
+                    const int32_t *seqused_k, varlen_dtype_t dtype, void *out, float *lse,
+                    varlen_stream_t stream) {
   // ---- host-side validation: nothing is launched or touched on error
   if (dtype != VARLEN_BF16 && dtype != VARLEN_FP16) return VARLEN_ERR_DTYPE;
   if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
@@ -154,7 +156,8 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
   if (total_k > 0 && (!k || !v)) return VARLEN_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return VARLEN_ERR_ALIGN;
-  if (!aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
+  if (!aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
+      !aligned(seqused_k, 4))
     return VARLEN_ERR_ALIGN;
   if (batch == 0 || total_q == 0) return VARLEN_OK;
 
@@ -222,6 +225,13 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
   kp.causal = causal ? 1 : 0;
   const float sc = (scale > 0.f) ? scale : 1.0f / sqrtf((float)D);  // NaN fails "> 0"
   kp.scale_log2 = sc * 1.4426950408889634f;
+  kp.seqused_k = seqused_k;
+  // Window bounds in canonical form: a bound that no query of the buffers can
+  // reach is dropped (this also keeps qi - left and qi + right + 1 in range),
+  // and the causal rule is the right bound 0.
+  kp.win_left = (window_left >= 0 && (int64_t)window_left < total_q) ? window_left : -1;
+  kp.win_right = (window_right >= 0 && (int64_t)window_right < total_k) ? window_right : -1;
+  if (causal) kp.win_right = 0;
 
   // Upper bound of work items from max_seqlen_q; at least one CTA so that an
   // understated bound never drops work (the CTAs loop over all items).
@@ -250,6 +260,29 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
       return bf16 ? launch_single<256, true>(tq, tk, tv, kp, grid, s, dev, 8)
                   : launch_single<256, false>(tq, tk, tv, kp, grid, s, dev, 9);
   }
+}
+
+extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                  int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
+                                  int max_seqlen_k, int num_heads, int num_kv_heads, int head_dim,
+                                  int causal, float scale, varlen_dtype_t dtype, void *out,
+                                  float *lse, varlen_stream_t stream) {
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, -1, -1, nullptr,
+                  dtype, out, lse, stream);
+}
+
+extern "C" int varlen_attn_fwd_v2(const void *q, const void *k, const void *v,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                  int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
+                                  int max_seqlen_k, int num_heads, int num_kv_heads, int head_dim,
+                                  int causal, float scale, int window_left, int window_right,
+                                  const int32_t *seqused_k, varlen_dtype_t dtype, void *out,
+                                  float *lse, varlen_stream_t stream) {
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, window_left,
+                  window_right, seqused_k, dtype, out, lse, stream);
 }
 
 extern "C" int varlen_attn_fwd(const void *q, const void *k, const void *v,
@@ -300,4 +333,4 @@ extern "C" int varlen_attn_device_status(unsigned int *status, int clear) {
   return VARLEN_OK;
 }
 
-extern "C" int varlen_attn_abi_version(void) { return 1; }
+extern "C" int varlen_attn_abi_version(void) { return 2; }

@@ -112,6 +112,41 @@ int varlen_attn_fwd(const void *q, const void *k, const void *v,
                     int causal, float scale, varlen_dtype_t dtype,
                     void *out, float *lse, varlen_stream_t stream);
 
+/*
+ * varlen_attn_fwd_v2 — varlen_attn_fwd_v1 plus a sliding window and a
+ * per-sequence count of used keys: the window_size_left, window_size_right
+ * and seqused_k arguments of the varlen forward schema in PyTorch pull
+ * request #176015 (whose rule on versioned symbols puts them in a new entry
+ * point rather than into v1's signature).  The boostr page has no window; its
+ * sequence-local indices are kept: key ki is visible to query qi iff
+ *
+ *   ki < Lk_used(b),  Lk_used(b) = min(Lk_b, seqused_k[b])  (Lk_b without seqused_k)
+ *   ki >= qi - window_left    when window_left  >= 0
+ *   ki <= qi + window_right   when window_right >= 0
+ *   not (causal && qi < ki)
+ *
+ * A negative window bound means "no bound" on that side; window_left =
+ * window_right = -1 with seqused_k = NULL is exactly varlen_attn_fwd_v1.
+ *
+ *   window_left, window_right   as above (any int; negative = unbounded).
+ *   seqused_k    NULL, or [batch] int32 device array (4-byte aligned); a
+ *                negative entry counts as 0, an entry above Lk_b as Lk_b.
+ *                Keys in [Lk_used(b), Lk_b) get weight exactly 0 but may be
+ *                read, so they must hold finite values.
+ *
+ * Every other argument, the ownership and the error behaviour are those of
+ * varlen_attn_fwd_v1.  A query that sees no key (possible with a window, a
+ * short seqused_k or Lk_b = 0) gets out = 0 and lse = -inf.
+ */
+int varlen_attn_fwd_v2(const void *q, const void *k, const void *v,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       int batch, int64_t total_q, int64_t total_k,
+                       int max_seqlen_q, int max_seqlen_k,
+                       int num_heads, int num_kv_heads, int head_dim,
+                       int causal, float scale, int window_left, int window_right,
+                       const int32_t *seqused_k, varlen_dtype_t dtype,
+                       void *out, float *lse, varlen_stream_t stream);
+
 /* Static, human-readable description of a status code.  Never NULL. */
 const char *varlen_attn_strerror(int code);
 
@@ -126,7 +161,7 @@ const char *varlen_attn_strerror(int code);
  */
 int varlen_attn_device_status(unsigned int *status, int clear);
 
-/* Library ABI version (1 for this header). */
+/* Library ABI version: 2 for this header (v2 added; v1 unchanged). */
 int varlen_attn_abi_version(void);
 
 #ifdef __cplusplus

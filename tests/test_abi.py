@@ -28,7 +28,7 @@ def test_library_loads_and_exports_every_symbol():
     raw = ctypes.CDLL(fa.LIB_PATH)
     for name in header_functions():
         assert hasattr(raw, name), name
-    assert lib.varlen_attn_abi_version() == 1
+    assert lib.varlen_attn_abi_version() == 2
 
 
 def test_library_is_built_for_sm100a():
@@ -68,6 +68,13 @@ BASE = dict(q_ptr=0x10000, k_ptr=0x20000, v_ptr=0x30000, cu_q_ptr=0x40000, cu_k_
     (dict(out_ptr=0x60002), -4),
     (dict(lse_ptr=0x70002), -4),
     (dict(cu_k_ptr=0x50001), -4),
+    # the v2 entry point (window / seqused_k) validates the same way
+    (dict(window_left=4, num_heads=5), -2),
+    (dict(window_right=0, head_dim=96), -2),
+    (dict(seqused_k_ptr=0x80000, dtype_code=7), -3),
+    (dict(window_left=2, q_ptr=0), -1),
+    (dict(seqused_k_ptr=0x80002), -4),       # seqused_k needs 4-byte alignment
+    (dict(window_left=1, window_right=1, lse_ptr=0x70001), -4),
 ])
 def test_host_validation_rejects(change, code):
     args = dict(BASE)
@@ -81,6 +88,9 @@ def test_empty_problems_are_noops_without_device():
     assert fa.varlen_attn_fwd_raw(**args) == 0
     args = dict(BASE)
     args.update(total_q=0, q_ptr=0, out_ptr=0, lse_ptr=0)
+    assert fa.varlen_attn_fwd_raw(**args) == 0
+    args = dict(BASE)
+    args.update(batch=0, window_left=8, window_right=0, seqused_k_ptr=0x80000)
     assert fa.varlen_attn_fwd_raw(**args) == 0
 
 

@@ -1,0 +1,63 @@
+"""The benchmark's work counts (unmasked pairs -> FLOPs, algorithmic bytes)
+against brute-force enumeration of the visibility rule: key ki is visible to
+query qi iff ki < min(Lk, seqused_k), qi - left <= ki (left >= 0),
+ki <= qi + right (right >= 0) and not (causal and qi < ki)."""
+import numpy as np
+import pytest
+
+import bench
+import workloads
+
+
+def brute(lq, lk, causal, left, right, used):
+    lim = lk if used is None else min(lk, max(used, 0))
+    return sum(1 for qi in range(lq) for ki in range(lk)
+               if ki < lim and (left < 0 or ki >= qi - left) and (right < 0 or ki <= qi + right)
+               and not (causal and qi < ki))
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_visible_keys_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    lq, lk = int(rng.integers(0, 40)), int(rng.integers(0, 40))
+    causal = bool(rng.integers(0, 2))
+    left = int(rng.integers(-1, 12))
+    right = int(rng.integers(-1, 12))
+    used = None if rng.integers(0, 2) else int(rng.integers(-2, 45))
+    assert bench.visible_keys(lq, lk, causal, left, right, used) == \
+        brute(lq, lk, causal, left, right, used)
+
+
+def test_plain_counts_match_closed_form():
+    for lq, lk in [(1, 1), (7, 3), (3, 7), (128, 128), (300, 129)]:
+        assert bench.visible_keys(lq, lk, True) == brute(lq, lk, True, -1, -1, None)
+        assert bench.visible_keys(lq, lk, False) == lq * lk
+
+
+def test_sampled_row_flops_agree_with_per_row_counts():
+    case = workloads.make_case([40, 9, 70], [50, 9, 64], 4, 2, 16, "bf16", True, seed=3)
+    case.mask = dict(window_left=5, seqused_k=[30, 9, 100])
+    rows, fl = bench.oracle_sample_rows(case, 50, seed=1)
+    cu = case.cu_q.tolist()
+    want = 0
+    for tok, h in rows.tolist():
+        b = max(i for i in range(case.B) if cu[i] <= tok)
+        qi = tok - cu[b]
+        want += brute(qi + 1, case.lens_k[b], True, 5, -1, case.mask["seqused_k"][b]) - \
+            brute(qi, case.lens_k[b], True, 5, -1, case.mask["seqused_k"][b])
+    assert fl == 4 * case.D * want
+
+
+def test_used_keys_bytes():
+    case = workloads.make_workload("tiny")
+    plain = bench.algorithmic_bytes(case)
+    case.mask = dict(seqused_k=[17, 0, 1])
+    # 64 keys of sequence 1 are not used: K and V rows of Hkv heads x D dropped
+    assert plain - bench.algorithmic_bytes(case) == 2 * 64 * case.Hkv * case.D * 2 - 4 * case.B
+
+
+def test_named_masked_workloads():
+    assert workloads.make_workload("long_swa").mask == {"window_left": 4095}
+    used = workloads.seqused_k("shortq_used")
+    _, lk = workloads.seqlens("shortq_used")
+    assert len(used) == 32 and all(k // 2 <= u <= k for u, k in zip(used, lk))

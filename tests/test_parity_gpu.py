@@ -15,80 +15,15 @@ import torch
 
 import oracle
 import workloads
+from parity_helpers import (O_MAX, O_MEAN, LSE_MAX, GUARD, check_close, full_check,  # noqa: F401
+                            require_gpu, run_gpu, sampled_check)
 
 pytestmark = pytest.mark.gpu
-
-O_MAX, O_MEAN, LSE_MAX = 1.5e-2, 2e-3, 5e-3
-GUARD = 3
-
-
-def run_gpu(case, scale=None, guard=GUARD, max_q=None, max_k=None):
-    """Runs the CUDA forward with NaN-filled outputs inside guard rows.
-    Returns (out float64 [Tq,H,D], lse float64 [Tq,H], raw out, raw lse)."""
-    import flash_attention_fwd_b200 as fa
-    dev = torch.device("cuda", 0)
-    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
-    cq, ck = case.cu_q.to(dev), case.cu_k.to(dev)
-    Tq, H, D = case.q.shape
-    tdt = case.q.dtype
-    out_buf = torch.full((Tq + 2 * guard, H, D), float("nan"), dtype=tdt, device=dev)
-    lse_buf = torch.full((Tq + 2 * guard, H), float("nan"), dtype=torch.float32, device=dev)
-    canary = torch.tensor(-12345.0, dtype=tdt)
-    out_buf[:guard] = canary
-    out_buf[guard + Tq:] = canary
-    lse_buf[:guard] = -777.0
-    lse_buf[guard + Tq:] = -777.0
-    out = out_buf[guard:guard + Tq]
-    lse = lse_buf[guard:guard + Tq]
-    fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q if max_q is None else max_q,
-                       case.max_k if max_k is None else max_k, case.causal,
-                       scale if scale is not None else case.scale, out=out, lse=lse)
-    torch.cuda.synchronize()
-    ob, lb = out_buf.cpu(), lse_buf.cpu()
-    assert torch.all(ob[:guard] == canary) and torch.all(ob[guard + Tq:] == canary), "guard rows of out written"
-    assert torch.all(lb[:guard] == -777.0) and torch.all(lb[guard + Tq:] == -777.0), "guard rows of lse written"
-    return (ob[guard:guard + Tq].to(torch.float64).numpy(), lb[guard:guard + Tq].to(torch.float64).numpy(),
-            ob[guard:guard + Tq], lb[guard:guard + Tq])
-
-
-def check_close(out, lse, ref_out, ref_lse, what=""):
-    assert not np.isnan(out).any(), "%s: NaN left in out (row not written)" % what
-    assert not np.isnan(lse).any(), "%s: NaN left in lse (row not written)" % what
-    fin = np.isfinite(ref_lse)
-    assert np.array_equal(np.isfinite(lse), fin), "%s: -inf pattern of lse differs" % what
-    err = np.abs(out - ref_out)
-    assert err.max() <= O_MAX, "%s: O max abs err %.3e" % (what, err.max())
-    assert err.mean() <= O_MEAN, "%s: O mean abs err %.3e" % (what, err.mean())
-    if fin.any():
-        lerr = np.abs(lse[fin] - ref_lse[fin]).max()
-        assert lerr <= LSE_MAX, "%s: LSE max abs err %.3e" % (what, lerr)
-
-
-def full_check(case, **kw):
-    out, lse, _, _ = run_gpu(case, **kw)
-    ref_out, ref_lse = oracle.run_case(case)
-    check_close(out, lse, ref_out, ref_lse, case.name)
-    return out, lse
-
-
-def sampled_check(case, n=2000, seed=7, **kw):
-    out, lse, _, _ = run_gpu(case, **kw)
-    assert not np.isnan(out).any() and not np.isnan(lse).any(), "a packed row was not written"
-    rows = workloads.sample_rows(case, n, seed=seed)
-    ref_out, ref_lse = oracle.run_case_rows(case, rows)
-    check_close(out[rows[:, 0], rows[:, 1]], lse[rows[:, 0], rows[:, 1]], ref_out, ref_lse,
-                case.name)
 
 
 @pytest.fixture(scope="module", autouse=True)
 def _require_gpu():
-    if not torch.cuda.is_available():
-        pytest.skip("no CUDA device")
-    import flash_attention_fwd_b200 as fa
-    fa.load_library()
-    fa.device_status(clear=True)
-    yield
-    assert fa.device_status(clear=True) == 0, "a bounded pipeline wait timed out on the device"
+    yield from require_gpu()
 
 
 # --- the benchmark configurations ----------------------------------------------------

@@ -48,6 +48,9 @@ class Workload:
     sigma_k: float = 1.0
     sigma_v: float = 1.0
     description: str = ""
+    window_left: int = -1   # sliding window (negative = unbounded)
+    window_right: int = -1
+    seqused: bool = False   # draw a per-sequence used-key count
 
 
 WORKLOADS = {
@@ -63,6 +66,16 @@ WORKLOADS = {
                                    "H=32, Hkv=4, D=128, bf16, non-causal"),
     "wide": Workload("wide", 5, 16, 16, 256, "fp16", True, sigma_q=3.0, sigma_k=3.0, sigma_v=1.0,
                      description="wide-head MHA: 4x4096, H=Hkv=16, D=256, fp16, Q/K sigma 3, causal"),
+    # Sliding window and used-key counts (the window_size_left/right and
+    # seqused_k arguments of PyTorch pull request #176015's varlen forward)
+    # on the shapes above.
+    "long_swa": Workload("long_swa", 3, 64, 8, 128, "bf16", True, window_left=4095,
+                         description="long ragged prefill lengths with a causal sliding window of "
+                                     "4096 keys (left 4095), H=64, Hkv=8, D=128, bf16"),
+    "shortq_used": Workload("shortq_used", 4, 32, 4, 128, "bf16", False, seqused=True,
+                            description="short-query/long-KV lengths with per-sequence used-key "
+                                        "counts seqused_k in [Lk/2, Lk], H=32, Hkv=4, D=128, "
+                                        "bf16, non-causal"),
     # Profiling case only (not a benchmark configuration): the long ragged
     # prefill lengths with a quarter of its heads, so that a many-pass profiler
     # capture stays small while its inputs still exceed the L2 cache.
@@ -98,10 +111,10 @@ def seqlens(name: str):
         rng = np.random.default_rng(w.seed)
         q = [int(x) for x in rng.integers(128, 2049, 8)]
         return q, list(q)
-    if name in ("long", "long_h16"):
+    if name in ("long", "long_h16", "long_swa"):
         q = _long_lengths(w.seed)
         return q, list(q)
-    if name == "shortq":
+    if name in ("shortq", "shortq_used"):
         rng = np.random.default_rng(w.seed)
         q = [int(x) for x in rng.integers(1, 65, 32)]
         k = [int(x) for x in rng.integers(512, 8193, 32)]
@@ -110,6 +123,36 @@ def seqlens(name: str):
         q = [4096] * 4
         return q, list(q)
     raise KeyError(name)
+
+
+def seqused_k(name: str) -> Optional[List[int]]:
+    """Per-sequence used-key counts of a named workload (None if it has none):
+    drawn uniformly in [Lk // 2, Lk] by the length generator's stream, after
+    the lengths."""
+    w = WORKLOADS[name]
+    if not w.seqused:
+        return None
+    if name != "shortq_used":
+        raise KeyError(name)
+    rng = np.random.default_rng(w.seed)
+    rng.integers(1, 65, 32)
+    k = rng.integers(512, 8193, 32)
+    return [int(x) for x in rng.integers(k // 2, k + 1)]
+
+
+def mask_of(name: str) -> dict:
+    """Window / used-key arguments of a named workload, in the keyword form
+    the oracle takes (empty for the plain forward)."""
+    w = WORKLOADS[name]
+    m = {}
+    if w.window_left >= 0:
+        m["window_left"] = w.window_left
+    if w.window_right >= 0:
+        m["window_right"] = w.window_right
+    used = seqused_k(name)
+    if used is not None:
+        m["seqused_k"] = used
+    return m
 
 
 def cu_seqlens(lens: Sequence[int]) -> torch.Tensor:
@@ -137,6 +180,7 @@ class Case:
     scale: float
     name: str = "custom"
     seed: int = 0
+    mask: dict = field(default_factory=dict)  # window_left / window_right / seqused_k
 
     @property
     def B(self) -> int:
@@ -183,8 +227,10 @@ def make_workload(name: str) -> Case:
     """Full-size inputs of a named workload (CPU tensors)."""
     w = WORKLOADS[name]
     lq, lk = seqlens(name)
-    return make_case(lq, lk, w.H, w.Hkv, w.D, w.dtype, w.causal, w.seed,
+    case = make_case(lq, lk, w.H, w.Hkv, w.D, w.dtype, w.causal, w.seed,
                      w.sigma_q, w.sigma_k, w.sigma_v, name=name)
+    case.mask = mask_of(name)
+    return case
 
 
 def sample_rows(case: Case, n: int, seed: int = 1234) -> np.ndarray:
