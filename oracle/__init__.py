@@ -58,10 +58,10 @@ def _bind(lib):
     lib.oracle_decode16.argtypes = [ctypes.c_uint16, i32]
     lib.oracle_decode16.restype = f64
     lib.oracle_varlen_attn_fwd_ext.argtypes = [P, P, P, i32, P, P, P, i32, i32, i32, i32,
-                                               i32, i32, i32, f64, P, P, i32]
+                                               i32, i32, i32, P, f64, P, P, i32]
     lib.oracle_varlen_attn_fwd_ext.restype = i32
     lib.oracle_varlen_attn_rows_ext.argtypes = [P, P, P, i32, P, P, P, i32, i32, i32, i32,
-                                                i32, i32, i32, f64, P, P, i64, P, P, i32]
+                                                i32, i32, i32, P, f64, P, P, i64, P, P, i32]
     lib.oracle_varlen_attn_rows_ext.restype = i32
     return lib
 
@@ -108,11 +108,21 @@ def _seqused(seqused_k):
     return a, _ptr(a)
 
 
+def _sinks(sinks, H):
+    if sinks is None:
+        return None, ctypes.c_void_p(0)
+    a = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64).reshape(-1))
+    if a.shape[0] != H:
+        raise ValueError("sinks needs one value per query head")
+    return a, _ptr(a)
+
+
 def varlen_attn_fwd(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, nthreads=None,
-                    lib=None, window_left=-1, window_right=-1, seqused_k=None):
+                    lib=None, window_left=-1, window_right=-1, seqused_k=None, sinks=None):
     """Full fp64 forward.  Returns (out [Tq,H,D] float64, lse [Tq,H] float64).
     window_left/right < 0 mean unbounded; seqused_k (length B) caps the keys
-    of each sequence."""
+    of each sequence; sinks (length H) adds one logit per query head to the
+    softmax normalisation."""
     lib = lib or _load()
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
@@ -122,7 +132,8 @@ def varlen_attn_fwd(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, nthrea
     out = np.zeros((Tq, H, D), dtype=np.float64)
     lse = np.zeros((Tq, H), dtype=np.float64)
     keep, su = _seqused(seqused_k)
-    if window_left < 0 and window_right < 0 and seqused_k is None:
+    keep_s, sk = _sinks(sinks, H)
+    if window_left < 0 and window_right < 0 and seqused_k is None and sinks is None:
         rc = lib.oracle_varlen_attn_fwd(_ptr(qb), _ptr(kb), _ptr(vb), DTYPE_CODE[dtype],
                                         _ptr(cq), _ptr(ck), B, H, Hkv, D, int(bool(causal)),
                                         float(scale), _ptr(out), _ptr(lse),
@@ -131,7 +142,7 @@ def varlen_attn_fwd(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, nthrea
         rc = lib.oracle_varlen_attn_fwd_ext(_ptr(qb), _ptr(kb), _ptr(vb), DTYPE_CODE[dtype],
                                             _ptr(cq), _ptr(ck), su, B, H, Hkv, D,
                                             int(bool(causal)), int(window_left),
-                                            int(window_right), float(scale), _ptr(out),
+                                            int(window_right), sk, float(scale), _ptr(out),
                                             _ptr(lse), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError("oracle_varlen_attn_fwd failed with code %d" % rc)
@@ -140,7 +151,7 @@ def varlen_attn_fwd(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, nthrea
 
 def varlen_attn_rows(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, rows,
                      nthreads=None, lib=None, window_left=-1, window_right=-1,
-                     seqused_k=None):
+                     seqused_k=None, sinks=None):
     """fp64 forward of selected rows.  rows: int array [n, 2] of (token, head).
     Returns (out [n, D], lse [n])."""
     lib = lib or _load()
@@ -154,10 +165,11 @@ def varlen_attn_rows(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, rows,
     out = np.zeros((n, D), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
     keep, su = _seqused(seqused_k)
+    keep_s, sk = _sinks(sinks, H)
     rc = lib.oracle_varlen_attn_rows_ext(_ptr(qb), _ptr(kb), _ptr(vb), DTYPE_CODE[dtype],
                                          _ptr(cq), _ptr(ck), su, len(cq) - 1, H, Hkv, D,
                                          int(bool(causal)), int(window_left), int(window_right),
-                                         float(scale), _ptr(tok), _ptr(head), n, _ptr(out),
+                                         sk, float(scale), _ptr(tok), _ptr(head), n, _ptr(out),
                                          _ptr(lse), nthreads or default_threads())
     if rc != 0:
         raise RuntimeError("oracle_varlen_attn_rows failed with code %d" % rc)
@@ -166,7 +178,7 @@ def varlen_attn_rows(q, k, v, cu_q, cu_k, H, Hkv, D, causal, scale, dtype, rows,
 
 def run_case(case, nthreads=None, lib=None, **mask):
     """Full oracle forward of a ``workloads.Case`` (mask: window_left,
-    window_right, seqused_k)."""
+    window_right, seqused_k, sinks)."""
     return varlen_attn_fwd(case.q, case.k, case.v, case.cu_q.numpy(), case.cu_k.numpy(),
                            case.H, case.Hkv, case.D, case.causal, case.scale, case.dtype,
                            nthreads, lib=lib, **mask)

@@ -27,11 +27,14 @@ def segment_ids(cu: np.ndarray) -> np.ndarray:
 
 def dense_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_q, cu_k, causal: bool,
                   scale: float, window_left: int = -1, window_right: int = -1,
-                  seqused_k=None):
+                  seqused_k=None, sinks=None):
     """q [Tq,H,D], k/v [Tk,Hkv,D] float64.  Returns (out [Tq,H,D], lse [Tq,H]).
     Optional sliding window (sequence-local: key ki visible to query qi only
     if qi - left <= ki <= qi + right, negative = unbounded) and per-sequence
-    used-key counts; rows without a visible key give O = 0, LSE = -inf."""
+    used-key counts; rows without a visible key give O = 0, LSE = -inf.
+    With ``sinks`` (one logit per query head) the score matrix gets one more
+    column holding sinks[h] for every row, and the value matrix a zero row:
+    the dense softmax over [S | sink] then weights V."""
     Tq, H, D = q.shape
     Tk, Hkv, _ = k.shape
     G = H // Hkv
@@ -54,6 +57,9 @@ def dense_forward(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_q, cu_k, causa
         vh = v[:, h // G, :]
         s = (q[:, h, :] @ kh.T) * scale
         s = np.where(visible, s, -np.inf)
+        if sinks is not None:
+            s = np.concatenate([s, np.full((Tq, 1), float(sinks[h]))], axis=1)
+            vh = np.concatenate([vh, np.zeros((1, D))], axis=0)
         m = s.max(axis=1, initial=-np.inf)
         has = np.isfinite(m)
         e = np.zeros_like(s)

@@ -32,6 +32,15 @@
  * right >= 0 and ki > qi + right.  A row with no visible key gets O = 0 and
  * LSE = -inf, what the page's loop gives for a sequence without keys.
  *
+ * Attention sinks (the `sinks` argument of the `_ext` entry points; the
+ * FLOAT32 per-head "sinks" input of the Ascend sparse shared-KV attention
+ * page, which gives no formula): sinks[h] is one more logit, already in score
+ * units (not multiplied by the scale), that joins the softmax of every row of
+ * query head h but has no value row.  So m = max(max_ki s_ki, sinks[h]),
+ * l = sum_ki exp(s_ki - m) + exp(sinks[h] - m), O = sum_ki exp(s_ki - m) / l
+ * * V_ki, LSE = m + ln(l); a row without visible keys then gets O = 0 and
+ * LSE = sinks[h].
+ *
  * Inputs are bf16 or fp16 bit patterns; they are widened exactly to double
  * before any arithmetic.  The widening of a key/value head of one sequence
  * is done once per (b, h) work item; that is a format conversion, not a
@@ -84,6 +93,7 @@ typedef struct {
     const int32_t *seqused_k; /* NULL: every key of the sequence */
     int B, H, Hkv, D, causal;
     int win_left, win_right;  /* < 0: unbounded */
+    const double *sinks;      /* NULL, or one extra logit per query head */
     double scale;
     /* full mode */
     double *out, *lse;
@@ -115,6 +125,10 @@ static int used_keys(const OracleCtx *c, int b) {
     return Lk;
 }
 
+static double head_sink(const OracleCtx *c, int h) {
+    return c->sinks ? c->sinks[h] : -INFINITY;
+}
+
 static int key_hidden(const OracleCtx *c, int qi, int ki) {
     if (c->causal && qi < ki) return 1;
     if (c->win_left >= 0 && ki < qi - c->win_left) return 1;
@@ -125,7 +139,7 @@ static int key_hidden(const OracleCtx *c, int qi, int ki) {
 /* One query row: the page's two-pass softmax, in double precision.
  * kd/vd hold the widened keys/values of head kv_h of sequence b, [Lk][D]. */
 static void oracle_attend_row(const OracleCtx *c, const double *qrow, int qi, int Lk,
-                              const double *kd, const double *vd, double *scores,
+                              const double *kd, const double *vd, double *scores, double sink,
                               double *out_row, double *lse_out) {
     const int D = c->D;
     double max_score = -INFINITY;
@@ -141,7 +155,8 @@ static void oracle_attend_row(const OracleCtx *c, const double *qrow, int qi, in
         if (s > max_score) max_score = s;
         scores[ki] = s;
     }
-    if (max_score == -INFINITY) { /* no visible key */
+    if (sink > max_score) max_score = sink; /* the sink logit takes part in the max */
+    if (max_score == -INFINITY) { /* no visible key and no sink */
         for (int d = 0; d < D; ++d) out_row[d] = 0.0;
         *lse_out = -INFINITY;
         return;
@@ -152,6 +167,7 @@ static void oracle_attend_row(const OracleCtx *c, const double *qrow, int qi, in
         sum_exp += e;
         scores[ki] = e;
     }
+    sum_exp += exp(sink - max_score); /* ... and in the normalisation (0 without a sink) */
     for (int d = 0; d < D; ++d) out_row[d] = 0.0;
     for (int ki = 0; ki < Lk; ++ki) {
         double weight = scores[ki] / sum_exp;
@@ -214,7 +230,7 @@ static void *full_worker(void *arg) {
         for (int qi = 0; qi < Lq; ++qi) {
             int64_t tok = (int64_t)q0 + qi;
             widen_q(c, tok, h, qd);
-            oracle_attend_row(c, qd, qi, Lk, kd, vd, scores,
+            oracle_attend_row(c, qd, qi, Lk, kd, vd, scores, head_sink(c, h),
                               c->out + ((size_t)tok * H + h) * D,
                               c->lse + (size_t)tok * H + h);
         }
@@ -265,7 +281,7 @@ static void *rows_worker(void *arg) {
             cached_kvh = kv_h;
         }
         widen_q(c, tok, h, qd);
-        oracle_attend_row(c, qd, qi, Lk, kd, vd, scores,
+        oracle_attend_row(c, qd, qi, Lk, kd, vd, scores, head_sink(c, h),
                           c->out_rows + (size_t)i * D, c->lse_rows + i);
     }
     free(kd); free(vd); free(scores); free(qd);
@@ -298,8 +314,8 @@ static int check_args(int B, int H, int Hkv, int D, int dtype) {
 int oracle_varlen_attn_fwd_ext(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                int dtype, const int32_t *cu_q, const int32_t *cu_k,
                                const int32_t *seqused_k, int B, int H, int Hkv, int D, int causal,
-                               int win_left, int win_right, double scale, double *out,
-                               double *lse, int nthreads) {
+                               int win_left, int win_right, const double *sinks, double scale,
+                               double *out, double *lse, int nthreads) {
     int rc = check_args(B, H, Hkv, D, dtype);
     if (rc) return rc;
     OracleCtx c;
@@ -307,7 +323,7 @@ int oracle_varlen_attn_fwd_ext(const uint16_t *q, const uint16_t *k, const uint1
     c.q = q; c.k = k; c.v = v; c.dtype = dtype; c.cu_q = cu_q; c.cu_k = cu_k;
     c.seqused_k = seqused_k;
     c.B = B; c.H = H; c.Hkv = Hkv; c.D = D; c.causal = causal != 0;
-    c.win_left = win_left; c.win_right = win_right;
+    c.win_left = win_left; c.win_right = win_right; c.sinks = sinks;
     c.scale = effective_scale(scale, D);
     c.out = out; c.lse = lse;
     c.n_items = (int64_t)B * H;
@@ -319,7 +335,7 @@ int oracle_varlen_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t 
                            int D, int causal, double scale, double *out, double *lse,
                            int nthreads) {
     return oracle_varlen_attn_fwd_ext(q, k, v, dtype, cu_q, cu_k, NULL, B, H, Hkv, D, causal,
-                                      -1, -1, scale, out, lse, nthreads);
+                                      -1, -1, NULL, scale, out, lse, nthreads);
 }
 
 /* Selected rows: for i in [0, nrows) computes the output row of packed query
@@ -327,9 +343,9 @@ int oracle_varlen_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t 
 int oracle_varlen_attn_rows_ext(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                                 int dtype, const int32_t *cu_q, const int32_t *cu_k,
                                 const int32_t *seqused_k, int B, int H, int Hkv, int D,
-                                int causal, int win_left, int win_right, double scale,
-                                const int64_t *row_tok, const int32_t *row_head, int64_t nrows,
-                                double *out_rows, double *lse_rows, int nthreads) {
+                                int causal, int win_left, int win_right, const double *sinks,
+                                double scale, const int64_t *row_tok, const int32_t *row_head,
+                                int64_t nrows, double *out_rows, double *lse_rows, int nthreads) {
     int rc = check_args(B, H, Hkv, D, dtype);
     if (rc) return rc;
     if (B < 1) return -2;
@@ -338,7 +354,7 @@ int oracle_varlen_attn_rows_ext(const uint16_t *q, const uint16_t *k, const uint
     c.q = q; c.k = k; c.v = v; c.dtype = dtype; c.cu_q = cu_q; c.cu_k = cu_k;
     c.seqused_k = seqused_k;
     c.B = B; c.H = H; c.Hkv = Hkv; c.D = D; c.causal = causal != 0;
-    c.win_left = win_left; c.win_right = win_right;
+    c.win_left = win_left; c.win_right = win_right; c.sinks = sinks;
     c.scale = effective_scale(scale, D);
     c.row_tok = row_tok; c.row_head = row_head; c.nrows = nrows;
     c.out_rows = out_rows; c.lse_rows = lse_rows;
@@ -351,6 +367,6 @@ int oracle_varlen_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t
                             const int32_t *row_head, int64_t nrows, double *out_rows,
                             double *lse_rows, int nthreads) {
     return oracle_varlen_attn_rows_ext(q, k, v, dtype, cu_q, cu_k, NULL, B, H, Hkv, D, causal,
-                                       -1, -1, scale, row_tok, row_head, nrows, out_rows,
+                                       -1, -1, NULL, scale, row_tok, row_head, nrows, out_rows,
                                        lse_rows, nthreads);
 }
