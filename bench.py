@@ -270,8 +270,18 @@ def run_gpu(args, rank: int, world: int):
 
     case = workloads.make_workload(args.workload)
     flops = step_flops(case)
-    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
-    cq, ck = case.cu_q.to(dev), case.cu_k.to(dev)
+    wl = workloads.WORKLOADS[args.workload]
+    table_t = None
+    if wl.page_size:
+        # the same keys in a page cache; the oracle legs read the packed copy
+        pk = workloads.to_paged(case, wl.page_size, seed=wl.seed)
+        q, k, v = case.q.to(dev), pk.k_cache.to(dev), pk.v_cache.to(dev)
+        table_t = pk.page_table.to(dev)
+        ck = None
+    else:
+        q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+        ck = case.cu_k.to(dev)
+    cq = case.cu_q.to(dev)
     out = torch.empty_like(q)
     lse = torch.empty((case.Tq, case.H), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -279,13 +289,18 @@ def run_gpu(args, rank: int, world: int):
     fa.device_status(clear=True)
 
     used = case.mask.get("seqused_k")
+    if table_t is not None and used is None:
+        used = case.lens_k
     used_t = None if used is None else torch.tensor(used, dtype=torch.int32, device=dev)
     wl, wr = case.mask.get("window_left", -1), case.mask.get("window_right", -1)
+    sinks = case.mask.get("sinks")
+    sinks_t = None if sinks is None else torch.tensor(sinks, dtype=torch.float32, device=dev)
 
     def step():
         fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, case.causal, case.scale,
                            out=out, lse=lse, stream=stream, window_size_left=wl,
-                           window_size_right=wr, seqused_k=used_t)
+                           window_size_right=wr, seqused_k=used_t, page_table=table_t,
+                           sinks=sinks_t)
 
     for _ in range(args.warmup):
         step()
@@ -317,7 +332,8 @@ def run_gpu(args, rank: int, world: int):
         e2e_ms, h2d, d2h = float("nan"), 0, 0
     else:
         e2e_ms, h2d, d2h = run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist,
-                                   extra=[used_t] if used_t is not None else [])
+                                   extra=[t for t in (used_t, table_t, sinks_t)
+                                          if t is not None])
 
     if dist:
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
@@ -330,11 +346,12 @@ def run_gpu(args, rank: int, world: int):
 def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist, extra=()):
     import torch
     hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
-    hcq, hck = case.cu_q.pin_memory(), case.cu_k.pin_memory()
+    hcq = case.cu_q.pin_memory()
+    hck = case.cu_k.pin_memory() if ck is not None else None
     ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     hx = [t.cpu().pin_memory() for t in extra]  # further inputs (seqused_k)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck, *hx))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck, *hx) if t is not None)
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
 
     def e2e_step():
@@ -342,7 +359,8 @@ def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist, extra=())
         k.copy_(hk, non_blocking=True)
         v.copy_(hv, non_blocking=True)
         cq.copy_(hcq, non_blocking=True)
-        ck.copy_(hck, non_blocking=True)
+        if ck is not None:
+            ck.copy_(hck, non_blocking=True)
         for d, h in zip(extra, hx):
             d.copy_(h, non_blocking=True)
         step()
@@ -393,6 +411,8 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
                 "D": case.D, "causal": case.causal, "flops_per_step": flops,
                 "window": [case.mask.get("window_left", -1), case.mask.get("window_right", -1)],
                 "seqused_k": "seqused_k" in case.mask,
+                "page_size": workloads.WORKLOADS[args.workload].page_size or None,
+                "sinks": "sinks" in case.mask,
                 "l2": "no flush: inputs (%.0f MB) exceed the 126 MB L2"
                       % (algorithmic_bytes(case) / 1e6),
                 "parallelism": "dp%d (one independent batch per GPU)" % world},

@@ -38,6 +38,7 @@ STATUS_NAMES = {
 EXPORTED_SYMBOLS = (
     "varlen_attn_fwd_v1",
     "varlen_attn_fwd_v2",
+    "varlen_attn_fwd_v3",
     "varlen_attn_fwd",
     "varlen_attn_strerror",
     "varlen_attn_device_status",
@@ -65,6 +66,10 @@ def _bind(lib):
     # v2: v1's arguments with window_left, window_right, seqused_k after scale
     lib.varlen_attn_fwd_v2.argtypes = fwd_args[:15] + [i32, i32, P] + fwd_args[15:]
     lib.varlen_attn_fwd_v2.restype = i32
+    # v3: v2's arguments with page_table, page_table_stride, page_size, sinks after seqused_k
+    lib.varlen_attn_fwd_v3.argtypes = (fwd_args[:15] + [i32, i32, P, P, i32, i32, P]
+                                       + fwd_args[15:])
+    lib.varlen_attn_fwd_v3.restype = i32
     lib.varlen_attn_strerror.argtypes = [i32]
     lib.varlen_attn_strerror.restype = ctypes.c_char_p
     lib.varlen_attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i32]
@@ -115,16 +120,24 @@ def varlen_attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, cu_q_ptr: int, cu_k_
                         max_seqlen_k: int, num_heads: int, num_kv_heads: int, head_dim: int,
                         causal: bool, scale: float, dtype_code: int, out_ptr: int,
                         lse_ptr: int, stream: int, window_left: int = -1,
-                        window_right: int = -1, seqused_k_ptr: int = 0) -> int:
+                        window_right: int = -1, seqused_k_ptr: int = 0,
+                        page_table_ptr: int = 0, page_table_stride: int = 0,
+                        page_size: int = 0, sinks_ptr: int = 0) -> int:
     """Direct call of the C entry point with integer addresses; returns the
-    status code unchanged.  Calls varlen_attn_fwd (v1) unless a window bound
-    or a seqused_k array is given, varlen_attn_fwd_v2 otherwise."""
+    status code unchanged.  Calls varlen_attn_fwd (v1) unless a window bound,
+    a seqused_k array, a page table or sinks are given; varlen_attn_fwd_v2 for
+    a window / seqused_k, varlen_attn_fwd_v3 for a page table or sinks."""
     lib = load_library()
     V = ctypes.c_void_p
     head = (V(q_ptr), V(k_ptr), V(v_ptr), V(cu_q_ptr), V(cu_k_ptr), int(batch), int(total_q),
             int(total_k), int(max_seqlen_q), int(max_seqlen_k), int(num_heads),
             int(num_kv_heads), int(head_dim), int(bool(causal)), float(scale))
     tail = (int(dtype_code), V(out_ptr), V(lse_ptr), V(stream))
+    if page_table_ptr or sinks_ptr:
+        return lib.varlen_attn_fwd_v3(*head, int(window_left), int(window_right),
+                                      V(seqused_k_ptr), V(page_table_ptr),
+                                      int(page_table_stride), int(page_size), V(sinks_ptr),
+                                      *tail)
     if window_left < 0 and window_right < 0 and not seqused_k_ptr:
         return lib.varlen_attn_fwd(*head, *tail)
     return lib.varlen_attn_fwd_v2(*head, int(window_left), int(window_right),
@@ -132,13 +145,15 @@ def varlen_attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, cu_q_ptr: int, cu_k_
 
 
 def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
-                    cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                    cu_seqlens_q: torch.Tensor, cu_seqlens_k: Optional[torch.Tensor],
                     max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,
                     scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                     lse: Optional[torch.Tensor] = None,
                     stream: Optional[torch.cuda.Stream] = None,
                     window_size_left: int = -1, window_size_right: int = -1,
-                    seqused_k: Optional[torch.Tensor] = None
+                    seqused_k: Optional[torch.Tensor] = None,
+                    page_table: Optional[torch.Tensor] = None,
+                    sinks: Optional[torch.Tensor] = None
                     ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Packed attention forward on the GPU.
 
@@ -151,21 +166,49 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     forward schema of PyTorch pull request #176015: key ki is visible to query
     qi iff ki < min(Lk, seqused_k[b]), qi - left <= ki <= qi + right, and
     not (causal and qi < ki).
+
+    With ``page_table`` (int32 [B, pages_per_seq] on the device) k and v are
+    paged caches [num_pages, page_size, Hkv, D], key ki of sequence b is
+    ``k[page_table[b, ki // page_size], ki % page_size]``, ``seqused_k`` is
+    required and gives the key counts, and ``cu_seqlens_k`` is not used (it
+    may be None).
+
+    ``sinks`` (float32 [H] on the device) adds one logit per query head to
+    the softmax normalisation (attention sinks): the row's weights become
+    exp(s - m) / (sum exp(s - m) + exp(sinks[h] - m)).
     """
     if q.dtype not in DTYPE_CODES or k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share dtype bfloat16 or float16")
-    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
-        raise ValueError("expected q [Tq,H,D] and k, v [Tk,Hkv,D]")
-    for name, t in (("q", q), ("k", k), ("v", v), ("cu_seqlens_q", cu_seqlens_q),
-                    ("cu_seqlens_k", cu_seqlens_k)):
-        if not t.is_cuda or not t.is_contiguous():
+    paged = page_table is not None
+    if q.dim() != 3 or k.dim() != (4 if paged else 3) or v.shape != k.shape:
+        raise ValueError("expected q [Tq,H,D] and k, v [Tk,Hkv,D] "
+                         "(paged: [num_pages,page_size,Hkv,D])")
+    tensors = [("q", q), ("k", k), ("v", v), ("cu_seqlens_q", cu_seqlens_q)]
+    if not paged or cu_seqlens_k is not None:
+        tensors.append(("cu_seqlens_k", cu_seqlens_k))
+    for name, t in tensors:
+        if t is None or not t.is_cuda or not t.is_contiguous():
             raise ValueError("%s must be a contiguous CUDA tensor" % name)
-    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+    B = cu_seqlens_q.numel() - 1
+    if cu_seqlens_q.dtype != torch.int32 or (cu_seqlens_k is not None
+                                             and cu_seqlens_k.dtype != torch.int32):
         raise TypeError("cu_seqlens must be int32")
-    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 1:
+    if B < 0 or (cu_seqlens_k is not None and cu_seqlens_k.numel() != B + 1):
         raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B+1 >= 1 entries")
     total_q, H, D = q.shape
-    total_k, Hkv, Dk = k.shape
+    page_size = stride = 0
+    if paged:
+        num_pages, page_size, Hkv, Dk = k.shape
+        total_k = num_pages * page_size
+        if (not page_table.is_cuda or not page_table.is_contiguous()
+                or page_table.dtype != torch.int32 or page_table.dim() != 2
+                or page_table.shape[0] != B):
+            raise ValueError("page_table must be a contiguous int32 CUDA tensor [B, pages]")
+        if seqused_k is None:
+            raise ValueError("a page table needs seqused_k (the key count of each sequence)")
+        stride = page_table.shape[1]
+    else:
+        total_k, Hkv, Dk = k.shape
     if Dk != D:
         raise ValueError("head dims of q and k differ")
     if out is None:
@@ -178,20 +221,25 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         raise ValueError("lse must be a contiguous float32 tensor [Tq, H]")
     if seqused_k is not None:
         if (not seqused_k.is_cuda or not seqused_k.is_contiguous()
-                or seqused_k.dtype != torch.int32
-                or seqused_k.numel() != cu_seqlens_q.numel() - 1):
+                or seqused_k.dtype != torch.int32 or seqused_k.numel() != B):
             raise ValueError("seqused_k must be a contiguous int32 CUDA tensor [B]")
+    if sinks is not None:
+        if (not sinks.is_cuda or not sinks.is_contiguous() or sinks.dtype != torch.float32
+                or sinks.numel() != H):
+            raise ValueError("sinks must be a contiguous float32 CUDA tensor [H]")
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+
+    def addr(t):
+        return t.data_ptr() if t is not None and t.numel() else 0
+
     with torch.cuda.device(q.device):
         rc = varlen_attn_fwd_raw(
-            q.data_ptr(), k.data_ptr() if k.numel() else 0, v.data_ptr() if v.numel() else 0,
-            cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), cu_seqlens_q.numel() - 1,
+            addr(q), addr(k), addr(v), addr(cu_seqlens_q), addr(cu_seqlens_k), B,
             total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), H, Hkv, D, causal,
-            0.0 if scale is None else float(scale), DTYPE_CODES[q.dtype],
-            out.data_ptr() if out.numel() else 0, lse.data_ptr() if lse.numel() else 0,
-            stream.cuda_stream, int(window_size_left), int(window_size_right),
-            seqused_k.data_ptr() if seqused_k is not None and seqused_k.numel() else 0)
+            0.0 if scale is None else float(scale), DTYPE_CODES[q.dtype], addr(out), addr(lse),
+            stream.cuda_stream, int(window_size_left), int(window_size_right), addr(seqused_k),
+            addr(page_table), stride, page_size, addr(sinks))
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return out, lse

@@ -27,6 +27,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;           // log2 units: rescale O only when max grows > 2^8
 constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull; // 2 s: far beyond any legitimate wait
 constexpr unsigned STATUS_TIMEOUT = 1u;
+constexpr unsigned STATUS_BAD_PAGE = 2u;  // a page-table entry outside [0, num_pages)
 
 // Device-side status word (bit STATUS_TIMEOUT: a bounded wait gave up).
 __device__ unsigned int g_device_status = 0;
@@ -48,7 +49,22 @@ struct KParams {
   int win_left;          // key ki visible to query qi only if ki >= qi - win_left (-1: no bound)
   int win_right;         // ... and ki <= qi + win_right (-1: no bound); the causal rule is
                          // folded in by the host (causal => win_right = 0)
+  // Paged K/V (page_table != nullptr): k and v are [num_pages * page_size, Hkv, D]
+  // (i.e. [num_pages, page_size, Hkv, D]); key ki of sequence b lives in row
+  // page_table[b * pt_stride + ki / page_size] * page_size + ki % page_size, and
+  // sequence b has seqused_k[b] keys (cu_k is not read).
+  const int *page_table;
+  int pt_stride;   // entries per sequence in page_table
+  int page_size;   // keys per page, a multiple of 16
+  int num_pages;
+  int page_chunk;  // rows per TMA box of a paged K/V tile (divides page_size and the key tile)
+  const float *sinks;  // optional [H]: one extra logit per query head in the softmax normalisation
 };
+
+// Sink logit of query head h in log2 units (-inf: none).
+__device__ __forceinline__ float sink_log2(const KParams &p, int h) {
+  return p.sinks ? __ldg(p.sinks + h) * 1.4426950408889634f : -INFINITY;
+}
 
 // Visible keys [key_lo, key_hi) of the sequence-local query qi in a sequence
 // with Lk used keys (empty when key_hi <= key_lo).
@@ -60,6 +76,7 @@ __device__ __forceinline__ int key_hi(const KParams &p, int qi, int Lk) {
 }
 
 struct WorkItem {
+  int b;        // sequence
   int hu;       // head unit (a head, a pair of heads 2hu, 2hu+1, or a key/value head)
   int q0;       // packed index of the item's first query token
   int q_rows;   // valid query tokens in the item (<= unit_tokens)
@@ -98,6 +115,8 @@ template <int BN>
 struct Scheduler {
   const int *cu_q, *cu_k, *seqused_k;
   int B, HU, U, R, causal, total_q, total_k;
+  bool paged;
+  int paged_keys;  // keys addressable through one page-table row
   int cta, grid, lane;
   long long round;
   int level;              // current cost level; -1 once the list is exhausted
@@ -109,13 +128,18 @@ struct Scheduler {
   __device__ void extents(int b, int &qs, int &lq, int &ks, int &lk) const {
     qs = __ldg(cu_q + b);
     int qe = __ldg(cu_q + b + 1);
-    ks = __ldg(cu_k + b);
-    int ke = __ldg(cu_k + b + 1);
     qs = min(max(qs, 0), total_q);
     qe = min(max(qe, qs), total_q);
+    lq = qe - qs;
+    if (paged) {
+      ks = 0;
+      lk = min(max(__ldg(seqused_k + b), 0), paged_keys);
+      return;
+    }
+    ks = __ldg(cu_k + b);
+    int ke = __ldg(cu_k + b + 1);
     ks = min(max(ks, 0), total_k);
     ke = min(max(ke, ks), total_k);
-    lq = qe - qs;
     lk = ke - ks;
     if (seqused_k) lk = min(lk, max(__ldg(seqused_k + b), 0));
   }
@@ -156,6 +180,8 @@ struct Scheduler {
     cu_q = p.cu_q;
     cu_k = p.cu_k;
     seqused_k = p.seqused_k;
+    paged = p.page_table != nullptr;
+    paged_keys = (int)min((long long)p.pt_stride * p.page_size, (long long)INT32_MAX);
     B = p.B;
     HU = p.head_units;
     U = p.unit_tokens;
@@ -225,6 +251,7 @@ struct Scheduler {
         lk = __shfl_sync(0xffffffffu, lk, src);
         cur_b += src;
         cur_units += before;
+        w.b = cur_b;
         const int k = (int)(unit - cur_units);
         const int qt = tile_of((lk + BM - 1) / BM, level, k);
         w.qi0 = qt * U;
@@ -272,6 +299,147 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     }
   }
 }
+
+// ---------------------------------------------------------------------------
+// Producer side of the K/V shared-memory ring: NSLOT slots of one BN-key tile
+// (D / 64 swizzled 128-byte column blocks) each, slot s guarded by full[s]
+// (TMA bytes landed) and empty[s] (the MMAs that read it completed).  Used by
+// one warp; lane 0 issues the copies.
+//
+// Packed K/V: a key tile is BN consecutive rows of k/v.  Paged K/V: a key tile
+// is BN / chunk boxes of `chunk` rows (chunk divides the page size and BN, so a
+// box never crosses a page); lane c of the warp looks up the page of box c.
+// A box past the sequence's used keys, or whose page-table entry is out of
+// range, is read at a row beyond the buffer, which the TMA fills with zeros.
+template <int BN, int D, int NSLOT>
+struct KVProducer {
+  static constexpr int DB = D / 64;
+  static constexpr uint32_t KV_BYTES = BN * D * 2;
+  uint8_t *sKV;
+  uint64_t *full, *empty;
+  volatile int *abort_flag;
+  uint64_t pol;
+  uint32_t slot, phase;
+  uint32_t fills[NSLOT];
+  int lane;
+
+  __device__ void init(uint8_t *s, uint64_t *f, uint64_t *e, volatile int *abort) {
+    sKV = s;
+    full = f;
+    empty = e;
+    abort_flag = abort;
+    pol = ptx::policy_evict_last();
+    slot = 0;
+    phase = 0;
+    for (int i = 0; i < NSLOT; ++i) fills[i] = 0;
+    lane = threadIdx.x & 31;
+  }
+  __device__ void advance() {
+    ++fills[slot];
+    if (++slot == NSLOT) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+  // lane 0: key rows [row, row + BN) of a packed k/v
+  __device__ bool load_packed(const CUtensorMap *tm, int kv_h, int row) {
+    if (!wait_bar(&empty[slot], phase ^ 1u, abort_flag)) return false;
+    uint8_t *dst = sKV + slot * KV_BYTES;
+    ptx::mbar_arrive_expect_tx(&full[slot], KV_BYTES);
+#pragma unroll
+    for (int db = 0; db < DB; ++db)
+      ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &full[slot], db * 64, kv_h, row, pol);
+    advance();
+    return true;
+  }
+  // paged: source row of box `lane` of the key tile that starts at key0
+  __device__ int chunk_row(const KParams &p, const WorkItem &w, int key0) const {
+    int row = p.total_k;  // beyond the buffer: zero fill
+    const int ch = p.page_chunk;
+    if (lane * ch < BN) {
+      const int key = key0 + lane * ch;
+      if (key < w.Lk) {
+        const int pg = __ldg(p.page_table + (size_t)w.b * p.pt_stride + key / p.page_size);
+        if (pg >= 0 && pg < p.num_pages)
+          row = pg * p.page_size + key % p.page_size;
+        else
+          atomicOr(&g_device_status, STATUS_BAD_PAGE);
+      }
+    }
+    return row;
+  }
+  // Whole warp: one paged key tile; lane c copies box c from row my_row.
+  // Lane 0 waits for the slot and posts the byte count first, so the lanes'
+  // copies (one warp instruction per column block) complete into a phase
+  // that already expects them.
+  __device__ bool load_paged(const CUtensorMap *tm, int kv_h, int my_row, int ch) {
+    bool ok = true;
+    if (lane == 0) {
+      ok = wait_bar(&empty[slot], phase ^ 1u, abort_flag);
+      if (ok) ptx::mbar_arrive_expect_tx(&full[slot], KV_BYTES);
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) return false;
+    if (lane * ch < BN) {
+      uint8_t *dst = sKV + slot * KV_BYTES + lane * ch * 128;
+#pragma unroll
+      for (int db = 0; db < DB; ++db)
+        ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &full[slot], db * 64, kv_h, my_row, pol);
+    }
+    advance();
+    return true;
+  }
+  // Whole warp: the K/V tiles of one item in the order the MMA warp consumes
+  // them (K0, K1, V0, K2, V1, K3, ..., V(n-1)), with the item's Q tile(s) after
+  // K0 through load_q (called by lane 0, returns false when a wait gave up).
+  template <class LoadQ>
+  __device__ bool load_item(const KParams &p, const WorkItem &w, int kv_h, const CUtensorMap *tm_k,
+                            const CUtensorMap *tm_v, LoadQ &&load_q) {
+    const int n = w.n_kv;
+    if (p.page_table == nullptr) {
+      bool ok = true;
+      if (lane == 0) {
+        ok = load_packed(tm_k, kv_h, w.k0) && load_q();
+        if (ok && n >= 2) ok = load_packed(tm_k, kv_h, w.k0 + BN);
+        for (int j = 0; ok && j < n; ++j) {
+          ok = load_packed(tm_v, kv_h, w.k0 + j * BN);
+          if (ok && j + 2 < n) ok = load_packed(tm_k, kv_h, w.k0 + (j + 2) * BN);
+        }
+      }
+      return __shfl_sync(0xffffffffu, ok, 0);
+    }
+    const int ch = p.page_chunk;
+    int r0 = chunk_row(p, w, w.kofs), r1 = 0;
+    bool ok = load_paged(tm_k, kv_h, r0, ch);
+    if (ok) {
+      bool q = true;
+      if (lane == 0) q = load_q();
+      ok = __shfl_sync(0xffffffffu, q, 0);
+    }
+    if (ok && n >= 2) {
+      r1 = chunk_row(p, w, w.kofs + BN);
+      ok = load_paged(tm_k, kv_h, r1, ch);
+    }
+    for (int j = 0; ok && j < n; ++j) {
+      // look up K(j+2) before waiting for V(j)'s slot, so that the two overlap
+      const int rn = (j + 2 < n) ? chunk_row(p, w, w.kofs + (j + 2) * BN) : 0;
+      ok = load_paged(tm_v, kv_h, (j & 1) ? r1 : r0, ch);
+      if (ok && j + 2 < n) {
+        if (j & 1)
+          r1 = rn;
+        else
+          r0 = rn;
+        ok = load_paged(tm_k, kv_h, rn, ch);
+      }
+    }
+    return ok;
+  }
+  // lane 0: every copy issued has landed (before the CTA exits)
+  __device__ void drain() {
+    for (int i = 0; i < NSLOT; ++i)
+      if (fills[i] > 0) wait_bar(&full[i], (fills[i] - 1) & 1u, abort_flag);
+  }
+};
 
 template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -481,15 +649,25 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, fl
 }
 
 // Epilogue of one row: O / l -> out (bf16/fp16, 16-byte stores), LSE -> lse.
-// A row that saw no visible key (l = 0; O is then 0 too) gets O = 0 and
-// LSE = -inf.  Arrives on o_free (one arrival per warp) as soon as O has been
-// read.
+// A sink logit (sink_l2 > -inf, log2 units) joins the normalisation: with
+// M = max(m, sink), l' = l 2^(m-M) + 2^(sink-M) and O' = O 2^(m-M), so the
+// row gets O / (l + 2^(sink-m)) and LSE = M + log2 l' without overflow.  A
+// row that saw no visible key (l = 0; O is then 0 too) gets O = 0 and
+// LSE = the sink, or -inf without one.  Arrives on o_free (one arrival per
+// warp) as soon as O has been read.
 template <int D, bool BF16>
-__device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, bool row_valid,
-                                             uint16_t *orow_ptr, float *lse_ptr,
+__device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, float sink_l2,
+                                             bool row_valid, uint16_t *orow_ptr, float *lse_ptr,
                                              uint64_t *o_free, int lane) {
+  float o_scale = 1.f;
+  if (sink_l2 != -INFINITY) {
+    const float M = fmaxf(m, sink_l2);
+    o_scale = ptx::ex2_approx(m - M);  // 0 when m = -inf
+    l = l * o_scale + ptx::ex2_approx(sink_l2 - M);
+    m = M;
+  }
   const bool any = l > 0.f;
-  const float inv_l = any ? 1.f / l : 0.f;
+  const float inv_l = any ? o_scale / l : 0.f;
 #pragma unroll
   for (int c0 = 0; c0 < D; c0 += 32) {
     uint32_t o[32];
@@ -513,13 +691,14 @@ __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, bool
   if (row_valid) *lse_ptr = any ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
 }
 
-// A query row whose sequence has no key: O = 0, LSE = -inf.
+// A query row of an item without visible keys: O = 0, LSE = the sink logit
+// (natural log units) or -inf without one.
 template <int D>
-__device__ __forceinline__ void empty_row(uint16_t *orow_ptr, float *lse_ptr) {
+__device__ __forceinline__ void empty_row(uint16_t *orow_ptr, float *lse_ptr, float sink_l2) {
   uint4 *dst = reinterpret_cast<uint4 *>(orow_ptr);
 #pragma unroll
   for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-  *lse_ptr = -INFINITY;
+  *lse_ptr = sink_l2 * 0.69314718055994530942f;
 }
 
 }  // namespace vattn

@@ -127,47 +127,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     {
       Scheduler<BN> sched;
       sched.init(p);
-      uint32_t rs = 0, rph = 0;
-      uint32_t slot = 0, phase = 0, q_count = 0;
-      uint32_t slot_fills[NSLOT];
-      for (int s = 0; s < NSLOT; ++s) slot_fills[s] = 0;
+      uint32_t rs = 0, rph = 0, q_count = 0;
       bool ok = true;
-      const uint64_t pol_kv = ptx::policy_evict_last();
-      auto load_kv = [&](const CUtensorMap *tm, int kv_h, int row) -> bool {
-        if (!wait_bar(&bars->empty[slot], phase ^ 1u, abort_flag)) return false;
-        uint8_t *dst = sKV + slot * KV_BYTES;
-        ptx::mbar_arrive_expect_tx(&bars->full[slot], KV_BYTES);
-#pragma unroll
-        for (int db = 0; db < DB; ++db)
-          ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &bars->full[slot], db * 64, kv_h, row,
-                                pol_kv);
-        ++slot_fills[slot];
-        if (++slot == NSLOT) {
-          slot = 0;
-          phase ^= 1u;
-        }
-        return true;
-      };
-      // Ring order per item: K0, K1, V0, K2, V1, K3, ..., V(n-1) — the order
-      // in which the MMA warp consumes them.
-      // Loads of one item, issued by lane 0; false when a bounded wait gave up.
-      auto load_item = [&](const WorkItem &w) -> bool {
-        const int n = w.n_kv;
-        bool ok = true;
-        const int kv_h = w.hu / p.group;
-        if (!load_kv(&tm_k, kv_h, w.k0)) return false;
+      KVProducer<BN, D, NSLOT> kv;
+      kv.init(sKV, bars->full, bars->empty, abort_flag);
+      // Q tile of an item (lane 0)
+      auto load_q = [&](const WorkItem &w) -> bool {
         if (!wait_bar(&bars->q_empty, (q_count & 1u) ^ 1u, abort_flag)) return false;
         ptx::mbar_arrive_expect_tx(&bars->q_full, Q_BYTES);
 #pragma unroll
         for (int db = 0; db < DB; ++db)
           ptx::tma_load_3d(sQ + db * (BM * 128), &tm_q, &bars->q_full, db * 64, w.hu, w.q0);
         ++q_count;
-        if (n >= 2) ok = load_kv(&tm_k, kv_h, w.k0 + BN);
-        for (int j = 0; ok && j < n; ++j) {
-          ok = load_kv(&tm_v, kv_h, w.k0 + j * BN);
-          if (ok && j + 2 < n) ok = load_kv(&tm_k, kv_h, w.k0 + (j + 2) * BN);
-        }
-        return ok;
+        return true;
       };
       for (;;) {
         WorkItem w;
@@ -186,14 +158,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!have || !ok) break;
-        if (lane == 0 && w.n_kv > 0) ok = load_item(w);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (w.n_kv > 0)
+          ok = kv.load_item(p, w, w.hu / p.group, &tm_k, &tm_v, [&]() { return load_q(w); });
         if (!ok) break;
       }
       if (lane == 0) {
-        // Drain: every copy this thread issued has landed before the CTA exits.
-        for (int s = 0; s < NSLOT; ++s)
-          if (slot_fills[s] > 0) wait_bar(&bars->full[s], (slot_fills[s] - 1) & 1u, abort_flag);
+        // Drain: every copy this warp issued has landed before the CTA exits.
+        kv.drain();
         if (q_count > 0) wait_bar(&bars->q_full, (q_count - 1) & 1u, abort_flag);
       }
     }
@@ -316,7 +287,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const size_t orow = (size_t)(w.q0 + r) * p.H + w.hu;  // row index into [total_q, H]
       uint16_t *orow_ptr = reinterpret_cast<uint16_t *>(p.out) + orow * D;
       if (n == 0) {
-        if (row_valid) empty_row<D>(orow_ptr, p.lse + orow);
+        if (row_valid) empty_row<D>(orow_ptr, p.lse + orow, sink_log2(p, w.hu));
         continue;
       }
       // visible keys of this row, relative to the first visited key tile
@@ -358,7 +329,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      epilogue_row<D, BF16>(tO, m, l, row_valid, orow_ptr, p.lse + orow, &bars->o_free, lane);
+      epilogue_row<D, BF16>(tO, m, l, sink_log2(p, w.hu), row_valid, orow_ptr, p.lse + orow,
+                            &bars->o_free, lane);
     }
   }
 

@@ -134,14 +134,26 @@ static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_
 
 using namespace vattn;
 
+static int gcd_int(int a, int b) {
+  while (b) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  return a;
+}
+
 // Common body of the entry points.  window_left / window_right < 0 mean "no
-// bound"; seqused_k may be NULL.
+// bound"; seqused_k may be NULL unless page_table is given; page_table NULL =
+// packed k/v.
 static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *cu_seqlens_q,
                     const int32_t *cu_seqlens_k, int batch, int64_t total_q, int64_t total_k,
                     int max_seqlen_q, int max_seqlen_k, int num_heads, int num_kv_heads,
                     int head_dim, int causal, float scale, int window_left, int window_right,
-                    const int32_t *seqused_k, varlen_dtype_t dtype, void *out, float *lse,
-                    varlen_stream_t stream) {
+                    const int32_t *seqused_k, const int32_t *page_table, int page_table_stride,
+                    int page_size, const float *sinks, varlen_dtype_t dtype, void *out,
+                    float *lse, varlen_stream_t stream) {
+  const bool paged = page_table != nullptr;
   // ---- host-side validation: nothing is launched or touched on error
   if (dtype != VARLEN_BF16 && dtype != VARLEN_FP16) return VARLEN_ERR_DTYPE;
   if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
@@ -151,13 +163,17 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   if (head_dim != 64 && head_dim != 128 && head_dim != 256) return VARLEN_ERR_SHAPE;
   if (total_q >= (int64_t(1) << 31) || total_k >= (int64_t(1) << 31)) return VARLEN_ERR_SHAPE;
   if (num_heads > 65535) return VARLEN_ERR_SHAPE;
-  if (batch > 0 && (!cu_seqlens_q || !cu_seqlens_k)) return VARLEN_ERR_NULL;
+  if (paged && (page_size < 16 || page_size % 16 != 0 || page_table_stride < 1 ||
+                total_k % page_size != 0))
+    return VARLEN_ERR_SHAPE;
+  if (batch > 0 && (!cu_seqlens_q || (!paged && !cu_seqlens_k))) return VARLEN_ERR_NULL;
+  if (paged && batch > 0 && !seqused_k) return VARLEN_ERR_NULL;
   if (total_q > 0 && (!q || !out || !lse)) return VARLEN_ERR_NULL;
   if (total_k > 0 && (!k || !v)) return VARLEN_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return VARLEN_ERR_ALIGN;
   if (!aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
-      !aligned(seqused_k, 4))
+      !aligned(seqused_k, 4) || !aligned(page_table, 4) || !aligned(sinks, 4))
     return VARLEN_ERR_ALIGN;
   if (batch == 0 || total_q == 0) return VARLEN_OK;
 
@@ -202,9 +218,12 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   if (!encode_qkv_map(enc, &tq, q, bf16, total_q, num_heads, D, BM >> pack_log2,
                       1 << pack_log2))
     return VARLEN_ERR_LAUNCH;
+  // paged: a key tile is fetched as boxes of `chunk` rows, which divide both
+  // the page and the tile, so that no box crosses a page
+  const int chunk = paged ? gcd_int(page_size, BN) : BN;
   if (total_k > 0) {
-    if (!encode_qkv_map(enc, &tk, k, bf16, total_k, num_kv_heads, D, BN) ||
-        !encode_qkv_map(enc, &tv, v, bf16, total_k, num_kv_heads, D, BN))
+    if (!encode_qkv_map(enc, &tk, k, bf16, total_k, num_kv_heads, D, chunk) ||
+        !encode_qkv_map(enc, &tv, v, bf16, total_k, num_kv_heads, D, chunk))
       return VARLEN_ERR_LAUNCH;
   }
 
@@ -229,9 +248,18 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   // Window bounds in canonical form: a bound that no query of the buffers can
   // reach is dropped (this also keeps qi - left and qi + right + 1 in range),
   // and the causal rule is the right bound 0.
+  // (a sequence has at most total_k keys, or page_table_stride pages of keys when paged: pages
+  // may be shared, so a paged sequence can hold more keys than the cache has rows)
+  const int64_t key_extent = paged ? (int64_t)page_table_stride * page_size : total_k;
   kp.win_left = (window_left >= 0 && (int64_t)window_left < total_q) ? window_left : -1;
-  kp.win_right = (window_right >= 0 && (int64_t)window_right < total_k) ? window_right : -1;
+  kp.win_right = (window_right >= 0 && (int64_t)window_right < key_extent) ? window_right : -1;
   if (causal) kp.win_right = 0;
+  kp.page_table = page_table;
+  kp.pt_stride = paged ? page_table_stride : 0;
+  kp.page_size = paged ? page_size : 0;
+  kp.num_pages = paged ? (int)(total_k / page_size) : 0;
+  kp.page_chunk = chunk;
+  kp.sinks = sinks;
 
   // Upper bound of work items from max_seqlen_q; at least one CTA so that an
   // understated bound never drops work (the CTAs loop over all items).
@@ -270,7 +298,7 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
                                   float *lse, varlen_stream_t stream) {
   return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                   max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, -1, -1, nullptr,
-                  dtype, out, lse, stream);
+                  nullptr, 0, 0, nullptr, dtype, out, lse, stream);
 }
 
 extern "C" int varlen_attn_fwd_v2(const void *q, const void *k, const void *v,
@@ -282,7 +310,22 @@ extern "C" int varlen_attn_fwd_v2(const void *q, const void *k, const void *v,
                                   float *lse, varlen_stream_t stream) {
   return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                   max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, window_left,
-                  window_right, seqused_k, dtype, out, lse, stream);
+                  window_right, seqused_k, nullptr, 0, 0, nullptr, dtype, out, lse, stream);
+}
+
+extern "C" int varlen_attn_fwd_v3(const void *q, const void *k, const void *v,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                  int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
+                                  int max_seqlen_k, int num_heads, int num_kv_heads, int head_dim,
+                                  int causal, float scale, int window_left, int window_right,
+                                  const int32_t *seqused_k, const int32_t *page_table,
+                                  int page_table_stride, int page_size, const float *sinks,
+                                  varlen_dtype_t dtype, void *out, float *lse,
+                                  varlen_stream_t stream) {
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, window_left,
+                  window_right, seqused_k, page_table, page_table_stride, page_size, sinks, dtype,
+                  out, lse, stream);
 }
 
 extern "C" int varlen_attn_fwd(const void *q, const void *k, const void *v,
@@ -313,7 +356,8 @@ extern "C" const char *varlen_attn_strerror(int code) {
     case VARLEN_ERR_LAUNCH:
       return "CUDA launch or tensor-map setup failed";
     case VARLEN_ERR_DEVICE:
-      return "device-side status word is set (a bounded pipeline wait timed out)";
+      return "device-side status word is set (a bounded pipeline wait timed out, or a page-table "
+             "entry was out of range)";
     case VARLEN_ERR_ARCH:
       return "current device is not compute capability 10.0 (sm_100a build)";
     default:
@@ -333,4 +377,4 @@ extern "C" int varlen_attn_device_status(unsigned int *status, int clear) {
   return VARLEN_OK;
 }
 
-extern "C" int varlen_attn_abi_version(void) { return 2; }
+extern "C" int varlen_attn_abi_version(void) { return 3; }

@@ -147,6 +147,60 @@ int varlen_attn_fwd_v2(const void *q, const void *k, const void *v,
                        const int32_t *seqused_k, varlen_dtype_t dtype,
                        void *out, float *lse, varlen_stream_t stream);
 
+/*
+ * varlen_attn_fwd_v3 — varlen_attn_fwd_v2 plus paged K/V and attention
+ * sinks.  Paged K/V: the page_table
+ * argument of the varlen forward schema in PyTorch pull request #176015 (its
+ * follow-up #175924 "add page_table"), with the cache layout of the
+ * PageAttention form of the Ascend sparse shared-KV attention page: a cache of
+ * num_pages blocks of page_size tokens, [num_pages, page_size, Hkv, D], a
+ * block table with one row per sequence, and the key lengths taken from the
+ * used-key counts (cu_seqlens_k is not read in that form).
+ *
+ *   page_table   NULL: k and v are packed exactly as in v2 (the remaining two
+ *                arguments are ignored).  Otherwise an int32 device array
+ *                [batch, page_table_stride] (4-byte aligned): logical page j of
+ *                sequence b is cache page page_table[b * page_table_stride + j],
+ *                so key ki of sequence b is row
+ *                  page_table[b * stride + ki / page_size] * page_size + ki % page_size
+ *                of k and v viewed as [total_k, Hkv, D].  Pages may be shared
+ *                between sequences.
+ *   page_table_stride   entries per table row (>= 1); a sequence addresses at
+ *                most page_table_stride * page_size keys.
+ *   page_size    keys per page: a positive multiple of 16 dividing total_k
+ *                (total_k = num_pages * page_size).
+ *
+ * With page_table != NULL, seqused_k is required and gives the number of keys
+ * of each sequence (a negative entry counts as 0, one above
+ * page_table_stride * page_size as that), cu_seqlens_k may be NULL, and only
+ * the table entries of pages holding used keys are read.  A table entry
+ * outside [0, num_pages) is never dereferenced: its keys read as zeros and
+ * bit 2 of the device status word is set.  The rows of a page past the used
+ * keys may be read (weight exactly 0) and must hold finite values.
+ *
+ * sinks        NULL, or a float32 device array [num_heads] (4-byte aligned):
+ *              attention sinks, the FLOAT32 per-head "sinks" input of the
+ *              Ascend sparse shared-KV attention page (which gives no
+ *              formula).  sinks[h] is one more logit in the softmax of every
+ *              row of query head h, in score units (not multiplied by scale),
+ *              with no value row:
+ *                m = max(max_ki s_ki, sinks[h]),
+ *                l = sum_ki exp(s_ki - m) + exp(sinks[h] - m),
+ *                out = sum_ki exp(s_ki - m) / l * V_ki,  lse = m + ln l.
+ *              A row without visible keys then gets out = 0, lse = sinks[h].
+ *
+ * Everything else is as in v2 (window rule, empty rows, ownership, errors).
+ */
+int varlen_attn_fwd_v3(const void *q, const void *k, const void *v,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       int batch, int64_t total_q, int64_t total_k,
+                       int max_seqlen_q, int max_seqlen_k,
+                       int num_heads, int num_kv_heads, int head_dim,
+                       int causal, float scale, int window_left, int window_right,
+                       const int32_t *seqused_k, const int32_t *page_table,
+                       int page_table_stride, int page_size, const float *sinks,
+                       varlen_dtype_t dtype, void *out, float *lse, varlen_stream_t stream);
+
 /* Static, human-readable description of a status code.  Never NULL. */
 const char *varlen_attn_strerror(int code);
 
@@ -155,13 +209,13 @@ const char *varlen_attn_strerror(int code);
  * kernels is bounded; a wait that runs out (which does not happen in a
  * correct launch) ORs a bit into this word, the kernel drains its own
  * in-flight copies and returns instead of hanging.  Bits: 1 = pipeline wait
- * timed out.  Reads the word synchronously into *status (device-wide,
- * shared by all launches of this library on the device); clears it when
- * clear != 0.  Returns VARLEN_OK or VARLEN_ERR_LAUNCH / VARLEN_ERR_NULL.
+ * timed out; 2 = a page-table entry was outside [0, num_pages) (v3).  Reads
+ * the word synchronously into *status (device-wide, shared by all launches of
+ * this library on the device); clears it when clear != 0.  Returns VARLEN_OK or VARLEN_ERR_LAUNCH / VARLEN_ERR_NULL.
  */
 int varlen_attn_device_status(unsigned int *status, int clear);
 
-/* Library ABI version: 2 for this header (v2 added; v1 unchanged). */
+/* Library ABI version: 3 for this header (v2 and v3 added; v1 unchanged). */
 int varlen_attn_abi_version(void);
 
 #ifdef __cplusplus

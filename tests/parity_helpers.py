@@ -7,9 +7,9 @@ output buffers carry guard rows before and after the packed extents, filled
 with a canary, and must come back with every packed row written (no NaN
 pre-fill left) and every guard row untouched.
 
-``mask`` (optional dict: window_left, window_right, seqused_k) selects the
-sliding-window / used-key form of the forward; the same dict goes to the
-oracle.
+``mask`` (optional dict: window_left, window_right, seqused_k, sinks) selects
+the sliding-window / used-key / sink form of the forward; the same dict goes
+to the oracle.
 """
 import numpy as np
 import torch
@@ -21,8 +21,10 @@ O_MAX, O_MEAN, LSE_MAX = 1.5e-2, 2e-3, 5e-3
 GUARD = 3
 
 
-def run_gpu(case, scale=None, guard=GUARD, max_q=None, max_k=None, mask=None):
+def run_gpu(case, scale=None, guard=GUARD, max_q=None, max_k=None, mask=None, paged=None):
     """Runs the CUDA forward with NaN-filled outputs inside guard rows.
+    ``paged`` (a workloads.PagedKV) replaces the packed K/V by its page cache,
+    page table and key counts (mask's seqused_k, if any, wins).
     Returns (out float64 [Tq,H,D], lse float64 [Tq,H], raw out, raw lse)."""
     import flash_attention_fwd_b200 as fa
     mask = mask or {}
@@ -41,12 +43,23 @@ def run_gpu(case, scale=None, guard=GUARD, max_q=None, max_k=None, mask=None):
     out = out_buf[guard:guard + Tq]
     lse = lse_buf[guard:guard + Tq]
     used = mask.get("seqused_k")
+    table = None
+    if paged is not None:
+        k, v = paged.k_cache.to(dev), paged.v_cache.to(dev)
+        table = paged.page_table.to(dev)
+        ck = None
+        if used is None:
+            used = paged.seqused_k
     used_t = None if used is None else torch.tensor(list(used), dtype=torch.int32, device=dev)
+    sinks = mask.get("sinks")
+    sinks_t = None if sinks is None else torch.tensor(list(sinks), dtype=torch.float32,
+                                                      device=dev)
     fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q if max_q is None else max_q,
                        case.max_k if max_k is None else max_k, case.causal,
                        scale if scale is not None else case.scale, out=out, lse=lse,
                        window_size_left=mask.get("window_left", -1),
-                       window_size_right=mask.get("window_right", -1), seqused_k=used_t)
+                       window_size_right=mask.get("window_right", -1), seqused_k=used_t,
+                       page_table=table, sinks=sinks_t)
     torch.cuda.synchronize()
     ob, lb = out_buf.cpu(), lse_buf.cpu()
     assert torch.all(ob[:guard] == canary) and torch.all(ob[guard + Tq:] == canary), \
@@ -74,6 +87,8 @@ def check_close(out, lse, ref_out, ref_lse, what=""):
 
 
 def full_check(case, mask=None, **kw):
+    """Whole output against the oracle (with a page cache, the oracle reads
+    the packed K/V the cache was built from)."""
     out, lse, _, _ = run_gpu(case, mask=mask, **kw)
     ref_out, ref_lse = oracle.run_case(case, **(mask or {}))
     check_close(out, lse, ref_out, ref_lse, case.name)

@@ -28,7 +28,7 @@ def test_library_loads_and_exports_every_symbol():
     raw = ctypes.CDLL(fa.LIB_PATH)
     for name in header_functions():
         assert hasattr(raw, name), name
-    assert lib.varlen_attn_abi_version() == 2
+    assert lib.varlen_attn_abi_version() == 3
 
 
 def test_library_is_built_for_sm100a():
@@ -47,6 +47,11 @@ BASE = dict(q_ptr=0x10000, k_ptr=0x20000, v_ptr=0x30000, cu_q_ptr=0x40000, cu_k_
             batch=2, total_q=10, total_k=10, max_seqlen_q=5, max_seqlen_k=5, num_heads=4,
             num_kv_heads=2, head_dim=128, causal=True, scale=0.0, dtype_code=0,
             out_ptr=0x60000, lse_ptr=0x70000, stream=0)
+
+
+# paged K/V: 4 pages of 16 keys, cu_seqlens_k unused
+PAGED = dict(page_table_ptr=0x90000, page_table_stride=2, page_size=16, total_k=64,
+             seqused_k_ptr=0x80000, cu_k_ptr=0)
 
 
 @pytest.mark.parametrize("change,code", [
@@ -75,6 +80,17 @@ BASE = dict(q_ptr=0x10000, k_ptr=0x20000, v_ptr=0x30000, cu_q_ptr=0x40000, cu_k_
     (dict(window_left=2, q_ptr=0), -1),
     (dict(seqused_k_ptr=0x80002), -4),       # seqused_k needs 4-byte alignment
     (dict(window_left=1, window_right=1, lse_ptr=0x70001), -4),
+    # the v3 entry point (paged K/V)
+    (dict(PAGED, page_size=24), -2),         # not a multiple of 16
+    (dict(PAGED, page_size=0), -2),
+    (dict(PAGED, total_k=40), -2),           # not a whole number of pages
+    (dict(PAGED, page_table_stride=0), -2),
+    (dict(PAGED, seqused_k_ptr=0), -1),      # a page table needs seqused_k
+    (dict(PAGED, cu_q_ptr=0), -1),
+    (dict(PAGED, page_table_ptr=0x90002), -4),
+    (dict(PAGED, num_heads=5), -2),
+    (dict(sinks_ptr=0x90002), -4),           # sinks need 4-byte alignment
+    (dict(sinks_ptr=0x90000, head_dim=48), -2),
 ])
 def test_host_validation_rejects(change, code):
     args = dict(BASE)
@@ -91,6 +107,9 @@ def test_empty_problems_are_noops_without_device():
     assert fa.varlen_attn_fwd_raw(**args) == 0
     args = dict(BASE)
     args.update(batch=0, window_left=8, window_right=0, seqused_k_ptr=0x80000)
+    assert fa.varlen_attn_fwd_raw(**args) == 0
+    args = dict(BASE)
+    args.update(PAGED, total_q=0, q_ptr=0, out_ptr=0, lse_ptr=0)
     assert fa.varlen_attn_fwd_raw(**args) == 0
 
 

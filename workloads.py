@@ -51,6 +51,8 @@ class Workload:
     window_left: int = -1   # sliding window (negative = unbounded)
     window_right: int = -1
     seqused: bool = False   # draw a per-sequence used-key count
+    page_size: int = 0      # > 0: K/V held in a page cache of this many keys per page
+    sinks: bool = False     # draw one attention-sink logit per query head
 
 
 WORKLOADS = {
@@ -76,6 +78,14 @@ WORKLOADS = {
                             description="short-query/long-KV lengths with per-sequence used-key "
                                         "counts seqused_k in [Lk/2, Lk], H=32, Hkv=4, D=128, "
                                         "bf16, non-causal"),
+    "shortq_paged": Workload("shortq_paged", 4, 32, 4, 128, "bf16", False, page_size=16,
+                             description="short-query/long-KV lengths with K/V in a page cache of "
+                                         "16-key pages in seeded random order, H=32, Hkv=4, "
+                                         "D=128, bf16, non-causal"),
+    "gqa_sinks": Workload("gqa_sinks", 2, 32, 8, 128, "bf16", True, sinks=True,
+                          description="GQA prefill lengths with one attention-sink logit per "
+                                      "query head (uniform in [-2, 4]), H=32, Hkv=8, D=128, bf16, "
+                                      "causal"),
     # Profiling case only (not a benchmark configuration): the long ragged
     # prefill lengths with a quarter of its heads, so that a many-pass profiler
     # capture stays small while its inputs still exceed the L2 cache.
@@ -107,14 +117,14 @@ def seqlens(name: str):
     if name == "tiny":
         q = [17, 64, 1]
         return q, list(q)
-    if name == "gqa":
+    if name in ("gqa", "gqa_sinks"):
         rng = np.random.default_rng(w.seed)
         q = [int(x) for x in rng.integers(128, 2049, 8)]
         return q, list(q)
     if name in ("long", "long_h16", "long_swa"):
         q = _long_lengths(w.seed)
         return q, list(q)
-    if name in ("shortq", "shortq_used"):
+    if name in ("shortq", "shortq_used", "shortq_paged"):
         rng = np.random.default_rng(w.seed)
         q = [int(x) for x in rng.integers(1, 65, 32)]
         k = [int(x) for x in rng.integers(512, 8193, 32)]
@@ -152,6 +162,10 @@ def mask_of(name: str) -> dict:
     used = seqused_k(name)
     if used is not None:
         m["seqused_k"] = used
+    if w.sinks:
+        # float32 values, so that the oracle and the kernels see the same logits
+        g = np.random.default_rng(w.seed + 1000)
+        m["sinks"] = [float(x) for x in g.uniform(-2.0, 4.0, w.H).astype(np.float32)]
     return m
 
 
@@ -250,3 +264,46 @@ def sample_rows(case: Case, n: int, seed: int = 1234) -> np.ndarray:
         rows.update(zip(toks.tolist(), hs.tolist()))
     arr = np.array(sorted(rows), dtype=np.int64).reshape(-1, 2)
     return arr
+
+
+# ----------------------------------------------------------------------------- paged K/V
+
+@dataclass
+class PagedKV:
+    k_cache: torch.Tensor      # [num_pages, page_size, Hkv, D]
+    v_cache: torch.Tensor
+    page_table: torch.Tensor   # int32 [B, pages_per_seq], -1 past each sequence's pages
+    seqused_k: List[int]       # keys of each sequence
+    page_size: int
+
+
+def to_paged(case: Case, page_size: int, seed: int = 0, spare_pages: int = 3,
+             fill: float = 7.0, table_pad: int = 1) -> PagedKV:
+    """Scatters the packed keys/values of ``case`` into a page cache: each
+    sequence's keys fill ceil(Lk / page_size) pages taken in a seeded random
+    order from a pool with ``spare_pages`` unused pages; key ki of sequence b
+    goes to row ki % page_size of page page_table[b, ki // page_size].  Rows
+    that hold no key (the tail of a sequence's last page, the spare pages) get
+    the finite value ``fill``; table entries past a sequence's pages are -1
+    (``table_pad`` extra columns of them)."""
+    rng = np.random.default_rng(seed)
+    need = [-(-lk // page_size) for lk in case.lens_k]
+    num_pages = sum(need) + spare_pages
+    order = rng.permutation(num_pages)
+    width = max(need + [0]) + table_pad
+    table = torch.full((case.B, max(width, 1)), -1, dtype=torch.int32)
+    shape = (num_pages, page_size, case.Hkv, case.D)
+    kc = torch.full(shape, fill, dtype=case.k.dtype)
+    vc = torch.full(shape, fill, dtype=case.v.dtype)
+    cu = case.cu_k.tolist()
+    nxt = 0
+    for b in range(case.B):
+        for j in range(need[b]):
+            pg = int(order[nxt])
+            nxt += 1
+            table[b, j] = pg
+            lo = cu[b] + j * page_size
+            hi = min(cu[b + 1], lo + page_size)
+            kc[pg, :hi - lo] = case.k[lo:hi]
+            vc[pg, :hi - lo] = case.v[lo:hi]
+    return PagedKV(kc, vc, table, list(case.lens_k), page_size)
