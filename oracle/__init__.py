@@ -63,6 +63,9 @@ def _bind(lib):
     lib.oracle_varlen_attn_rows_ext.argtypes = [P, P, P, i32, P, P, P, i32, i32, i32, i32,
                                                 i32, i32, i32, P, f64, P, P, i64, P, P, i32]
     lib.oracle_varlen_attn_rows_ext.restype = i32
+    lib.oracle_varlen_attn_bwd.argtypes = [P, P, P, P, P, P, i32, P, P, i32, i32, i32, i32,
+                                           i32, f64, P, P, P, i32]
+    lib.oracle_varlen_attn_bwd.restype = i32
     return lib
 
 
@@ -95,6 +98,13 @@ def _bits(t: torch.Tensor) -> np.ndarray:
 
 def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f64(x) -> np.ndarray:
+    """Any float tensor or array, widened exactly to a C-contiguous float64 array."""
+    if isinstance(x, torch.Tensor):
+        x = x.detach().cpu().to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
 
 
 def decode16(bits: int, dtype: str) -> float:
@@ -188,3 +198,36 @@ def run_case_rows(case, rows, nthreads=None, **mask):
     return varlen_attn_rows(case.q, case.k, case.v, case.cu_q.numpy(), case.cu_k.numpy(),
                             case.H, case.Hkv, case.D, case.causal, case.scale, case.dtype,
                             rows, nthreads, **mask)
+
+
+def varlen_attn_bwd(dout, q, k, v, out, lse, cu_q, cu_k, H, Hkv, D, causal, scale, dtype,
+                    nthreads=None, lib=None):
+    """fp64 backward of the page's loop.  dout/q [Tq,H,D] and k/v [Tk,Hkv,D]
+    are bf16/fp16 tensors; out [Tq,H,D] and lse [Tq,H] any float tensor or
+    array (widened to double).  Returns (dq [Tq,H,D], dk [Tk,Hkv,D],
+    dv [Tk,Hkv,D]) float64."""
+    lib = lib or _load()
+    db, qb, kb, vb = _bits(dout), _bits(q), _bits(k), _bits(v)
+    ob = _f64(out)
+    lse_d = _f64(lse)
+    cq = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
+    ck = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int32))
+    B = len(cq) - 1
+    Tq, Tk = int(cq[-1]), int(ck[-1])
+    dq = np.zeros((Tq, H, D), dtype=np.float64)
+    dk = np.zeros((Tk, Hkv, D), dtype=np.float64)
+    dv = np.zeros((Tk, Hkv, D), dtype=np.float64)
+    rc = lib.oracle_varlen_attn_bwd(_ptr(db), _ptr(qb), _ptr(kb), _ptr(vb), _ptr(ob),
+                                    _ptr(lse_d), DTYPE_CODE[dtype], _ptr(cq), _ptr(ck), B, H, Hkv,
+                                    D, int(bool(causal)), float(scale), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("oracle_varlen_attn_bwd failed with code %d" % rc)
+    return dq, dk, dv
+
+
+def run_case_bwd(case, dout, out, lse, nthreads=None, lib=None):
+    """Backward of a ``workloads.Case`` for the given dO, O and LSE."""
+    return varlen_attn_bwd(dout, case.q, case.k, case.v, out, lse, case.cu_q.numpy(),
+                           case.cu_k.numpy(), case.H, case.Hkv, case.D, case.causal, case.scale,
+                           case.dtype, nthreads, lib=lib)

@@ -41,6 +41,29 @@
  * * V_ki, LSE = m + ln(l); a row without visible keys then gets O = 0 and
  * LSE = sinks[h].
  *
+ * Backward (oracle_varlen_attn_bwd): the CPU backward loop of the same page
+ * (VarLenAttentionOps::varlen_attention_bwd), step for step in double
+ * precision.  Given dO, Q, K, V, the forward output O and LSE:
+ *
+ *   for each sequence b, query head h (kv_h = h / (H / Hkv)), query qi:
+ *     delta = sum_d dO[qi, h, d] * O[qi, h, d]
+ *     for each visible key ki (causal: skip qi < ki):
+ *       s  = scale * <Q[qi, h], K[ki, kv_h]>
+ *       p  = exp(s - LSE[qi, h])                 (the softmax weight)
+ *       dp = <V[ki, kv_h], dO[qi, h]>
+ *       ds = p * (dp - delta)
+ *       dQ[qi, h]     += scale * ds * K[ki, kv_h]
+ *       dK[ki, kv_h]  += scale * ds * Q[qi, h]
+ *       dV[ki, kv_h]  += p * dO[qi, h]
+ *
+ * dK and dV sum over the H / Hkv query heads of their key/value head.  The
+ * scale is the page's 1/sqrt(D) unless given (as in the forward).  dO is
+ * 16-bit like Q/K/V; O and LSE are given in double (the caller widens the
+ * stored bf16/fp16 O and float32 LSE exactly, or passes exact values).  Work items are (b, kv_h): each owns the dK/dV rows
+ * of that key/value head of sequence b and the dQ rows of its query heads,
+ * and runs the loop above serially, so the result does not depend on the
+ * thread count.
+ *
  * Inputs are bf16 or fp16 bit patterns; they are widened exactly to double
  * before any arithmetic.  The widening of a key/value head of one sequence
  * is done once per (b, h) work item; that is a format conversion, not a
@@ -369,4 +392,97 @@ int oracle_varlen_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t
     return oracle_varlen_attn_rows_ext(q, k, v, dtype, cu_q, cu_k, NULL, B, H, Hkv, D, causal,
                                        -1, -1, NULL, scale, row_tok, row_head, nrows, out_rows,
                                        lse_rows, nthreads);
+}
+
+
+/* ------------------------------------------------------------------ backward */
+
+typedef struct {
+    const uint16_t *dout, *q, *k, *v;
+    const double *o, *lse;
+    int dtype;
+    const int32_t *cu_q, *cu_k;
+    int B, H, Hkv, D, causal;
+    double scale;
+    double *dq, *dk, *dv;
+    int64_t next_item, n_items;
+    int status;
+} OracleBwdCtx;
+
+static double bwd_elem(const OracleBwdCtx *c, const uint16_t *t, size_t off) {
+    return oracle_decode16(t[off], c->dtype);
+}
+
+static void *bwd_worker(void *arg) {
+    OracleBwdCtx *c = (OracleBwdCtx *)arg;
+    const int D = c->D, H = c->H, Hkv = c->Hkv, G = c->H / c->Hkv;
+    for (;;) {
+        int64_t item = __atomic_fetch_add(&c->next_item, 1, __ATOMIC_RELAXED);
+        if (item >= c->n_items) break;
+        int b = (int)(item / Hkv), kv_h = (int)(item % Hkv);
+        int q0 = c->cu_q[b], Lq = c->cu_q[b + 1] - c->cu_q[b];
+        int k0 = c->cu_k[b], Lk = c->cu_k[b + 1] - c->cu_k[b];
+        for (int h = kv_h * G; h < (kv_h + 1) * G; ++h) {
+            for (int qi = 0; qi < Lq; ++qi) {
+                size_t qoff = ((size_t)(q0 + qi) * H + h) * D;
+                double lse = c->lse[(size_t)(q0 + qi) * H + h];
+                double delta = 0.0;
+                for (int d = 0; d < D; ++d)
+                    delta += bwd_elem(c, c->dout, qoff + d) * c->o[qoff + d];
+                for (int ki = 0; ki < Lk; ++ki) {
+                    if (c->causal && qi < ki) continue;
+                    size_t koff = ((size_t)(k0 + ki) * Hkv + kv_h) * D;
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dot += bwd_elem(c, c->q, qoff + d) * bwd_elem(c, c->k, koff + d);
+                    double prob = exp(dot * c->scale - lse);
+                    double dp = 0.0;
+                    for (int d = 0; d < D; ++d)
+                        dp += bwd_elem(c, c->v, koff + d) * bwd_elem(c, c->dout, qoff + d);
+                    double ds = prob * (dp - delta);
+                    for (int d = 0; d < D; ++d) {
+                        c->dq[qoff + d] += c->scale * ds * bwd_elem(c, c->k, koff + d);
+                        c->dk[koff + d] += c->scale * ds * bwd_elem(c, c->q, qoff + d);
+                        c->dv[koff + d] += prob * bwd_elem(c, c->dout, qoff + d);
+                    }
+                }
+            }
+        }
+    }
+    return NULL;
+}
+
+/* Full backward: writes dq[Tq*H*D], dk[Tk*Hkv*D], dv[Tk*Hkv*D] (zeroed first
+ * over the packed extents cu_q[B] / cu_k[B]).  Returns 0 or a negative code. */
+int oracle_varlen_attn_bwd(const uint16_t *dout, const uint16_t *q, const uint16_t *k,
+                           const uint16_t *v, const double *o, const double *lse, int dtype,
+                           const int32_t *cu_q, const int32_t *cu_k, int B, int H, int Hkv,
+                           int D, int causal, double scale, double *dq, double *dk, double *dv,
+                           int nthreads) {
+    int rc = check_args(B, H, Hkv, D, dtype);
+    if (rc) return rc;
+    OracleBwdCtx c;
+    memset(&c, 0, sizeof c);
+    c.dout = dout; c.q = q; c.k = k; c.v = v; c.o = o; c.lse = lse; c.dtype = dtype;
+    c.cu_q = cu_q; c.cu_k = cu_k;
+    c.B = B; c.H = H; c.Hkv = Hkv; c.D = D; c.causal = causal != 0;
+    c.scale = effective_scale(scale, D);
+    c.dq = dq; c.dk = dk; c.dv = dv;
+    if (B > 0) {
+        memset(dq, 0, (size_t)cu_q[B] * H * D * sizeof(double));
+        memset(dk, 0, (size_t)cu_k[B] * Hkv * D * sizeof(double));
+        memset(dv, 0, (size_t)cu_k[B] * Hkv * D * sizeof(double));
+    }
+    c.n_items = (int64_t)B * Hkv;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 512) nthreads = 512;
+    pthread_t tids[512];
+    int started = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        if (pthread_create(&tids[t], NULL, bwd_worker, &c) != 0) break;
+        ++started;
+    }
+    if (started == 0) bwd_worker(&c);
+    for (int t = 0; t < started; ++t) pthread_join(tids[t], NULL);
+    return c.status;
 }
