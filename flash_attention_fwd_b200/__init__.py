@@ -31,7 +31,7 @@ VARLEN_OK = 0
 STATUS_NAMES = {
     0: "VARLEN_OK", -1: "VARLEN_ERR_NULL", -2: "VARLEN_ERR_SHAPE", -3: "VARLEN_ERR_DTYPE",
     -4: "VARLEN_ERR_ALIGN", -5: "VARLEN_ERR_LAUNCH", -6: "VARLEN_ERR_DEVICE",
-    -7: "VARLEN_ERR_ARCH",
+    -7: "VARLEN_ERR_ARCH", -8: "VARLEN_ERR_WORKSPACE",
 }
 
 # Every symbol include/varlen_attn.h declares.
@@ -43,6 +43,8 @@ EXPORTED_SYMBOLS = (
     "varlen_attn_strerror",
     "varlen_attn_device_status",
     "varlen_attn_abi_version",
+    "varlen_attn_bwd_workspace_size",
+    "varlen_attn_bwd_v1",
 )
 
 _lock = threading.Lock()
@@ -76,6 +78,11 @@ def _bind(lib):
     lib.varlen_attn_device_status.restype = i32
     lib.varlen_attn_abi_version.argtypes = []
     lib.varlen_attn_abi_version.restype = i32
+    lib.varlen_attn_bwd_workspace_size.argtypes = [i64, i32]
+    lib.varlen_attn_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.varlen_attn_bwd_v1.argtypes = ([P] * 8 + [i32, i64, i64, i32, i32, i32, i32, i32, i32, f32,
+                                                  i32, P, P, P, P, ctypes.c_size_t, P])
+    lib.varlen_attn_bwd_v1.restype = i32
     return lib
 
 
@@ -243,3 +250,79 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return out, lse
+
+
+def bwd_workspace_size(total_q: int, num_heads: int) -> int:
+    """Bytes of device workspace ``varlen_attn_bwd`` needs."""
+    return int(load_library().varlen_attn_bwd_workspace_size(int(total_q), int(num_heads)))
+
+
+def varlen_attn_bwd_raw(dout_ptr: int, q_ptr: int, k_ptr: int, v_ptr: int, out_ptr: int,
+                        lse_ptr: int, cu_q_ptr: int, cu_k_ptr: int, batch: int, total_q: int,
+                        total_k: int, max_seqlen_q: int, max_seqlen_k: int, num_heads: int,
+                        num_kv_heads: int, head_dim: int, causal: bool, scale: float,
+                        dtype_code: int, dq_ptr: int, dk_ptr: int, dv_ptr: int,
+                        workspace_ptr: int, workspace_bytes: int, stream: int) -> int:
+    """Direct call of varlen_attn_bwd_v1 with integer addresses; returns the
+    status code unchanged."""
+    lib = load_library()
+    V = ctypes.c_void_p
+    return lib.varlen_attn_bwd_v1(V(dout_ptr), V(q_ptr), V(k_ptr), V(v_ptr), V(out_ptr),
+                                  V(lse_ptr), V(cu_q_ptr), V(cu_k_ptr), int(batch), int(total_q),
+                                  int(total_k), int(max_seqlen_q), int(max_seqlen_k),
+                                  int(num_heads), int(num_kv_heads), int(head_dim),
+                                  int(bool(causal)), float(scale), int(dtype_code), V(dq_ptr),
+                                  V(dk_ptr), V(dv_ptr), V(workspace_ptr), int(workspace_bytes),
+                                  V(stream))
+
+
+def varlen_attn_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                    out: torch.Tensor, lse: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                    cu_seqlens_k: torch.Tensor, max_seqlen_q: int, max_seqlen_k: int,
+                    causal: bool = False, scale: Optional[float] = None,
+                    dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+                    dv: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Gradients (dq, dk, dv) of the packed attention forward, given dO and
+    the forward's out and lse.  Shapes and dtypes as in ``varlen_attn_fwd``
+    (head dim 64 or 128); outputs and the workspace (``bwd_workspace_size``
+    bytes, uint8 on the device) are allocated here when not given."""
+    if q.dtype not in DTYPE_CODES or any(t.dtype != q.dtype for t in (k, v, dout, out)):
+        raise TypeError("dout, q, k, v, out must share dtype bfloat16 or float16")
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or dout.shape != q.shape \
+            or out.shape != q.shape:
+        raise ValueError("expected dout/q/out [Tq,H,D] and k, v [Tk,Hkv,D]")
+    for name, t in (("dout", dout), ("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse),
+                    ("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    total_q, H, D = q.shape
+    total_k, Hkv, _ = k.shape
+    if lse.dtype != torch.float32 or lse.shape != (total_q, H):
+        raise ValueError("lse must be float32 [Tq, H]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t.shape != ref.shape or t.dtype != ref.dtype or not t.is_contiguous():
+            raise ValueError("%s must be contiguous and shaped / typed like its input" % name)
+    need = bwd_workspace_size(total_q, H)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+
+    def addr(t):
+        return t.data_ptr() if t is not None and t.numel() else 0
+
+    with torch.cuda.device(q.device):
+        rc = varlen_attn_bwd_raw(
+            addr(dout), addr(q), addr(k), addr(v), addr(out), addr(lse), addr(cu_seqlens_q),
+            addr(cu_seqlens_k), cu_seqlens_q.numel() - 1, total_q, total_k, int(max_seqlen_q),
+            int(max_seqlen_k), H, Hkv, D, causal, 0.0 if scale is None else float(scale),
+            DTYPE_CODES[q.dtype], addr(dq), addr(dk), addr(dv), addr(workspace),
+            workspace.numel() * workspace.element_size(), stream.cuda_stream)
+    if rc != VARLEN_OK:
+        raise VarlenAttnError(rc, strerror(rc))
+    return dq, dk, dv

@@ -83,7 +83,7 @@ static bool encode_qkv_map(EncodeTiledFn enc, CUtensorMap *map, const void *base
 struct DeviceInfo {
   int sms = 0;
   int major = 0, minor = 0;
-  bool attr_set[16] = {};
+  bool attr_set[24] = {};
 };
 static DeviceInfo g_dev[64];
 
@@ -360,6 +360,8 @@ extern "C" const char *varlen_attn_strerror(int code) {
              "entry was out of range)";
     case VARLEN_ERR_ARCH:
       return "current device is not compute capability 10.0 (sm_100a build)";
+    case VARLEN_ERR_WORKSPACE:
+      return "workspace missing or smaller than varlen_attn_bwd_workspace_size()";
     default:
       return "unknown status code";
   }
@@ -377,4 +379,7 @@ extern "C" int varlen_attn_device_status(unsigned int *status, int clear) {
   return VARLEN_OK;
 }
 
-extern "C" int varlen_attn_abi_version(void) { return 3; }
+extern "C" int varlen_attn_abi_version(void) { return 4; }
+
+// Backward entry points (same translation unit: one device status word).
+#include "bwd_host.cuh"

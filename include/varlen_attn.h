@@ -33,6 +33,7 @@
 #ifndef VARLEN_ATTN_H_
 #define VARLEN_ATTN_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -59,6 +60,7 @@ typedef enum {
 #define VARLEN_ERR_LAUNCH (-5)      /* the CUDA launch itself failed (see varlen_attn_strerror) */
 #define VARLEN_ERR_DEVICE (-6)      /* device-side status word set (see varlen_attn_device_status) */
 #define VARLEN_ERR_ARCH (-7)        /* current device is not compute capability 10.0 (B200/B100 class) */
+#define VARLEN_ERR_WORKSPACE (-8)   /* backward: workspace NULL or smaller than varlen_attn_bwd_workspace_size */
 
 /*
  * varlen_attn_fwd_v1 — packed attention forward, output written in place.
@@ -215,7 +217,59 @@ const char *varlen_attn_strerror(int code);
  */
 int varlen_attn_device_status(unsigned int *status, int clear);
 
-/* Library ABI version: 3 for this header (v2 and v3 added; v1 unchanged). */
+/*
+ * Backward of the packed attention forward (varlen_attn_fwd_v1's operation):
+ * the CPU backward loop of boostr 0.2.0, src/ops/cpu/attention/
+ * varlen_attention.rs (VarLenAttentionOps::varlen_attention_bwd).  For every
+ * sequence b, query head h (kv_h = h / (H / Hkv)) and query qi, with
+ * delta = <dO[qi,h], O[qi,h]> and for every key ki visible to qi (causal: not
+ * qi < ki, sequence-local):
+ *   p  = exp(scale <Q[qi,h], K[ki,kv_h]> - LSE[qi,h])
+ *   ds = p (<V[ki,kv_h], dO[qi,h]> - delta)
+ *   dQ[qi,h] += scale ds K[ki,kv_h];   dK[ki,kv_h] += scale ds Q[qi,h];
+ *   dV[ki,kv_h] += p dO[qi,h]
+ * dK and dV of a key/value head sum over its H / Hkv query heads.
+ *
+ * varlen_attn_bwd_workspace_size — bytes of device workspace the backward
+ * needs for total_q query rows and num_heads query heads (0 when either is
+ * <= 0).  The workspace holds delta, float32 [total_q, H]; it needs no
+ * initialisation and its contents after a call are unspecified.
+ */
+size_t varlen_attn_bwd_workspace_size(int64_t total_q, int num_heads);
+
+/*
+ * varlen_attn_bwd_v1 — gradients of the forward with respect to q, k, v.
+ *
+ *   dout         [total_q, H, D] dtype: gradient of the loss with respect to out
+ *   q, k, v      the forward's inputs (layouts and rules as in varlen_attn_fwd_v1)
+ *   out, lse     the forward's outputs for these inputs (out dtype, lse float32)
+ *   cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+ *   max_seqlen_k, num_heads, num_kv_heads, causal, scale, dtype
+ *                as in varlen_attn_fwd_v1; head_dim must be 64 or 128.
+ *   dq           [total_q, H, D] dtype, written for rows [0, cu_seqlens_q[batch])
+ *   dk, dv       [total_k, Hkv, D] dtype, written for rows [0, cu_seqlens_k[batch]);
+ *                a key that no query sees gets zeros.
+ *   workspace    device buffer of at least varlen_attn_bwd_workspace_size(total_q,
+ *                num_heads) bytes, 16-byte aligned, owned by the caller; it must
+ *                not be used by another call running at the same time.
+ *   stream       CUDA stream of the two kernel launches.
+ *
+ * All tensors are device pointers owned by the caller (16-byte aligned;
+ * lse and cu_seqlens 4-byte); nothing is allocated.  Returns VARLEN_OK or a
+ * negative code (VARLEN_ERR_WORKSPACE when the workspace is missing or too
+ * small); every error but VARLEN_ERR_LAUNCH is detected before any launch.
+ */
+int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k, const void *v,
+                       const void *out, const float *lse,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       int batch, int64_t total_q, int64_t total_k,
+                       int max_seqlen_q, int max_seqlen_k,
+                       int num_heads, int num_kv_heads, int head_dim,
+                       int causal, float scale, varlen_dtype_t dtype,
+                       void *dq, void *dk, void *dv,
+                       void *workspace, size_t workspace_bytes, varlen_stream_t stream);
+
+/* Library ABI version: 4 for this header (v2, v3 and the backward added; v1 unchanged). */
 int varlen_attn_abi_version(void);
 
 #ifdef __cplusplus

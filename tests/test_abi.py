@@ -28,7 +28,7 @@ def test_library_loads_and_exports_every_symbol():
     raw = ctypes.CDLL(fa.LIB_PATH)
     for name in header_functions():
         assert hasattr(raw, name), name
-    assert lib.varlen_attn_abi_version() == 3
+    assert lib.varlen_attn_abi_version() == 4
 
 
 def test_library_is_built_for_sm100a():
@@ -38,7 +38,7 @@ def test_library_is_built_for_sm100a():
 
 
 def test_strerror_covers_codes():
-    for code in (0, -1, -2, -3, -4, -5, -6, -7, -99):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7, -8, -99):
         msg = fa.strerror(code)
         assert isinstance(msg, str) and msg
 
@@ -120,3 +120,38 @@ def test_product_module_does_not_import_oracle():
         if fn.endswith(".py"):
             src = open(os.path.join(pkg_dir, fn)).read()
             assert "oracle" not in re.sub(r'""".*?"""', "", src, flags=re.S), fn
+
+
+BWD = dict(dout_ptr=0x11000, q_ptr=0x10000, k_ptr=0x20000, v_ptr=0x30000, out_ptr=0x60000,
+           lse_ptr=0x70000, cu_q_ptr=0x40000, cu_k_ptr=0x50000, batch=2, total_q=10,
+           total_k=10, max_seqlen_q=5, max_seqlen_k=5, num_heads=4, num_kv_heads=2,
+           head_dim=128, causal=True, scale=0.0, dtype_code=0, dq_ptr=0x61000,
+           dk_ptr=0x62000, dv_ptr=0x63000, workspace_ptr=0x80000, workspace_bytes=4096,
+           stream=0)
+
+
+@pytest.mark.parametrize("change,code", [
+    (dict(head_dim=256), -2),                # the backward covers D = 64, 128
+    (dict(num_heads=5), -2),
+    (dict(dtype_code=3), -3),
+    (dict(dout_ptr=0), -1),
+    (dict(dk_ptr=0), -1),
+    (dict(cu_k_ptr=0), -1),
+    (dict(dq_ptr=0x61008), -4),
+    (dict(workspace_ptr=0x80008), -4),
+    (dict(workspace_ptr=0), -8),
+    (dict(workspace_bytes=100), -8),         # needs 10 * 4 * 4 bytes rounded up to 256
+])
+def test_backward_host_validation_rejects(change, code):
+    args = dict(BWD)
+    args.update(change)
+    assert fa.varlen_attn_bwd_raw(**args) == code
+
+
+def test_backward_workspace_size_and_empty_call():
+    assert fa.bwd_workspace_size(10, 4) == 256
+    assert fa.bwd_workspace_size(1000, 3) == 12032
+    assert fa.bwd_workspace_size(0, 4) == 0
+    args = dict(BWD)
+    args.update(batch=0)
+    assert fa.varlen_attn_bwd_raw(**args) == 0
