@@ -55,16 +55,16 @@ extern "C" size_t varlen_attn_bwd_workspace_size(int64_t total_q, int num_heads)
   return ((size_t)total_q * (size_t)num_heads * sizeof(float) + 255) & ~(size_t)255;
 }
 
-extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k, const void *v,
-                                  const void *out, const float *lse,
-                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
-                                  int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
-                                  int max_seqlen_k, int num_heads, int num_kv_heads, int head_dim,
-                                  int causal, float scale, varlen_dtype_t dtype, void *dq,
-                                  void *dk, void *dv, void *workspace, size_t workspace_bytes,
-                                  varlen_stream_t stream) {
-  using namespace vattn;
-  // ---- host-side validation: nothing is launched or touched on error
+namespace vattn {
+
+// Host-side validation of the backward's arguments except the workspace:
+// nothing is launched or touched on error.
+static int bwd_check_args(const void *dout, const void *q, const void *k, const void *v,
+                          const void *out, const float *lse, const int32_t *cu_seqlens_q,
+                          const int32_t *cu_seqlens_k, int batch, int64_t total_q,
+                          int64_t total_k, int max_seqlen_q, int max_seqlen_k, int num_heads,
+                          int num_kv_heads, int head_dim, varlen_dtype_t dtype, const void *dq,
+                          const void *dk, const void *dv) {
   if (dtype != VARLEN_BF16 && dtype != VARLEN_FP16) return VARLEN_ERR_DTYPE;
   if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0)
     return VARLEN_ERR_SHAPE;
@@ -77,11 +77,29 @@ extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k
   if (total_q > 0 && (!dout || !q || !out || !lse || !dq)) return VARLEN_ERR_NULL;
   if (total_k > 0 && (!k || !v || !dk || !dv)) return VARLEN_ERR_NULL;
   if (!aligned(dout, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
-      !aligned(out, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
-      !aligned(workspace, 16))
+      !aligned(out, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
     return VARLEN_ERR_ALIGN;
   if (!aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
     return VARLEN_ERR_ALIGN;
+  return VARLEN_OK;
+}
+
+}  // namespace vattn
+
+extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k, const void *v,
+                                  const void *out, const float *lse,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                  int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
+                                  int max_seqlen_k, int num_heads, int num_kv_heads, int head_dim,
+                                  int causal, float scale, varlen_dtype_t dtype, void *dq,
+                                  void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                                  varlen_stream_t stream) {
+  using namespace vattn;
+  int rc = bwd_check_args(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q,
+                          total_k, max_seqlen_q, max_seqlen_k, num_heads, num_kv_heads, head_dim,
+                          dtype, dq, dk, dv);
+  if (rc != VARLEN_OK) return rc;
+  if (!aligned(workspace, 16)) return VARLEN_ERR_ALIGN;
   if (total_q > 0 &&
       (!workspace || workspace_bytes < varlen_attn_bwd_workspace_size(total_q, num_heads)))
     return VARLEN_ERR_WORKSPACE;
