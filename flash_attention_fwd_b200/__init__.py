@@ -45,6 +45,7 @@ EXPORTED_SYMBOLS = (
     "varlen_attn_abi_version",
     "varlen_attn_bwd_workspace_size",
     "varlen_attn_bwd_v1",
+    "varlen_attn_bwd_noalloc",
 )
 
 _lock = threading.Lock()
@@ -83,6 +84,8 @@ def _bind(lib):
     lib.varlen_attn_bwd_v1.argtypes = ([P] * 8 + [i32, i64, i64, i32, i32, i32, i32, i32, i32, f32,
                                                   i32, P, P, P, P, ctypes.c_size_t, P])
     lib.varlen_attn_bwd_v1.restype = i32
+    lib.varlen_attn_bwd_noalloc.argtypes = lib.varlen_attn_bwd_v1.argtypes[:22] + [P]
+    lib.varlen_attn_bwd_noalloc.restype = i32
     return lib
 
 
@@ -326,3 +329,31 @@ def varlen_attn_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: tor
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return dq, dk, dv
+
+
+def varlen_attn_bwd_noalloc(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor,
+                            v: torch.Tensor, out: torch.Tensor, lse: torch.Tensor,
+                            cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor,
+                            max_seqlen_q: int, max_seqlen_k: int, dq: torch.Tensor,
+                            dk: torch.Tensor, dv: torch.Tensor, causal: bool = False,
+                            scale: Optional[float] = None,
+                            stream: Optional[torch.cuda.Stream] = None) -> int:
+    """varlen_attn_bwd_noalloc: the backward into the given dq/dk/dv with the
+    library's own fixed scratch (no workspace, nothing allocated).  Returns
+    the status code (raises nothing); see the header for its limits."""
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    total_q, H, D = q.shape
+    total_k, Hkv, _ = k.shape
+
+    def addr(t):
+        return t.data_ptr() if t is not None and t.numel() else 0
+
+    V = ctypes.c_void_p
+    with torch.cuda.device(q.device):
+        return load_library().varlen_attn_bwd_noalloc(
+            V(addr(dout)), V(addr(q)), V(addr(k)), V(addr(v)), V(addr(out)), V(addr(lse)),
+            V(addr(cu_seqlens_q)), V(addr(cu_seqlens_k)), cu_seqlens_q.numel() - 1, total_q,
+            total_k, int(max_seqlen_q), int(max_seqlen_k), H, Hkv, D, int(bool(causal)),
+            0.0 if scale is None else float(scale), DTYPE_CODES[q.dtype], V(addr(dq)),
+            V(addr(dk)), V(addr(dv)), V(stream.cuda_stream))

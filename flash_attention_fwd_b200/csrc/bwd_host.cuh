@@ -192,3 +192,50 @@ extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k
               : launch_bwd<128, false>(m_dq, m_kv, bp, grid_q, grid_k, run_dq, run_dkdv, s, dev,
                                        16);
 }
+
+// ---------------------------------------------------------------------------
+// varlen_attn_bwd_noalloc: the backward with its scratch (delta, float32
+// [total_q, H]) in a fixed file-scope device array instead of a caller
+// workspace.  NOALLOC_SCRATCH_BYTES bounds total_q * H * 4 (16 MiB: 4,194,304
+// (token, head) rows, e.g. 65,536 tokens x 64 heads).  The array's device
+// address is looked up once per device, on the first call, and cached.
+// Nothing in the scratch has to start at zero: every delta the dK/dV pass
+// reads is written by the dQ pass of the same call.  All calls on a device
+// share the array, so calls that overlap in time (other streams, other host
+// threads) race on it.
+namespace vattn {
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_bwd_scratch[NOALLOC_SCRATCH_BYTES];
+static void *g_bwd_scratch_addr[64];
+}  // namespace vattn
+
+extern "C" int varlen_attn_bwd_noalloc(const void *dout, const void *q, const void *k,
+                                       const void *v, const void *out, const float *lse,
+                                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                       int batch, int64_t total_q, int64_t total_k,
+                                       int max_seqlen_q, int max_seqlen_k, int num_heads,
+                                       int num_kv_heads, int head_dim, int causal, float scale,
+                                       varlen_dtype_t dtype, void *dq, void *dk, void *dv,
+                                       varlen_stream_t stream) {
+  using namespace vattn;
+  int rc = bwd_check_args(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q,
+                          total_k, max_seqlen_q, max_seqlen_k, num_heads, num_kv_heads, head_dim,
+                          dtype, dq, dk, dv);
+  if (rc != VARLEN_OK) return rc;
+  if (varlen_attn_bwd_workspace_size(total_q, num_heads) > NOALLOC_SCRATCH_BYTES)
+    return VARLEN_ERR_WORKSPACE;
+  if (batch == 0 || (total_q == 0 && total_k == 0)) return VARLEN_OK;
+  int dev_id = 0;
+  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= 64)
+    return VARLEN_ERR_LAUNCH;
+  if (!g_bwd_scratch_addr[dev_id]) {
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_bwd_scratch) != cudaSuccess || !addr)
+      return VARLEN_ERR_LAUNCH;
+    g_bwd_scratch_addr[dev_id] = addr;
+  }
+  return varlen_attn_bwd_v1(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q,
+                            total_k, max_seqlen_q, max_seqlen_k, num_heads, num_kv_heads,
+                            head_dim, causal, scale, dtype, dq, dk, dv,
+                            g_bwd_scratch_addr[dev_id], NOALLOC_SCRATCH_BYTES, stream);
+}

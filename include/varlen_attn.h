@@ -269,6 +269,30 @@ int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k, const voi
                        void *dq, void *dk, void *dv,
                        void *workspace, size_t workspace_bytes, varlen_stream_t stream);
 
+/*
+ * varlen_attn_bwd_noalloc — varlen_attn_bwd_v1 without a workspace argument
+ * and without any allocation: the scratch (delta, float32 [total_q, H]) lives
+ * in a fixed 16 MiB device array of the library (so total_q * H <= 4,194,304;
+ * larger problems return VARLEN_ERR_WORKSPACE before anything is launched).
+ * The pages have no counterpart: their backward allocates its buffers.
+ *
+ * The array's device address is looked up once per device on the first call
+ * (cudaGetSymbolAddress), so the first call on each device must not be made
+ * while the stream is being captured into a CUDA graph; later calls can be
+ * captured.  Nothing in the scratch has to start at zero.  Every call on a
+ * device uses the same array: calls that overlap in time (other streams or
+ * host threads) race on it and give wrong gradients; serialise them.
+ * Arguments, results and errors are otherwise those of varlen_attn_bwd_v1.
+ */
+int varlen_attn_bwd_noalloc(const void *dout, const void *q, const void *k, const void *v,
+                            const void *out, const float *lse,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            int batch, int64_t total_q, int64_t total_k,
+                            int max_seqlen_q, int max_seqlen_k,
+                            int num_heads, int num_kv_heads, int head_dim,
+                            int causal, float scale, varlen_dtype_t dtype,
+                            void *dq, void *dk, void *dv, varlen_stream_t stream);
+
 /* Library ABI version: 4 for this header (v2, v3 and the backward added; v1 unchanged). */
 int varlen_attn_abi_version(void);
 

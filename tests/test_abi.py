@@ -155,3 +155,24 @@ def test_backward_workspace_size_and_empty_call():
     args = dict(BWD)
     args.update(batch=0)
     assert fa.varlen_attn_bwd_raw(**args) == 0
+
+
+def test_noalloc_backward_rejects_before_any_device_call():
+    lib = fa.load_library()
+    V = ctypes.c_void_p
+    args = dict(BWD)
+    # 2^20 query rows x 8 heads x 4 bytes of scratch = 32 MiB > the fixed 16 MiB
+    rc = lib.varlen_attn_bwd_noalloc(*(V(args[n]) for n in (
+        "dout_ptr", "q_ptr", "k_ptr", "v_ptr", "out_ptr", "lse_ptr", "cu_q_ptr", "cu_k_ptr")),
+        2, 1 << 20, 10, 5, 5, 8, 2, 128, 1, 0.0, 0, V(0x61000), V(0x62000), V(0x63000), V(0))
+    assert rc == -8
+    # invalid arguments are reported as by varlen_attn_bwd_v1
+    rc = lib.varlen_attn_bwd_noalloc(*(V(args[n]) for n in (
+        "dout_ptr", "q_ptr", "k_ptr", "v_ptr", "out_ptr", "lse_ptr", "cu_q_ptr", "cu_k_ptr")),
+        2, 10, 10, 5, 5, 8, 2, 96, 1, 0.0, 0, V(0x61000), V(0x62000), V(0x63000), V(0))
+    assert rc == -2
+    # an empty batch is a no-op that touches nothing
+    rc = lib.varlen_attn_bwd_noalloc(*(V(args[n]) for n in (
+        "dout_ptr", "q_ptr", "k_ptr", "v_ptr", "out_ptr", "lse_ptr", "cu_q_ptr", "cu_k_ptr")),
+        0, 10, 10, 5, 5, 8, 2, 128, 1, 0.0, 0, V(0x61000), V(0x62000), V(0x63000), V(0))
+    assert rc == 0
