@@ -34,6 +34,8 @@ if ROOT not in sys.path:
 import workloads  # noqa: E402
 
 METRIC = "varlen attn fwd TFLOP/s (unmasked FLOPs) and % of B200 dense bf16 peak"
+METRIC_BWD = ("varlen attn bwd TFLOP/s (10*D per unmasked pair: the backward's five products) "
+              "and % of B200 dense bf16 peak")
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_DIR = "flash_attention_fwd_b200/csrc"
@@ -258,6 +260,9 @@ def run_gpu(args, rank: int, world: int):
     import torch
     import flash_attention_fwd_b200 as fa
 
+    if args.pass_ == "bwd":
+        return run_gpu_bwd(args, rank, world)
+
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -383,7 +388,8 @@ def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist, extra=())
     return e2e_ms, h2d, d2h
 
 
-def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk):
+def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk,
+         metric=METRIC, cpu_fn=None, launches_per_step=1, traffic_key=None):
     if rank == 0:
         ms = total_ms / args.steps
         value = whole_job_tflops(world, flops, ms)
@@ -393,14 +399,16 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
         avg_launch_ms = sum(per_launch) / len(per_launch)
         achieved = flops / (avg_launch_ms * 1e-3) / 1e12
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and cpu_fn is not None:
+            cpu = cpu_fn()
+        elif world == 1 and not args.no_cpu_baseline:
             tfs, nrows, fl, dt, thr = time_oracle(case, args.cpu_seconds)
             cpu = {"value": tfs, "unit": UNIT, "cores": thr, "kind": "oracle",
                    "sample": "%d seeded random (token, head) rows of the %s workload, "
                              "%.2f GFLOP of its %.2f TFLOP step, %.1f s on %d threads"
                              % (nrows, args.workload, fl / 1e9, flops / 1e12, dt, thr)}
         line = {
-            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "metric": metric, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": case.dtype, "data": "synthetic (seeded N(0,1) Q/K/V, seeded lengths)",
@@ -419,7 +427,7 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
             "pct_of_peak": round(100.0 * achieved / peak, 2),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                         "traffic": traffic_for(args.workload),
+                         "traffic": traffic_for(traffic_key or args.workload),
                          "peak_source": "%s burst bf16 (sustained %.1f -> frac %.4f)"
                                         % (peak_src, peak_sus, achieved / peak_sus)},
             "launch_ms": {"min": round(min(per_launch), 4),
@@ -428,7 +436,7 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
             "e2e": {"value": round(whole_job_tflops(world, flops, e2e_ms), 3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 3)},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * launches_per_step,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -437,7 +445,191 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- backward
+
+def bwd_flops(case) -> int:
+    """10 * D per unmasked (query, key, head) pair: S = QK^T and dP = dO V^T
+    (recomputed), dV += P^T dO, dK += dS^T Q, dQ += dS K, 2 * D each."""
+    return 10 * case.D * unmasked_pairs(case.lens_q, case.lens_k, case.H, case.causal)
+
+
+def prefix_case(case, m: int):
+    """The workload's first m sequences (a packed prefix) as a case of its own."""
+    cq, ck = case.cu_q.tolist(), case.cu_k.tolist()
+    return workloads.Case(case.q[:cq[m]], case.k[:ck[m]], case.v[:ck[m]], case.cu_q[:m + 1].clone(),
+                          case.cu_k[:m + 1].clone(), case.lens_q[:m], case.lens_k[:m], case.H,
+                          case.Hkv, case.D, case.causal, case.dtype, case.scale,
+                          name=case.name + "[:%d]" % m, seed=case.seed)
+
+
+def time_oracle_bwd(case, seconds: float, nthreads: int | None = None):
+    """Times the fp64 oracle backward (as it stands) on the workload's first
+    sequences, as many as fit in about ``seconds`` of CPU work (O and LSE from
+    the oracle forward of the same sample, not timed).  Returns the
+    cpu_baseline object."""
+    import torch
+    import oracle
+    nthreads = nthreads or oracle.default_threads()
+
+    def run(m):
+        sub = prefix_case(case, m)
+        g = torch.Generator("cpu").manual_seed(97)
+        dout = torch.randn(sub.q.shape, generator=g).to(sub.q.dtype)
+        o, lse = oracle.run_case(sub, nthreads=nthreads)
+        t0 = time.perf_counter()
+        oracle.run_case_bwd(sub, dout, o, lse, nthreads=nthreads)
+        return time.perf_counter() - t0, bwd_flops(sub)
+
+    dt, fl = run(1)
+    m = 1
+    rate = fl / max(dt, 1e-6)
+    while m < case.B and bwd_flops(prefix_case(case, m + 1)) / rate < seconds:
+        m += 1
+    if m > 1:
+        dt, fl = run(m)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": "backward of the workload's first %d sequences (%.2f GFLOP of its %.2f "
+                      "TFLOP step), %.1f s on %d threads"
+                      % (m, fl / 1e9, bwd_flops(case) / 1e12, dt, nthreads)}
+
+
+def run_gpu_bwd(args, rank: int, world: int):
+    """One step = one varlen_attn_bwd call (its two kernels) over the workload,
+    with dO seeded and O / LSE from one forward call before the timing."""
+    import torch
+    import flash_attention_fwd_b200 as fa
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    case = workloads.make_workload(args.workload)
+    if case.mask or workloads.WORKLOADS[args.workload].page_size:
+        raise SystemExit("the backward covers the plain forward (no window, paged K/V or sinks)")
+    flops = bwd_flops(case)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    cq, ck = case.cu_q.to(dev), case.cu_k.to(dev)
+    fa.load_library()
+    fa.device_status(clear=True)
+    out, lse = fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, case.causal,
+                                  case.scale)
+    g = torch.Generator("cpu").manual_seed(case.seed + 7)
+    dout = torch.randn(case.q.shape, generator=g).to(case.q.dtype).to(dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(fa.bwd_workspace_size(case.Tq, case.H), 1), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.varlen_attn_bwd(dout, q, k, v, out, lse, cq, ck, case.max_q, case.max_k, case.causal,
+                           case.scale, dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_bus_id(local))
+    clocks.start()
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    ev[0].record(stream)
+    for i in range(args.steps):
+        step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    per_launch = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    status = fa.device_status(clear=True)
+    if status != 0:
+        raise RuntimeError("device status word set: %d" % status)
+
+    e2e_ms, h2d, d2h = float("nan"), 0, 0
+    if not args.no_e2e:
+        host_in = [t.cpu().pin_memory() for t in (dout, q, k, v, out, lse, cq, ck)]
+        dev_in = [dout, q, k, v, out, lse, cq, ck]
+        host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+        def e2e_step():
+            for d_, h_ in zip(dev_in, host_in):
+                d_.copy_(h_, non_blocking=True)
+            step()
+            for h_, d_ in zip(host_out, (dq, dk, dv)):
+                h_.copy_(d_, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        n = max(1, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n
+    if dist:
+        total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
+        dist.barrier()
+    emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk,
+         metric=METRIC_BWD, cpu_fn=lambda: time_oracle_bwd(case, args.cpu_seconds),
+         launches_per_step=2, traffic_key=args.workload + ":bwd")
+    if dist:
+        dist.destroy_process_group()
+
+
 # ----------------------------------------------------------------------------- reference arm
+
+def run_reference_bwd(args, world, case, nthreads, budget):
+    """Reference arm of the backward: the oracle backward on the workload's
+    first sequences (as many as fit the per-step budget), every step."""
+    import torch
+    import oracle
+    m = 1
+    calib = time_oracle_bwd(prefix_case(case, 1), 0.0, nthreads)
+    rate = calib["value"] * 1e12
+    while m < case.B and bwd_flops(prefix_case(case, m + 1)) / rate < budget:
+        m += 1
+    sub = prefix_case(case, m)
+    g = torch.Generator("cpu").manual_seed(97)
+    dout = torch.randn(sub.q.shape, generator=g).to(sub.q.dtype)
+    o, lse = oracle.run_case(sub, nthreads=nthreads)
+    for _ in range(args.warmup):
+        oracle.run_case_bwd(sub, dout, o, lse, nthreads=nthreads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.run_case_bwd(sub, dout, o, lse, nthreads=nthreads)
+    dt = (time.perf_counter() - t0) / args.steps
+    fl = bwd_flops(sub)
+    value = fl / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC_BWD, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) Q/K/V/dO, seeded lengths)",
+        "config": {"workload": workloads.WORKLOADS[args.workload].description,
+                   "name": args.workload, "pass": "bwd", "sample_sequences": m,
+                   "sample_flops": fl},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": "backward of the first %d sequences per step, %.2f GFLOP"
+                                   % (m, fl / 1e9)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
 
 def run_reference(args, rank: int, world: int):
     """The fp64 CPU oracle as it stands, on the host cores, one bounded row
@@ -448,6 +640,8 @@ def run_reference(args, rank: int, world: int):
     case = workloads.make_workload(args.workload)
     nthreads = oracle.default_threads()
     budget = max(0.5, min(30.0, args.reference_seconds / max(1, args.steps + args.warmup)))
+    if args.pass_ == "bwd":
+        return run_reference_bwd(args, world, case, nthreads, budget)
     rows0, fl0 = oracle_sample_rows(case, 256, seed=98)
     t0 = time.perf_counter()
     oracle.run_case_rows(case, rows0, nthreads=nthreads, **case.mask)
@@ -484,6 +678,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="long", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--pass", dest="pass_", default="fwd", choices=["fwd", "bwd"],
+                    help="time the forward (default) or the backward (dQ, dK, dV)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -5,20 +5,27 @@
  *
  *   S^T  = K Q^T,  dP^T = V dO^T          tcgen05 (keys on the TMEM lanes)
  *   P^T  = exp2(S^T scale log2e - LSE log2e),  dS^T = P^T (dP^T - delta)
- *                                          one thread per key row, written as
- *                                          bf16/fp16 MMA operands in shared memory
- *   dV  += P^T dO,  dK += dS^T Q           tcgen05, accumulated in TMEM
+ *                                          one thread per key row, written back
+ *                                          as bf16/fp16 over the first columns
+ *                                          of S^T and dP^T in TMEM
+ *   dV  += P^T dO,  dK += dS^T Q           tcgen05, A operand from TMEM,
+ *                                          accumulated in TMEM
  *
  * and at the end dV -> dv, dK * scale -> dk.  This is the key side of the
  * page's backward loop (see bwd_common.cuh); dK and dV of a key/value head sum
  * over its query heads inside one item, so no accumulation crosses CTAs.
  * delta comes from the dQ pass (workspace), LSE from the forward.
  *
- * One persistent CTA per SM, 192 threads: warps 0-3 one key row per thread,
- * warp 4 scheduler + TMA producer, warp 5 TMEM owner + MMA issuer.  TMEM:
+ * One persistent CTA per SM, 320 threads: two warpgroups of row threads
+ * (warps 0-3 and 4-7, one key row per thread each) that take the steps in
+ * turn — even global steps to the first, odd to the second, matching the
+ * double-buffered S^T / dP^T in TMEM and P^T / dS^T in shared memory — so one
+ * computes while the tensor cores serve the other; warp 8 scheduler + TMA
+ * producer, warp 9 TMEM owner + MMA issuer.  TMEM:
  * dV (D) | dK (D) | S^T[2] (BQ) | dP^T[2] (BQ).  Shared memory: K and V
- * tiles of the item, NST stages of (Q, dO) query tiles, and two buffers each
- * of P^T and dS^T.
+ * tiles of the item and NST stages of (Q, dO) query tiles; a stage is held
+ * from its load until the step's dV / dK products complete, so the depth is
+ * what hides the load latency.
  */
 #pragma once
 #include "bwd_common.cuh"
@@ -26,13 +33,13 @@
 namespace vattn {
 namespace bwd_dkdv {
 
-constexpr int NUM_THREADS = 192;
-constexpr int PRODUCER_WARP = 4;
-constexpr int MMA_WARP = 5;
-constexpr int RING_CONSUMERS = 1 + 4;
+constexpr int NUM_THREADS = 320;
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int RING_CONSUMERS = 1 + 8;
 constexpr int BK = 128;  // keys per item (TMEM lanes)
 constexpr int BQ = 64;   // queries per step
-constexpr int NST = 3;   // (Q, dO) stages
+constexpr int NST = 5;   // (Q, dO) stages
 
 struct KeyItem {
   int b;       // sequence; < 0 ends the list
@@ -52,18 +59,20 @@ struct KeyRing {
   uint64_t empty[ITEM_RING];
 };
 
-// Items are (key tile kt, sequence b, key/value head), listed by kt, then b,
-// then head, and dealt to CTA i mod G with the direction reversed every round.
-// With the causal rule the first key tiles see the most queries, so the list
-// runs roughly from the largest item to the smallest.  The walk is
-// warp-cooperative over 32 sequences at a time, like the forward scheduler.
+// Items are (sequence b, key tile kt, key/value head); an item's cost is its
+// number of query tiles per query head, nqt = ceil(Lq / BQ) - R kt with the
+// causal rule (R = BK / BQ: key tile kt is first seen by query tile R kt) and
+// ceil(Lq / BQ) without it.  Items are listed by cost level, highest first
+// ("longest processing time first", as in the forward scheduler), then by
+// sequence and head, and dealt to CTA i mod G with the direction reversed
+// every round.  The walk is warp-cooperative over 32 sequences at a time.
 struct KeyScheduler {
+  static constexpr int R = BK / BQ;
   const int *cu_q, *cu_k;
   int B, Hkv, group, causal, total_q, total_k;
   int cta, grid, lane;
   long long round;
-  int level;  // current key tile index; max_kt + 1 once exhausted
-  int max_kt;
+  int level;  // current cost level; -1 once the list is exhausted
   long long level_base, level_items;
   int cur_b;
   long long cur_units;
@@ -80,7 +89,20 @@ struct KeyScheduler {
     lq = qe - qs;
     lk = ke - ks;
   }
-  __device__ long long count_level(int kt) const {
+  // key tiles of a sequence (nq query tiles, nk key tiles) at cost level c
+  __device__ int units_at(int nq, int nk, int c) const {
+    if (!causal) return (c == nq) ? nk : 0;
+    if (c == 0) return max(0, nk - (nq + R - 1) / R);
+    const int d = nq - c;
+    return (d >= 0 && d % R == 0 && d / R < nk) ? 1 : 0;
+  }
+  // key tile of the k-th unit of a sequence at cost level c
+  __device__ int tile_of(int nq, int c, int k) const {
+    if (!causal) return k;
+    if (c == 0) return (nq + R - 1) / R + k;
+    return (nq - c) / R;
+  }
+  __device__ long long count_level(int c) const {
     long long u = 0;
     for (int b0 = 0; b0 < B; b0 += 32) {
       const int b = b0 + lane;
@@ -88,7 +110,7 @@ struct KeyScheduler {
       if (b < B) {
         int qs, lq, ks, lk;
         extents(b, qs, lq, ks, lk);
-        v = (lk + BK - 1) / BK > kt ? 1 : 0;
+        v = units_at((lq + BQ - 1) / BQ, (lk + BK - 1) / BK, c);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -109,37 +131,37 @@ struct KeyScheduler {
     grid = gridDim.x;
     lane = threadIdx.x & 31;
     round = 0;
+    // the top level: the largest query-tile count of a sequence with keys
     int top = -1;
     for (int b0 = 0; b0 < B; b0 += 32) {
       const int b = b0 + lane;
       if (b < B) {
         int qs, lq, ks, lk;
         extents(b, qs, lq, ks, lk);
-        top = max(top, (lk + BK - 1) / BK - 1);
+        if (lk > 0) top = max(top, (lq + BQ - 1) / BQ);
       }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) top = max(top, __shfl_xor_sync(0xffffffffu, top, o));
-    max_kt = top;
-    level = 0;
+    level = top;
     level_base = 0;
-    level_items = (max_kt >= 0) ? count_level(0) : 0;
+    level_items = (level >= 0) ? count_level(level) : 0;
     cur_b = 0;
     cur_units = 0;
   }
   __device__ bool next(KeyItem &w) {
     const long long idx = round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
     ++round;
-    while (level <= max_kt && idx >= level_base + level_items) {
+    while (level >= 0 && idx >= level_base + level_items) {
       level_base += level_items;
-      ++level;
-      if (level <= max_kt) {
+      --level;
+      if (level >= 0) {
         level_items = count_level(level);
         cur_b = 0;
         cur_units = 0;
       }
     }
-    if (level > max_kt) return false;
+    if (level < 0) return false;
     const long long local = idx - level_base;
     const long long unit = local / Hkv;
     w.kvh = (int)(local % Hkv);
@@ -148,7 +170,7 @@ struct KeyScheduler {
       int qs = 0, lq = 0, ks = 0, lk = 0, u = 0;
       if (b < B) {
         extents(b, qs, lq, ks, lk);
-        u = (lk + BK - 1) / BK > level ? 1 : 0;
+        u = units_at((lq + BQ - 1) / BQ, (lk + BK - 1) / BK, level);
       }
       int incl = u;
 #pragma unroll
@@ -167,15 +189,17 @@ struct KeyScheduler {
         lk = __shfl_sync(0xffffffffu, lk, src);
         cur_b += src;
         cur_units += before;
+        const int nq = (lq + BQ - 1) / BQ;
+        const int kt = tile_of(nq, level, (int)(unit - cur_units));
         w.b = cur_b;
-        w.kt = level;
-        w.k0 = ks + level * BK;
+        w.kt = kt;
+        w.k0 = ks + kt * BK;
         w.Lk = lk;
         w.Lq = lq;
         w.q0 = qs;
         // causal (sequence-local, top-left): key kk is seen by the queries qi >= kk
-        w.qt0 = causal ? (level * BK) / BQ : 0;
-        w.nqt = max(0, (lq + BQ - 1) / BQ - w.qt0);
+        w.qt0 = causal ? R * kt : 0;
+        w.nqt = max(0, nq - w.qt0);
         w.nsteps = group * w.nqt;
         return true;
       }
@@ -189,31 +213,19 @@ struct Barriers {
   uint64_t kv_full, kv_empty;
   uint64_t st_full[NST], st_empty[NST];
   uint64_t s_full[2];    // S^T and dP^T of a step in TMEM buffer
-  uint64_t pd_full[2];   // P^T and dS^T written (one arrival per row warp)
-  uint64_t pd_free[2];   // the MMAs that read them completed
+  uint64_t pd_full[2];   // P^T and dS^T written to TMEM (one arrival per row warp)
   uint64_t acc_ready, acc_free;
-  uint64_t lsd_full[2];  // a step's LSE / delta values written (one arrival per row warp)
+  uint64_t lsd_full[2];  // [warpgroup]: a step's LSE / delta values written (one arrival per warp)
   uint64_t drain;
   KeyRing ring;
-  alignas(16) float lsd[2][2][BQ];  // per step parity: LSE * log2e and delta of the step's queries
+  alignas(16) float lsd[2][2][BQ];  // [warpgroup]: LSE * log2e and delta of the step's queries
   uint32_t tmem_base;
   int abort_flag;
 };
 
 template <int D>
 constexpr size_t smem_bytes() {
-  return (size_t)2 * BK * D * 2 + (size_t)NST * 2 * BQ * D * 2 + (size_t)4 * BK * BQ * 2 +
-         sizeof(Barriers) + 1024;
-}
-
-// Writes one 64-value row (8 x 16 bytes) of a K-major operand tile with the
-// 128-byte swizzle: row r, 16-byte chunk c at chunk position c ^ (r & 7).
-__device__ __forceinline__ void store_sw128_row(uint8_t *tile, int r, const uint32_t (&v)[32]) {
-  uint8_t *row = tile + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-    *reinterpret_cast<uint4 *>(row + ((c ^ (r & 7)) << 4)) =
-        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  return (size_t)2 * BK * D * 2 + (size_t)NST * 2 * BQ * D * 2 + sizeof(Barriers) + 1024;
 }
 
 template <int D, bool BF16>
@@ -224,7 +236,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int DB = D / 64;
   constexpr uint32_t KV_BYTES = BK * D * 2;
   constexpr uint32_t QS_BYTES = BQ * D * 2;
-  constexpr uint32_t PT_BYTES = BK * BQ * 2;
   constexpr uint32_t DV_COL = 0, DK_COL = D;
   constexpr uint32_t ST_COL = 2 * D, DPT_COL = 2 * D + 2 * BQ;
   static_assert(DPT_COL + 2 * BQ <= TMEM_COLS, "TMEM budget");
@@ -237,10 +248,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sK = smem;
   uint8_t *sV = sK + KV_BYTES;
-  uint8_t *sQs = sV + KV_BYTES;               // stage s: Q at sQs + s * 2 * QS_BYTES, dO after it
-  uint8_t *sPT = sQs + NST * 2 * QS_BYTES;    // P^T[2]
-  uint8_t *sDST = sPT + 2 * PT_BYTES;         // dS^T[2]
-  Barriers *bars = reinterpret_cast<Barriers *>(sDST + 2 * PT_BYTES);
+  uint8_t *sQs = sV + KV_BYTES;  // stage s: Q at sQs + s * 2 * QS_BYTES, dO after it
+  Barriers *bars = reinterpret_cast<Barriers *>(sQs + NST * 2 * QS_BYTES);
   volatile int *abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x / 32;
@@ -256,10 +265,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars->s_full[i], 1);
       ptx::mbar_init(&bars->pd_full[i], 4);
-      ptx::mbar_init(&bars->pd_free[i], 1);
     }
     ptx::mbar_init(&bars->acc_ready, 1);
-    ptx::mbar_init(&bars->acc_free, 4);
+    ptx::mbar_init(&bars->acc_free, 8);
     ptx::mbar_init(&bars->lsd_full[0], 4);
     ptx::mbar_init(&bars->lsd_full[1], 4);
     ptx::mbar_init(&bars->drain, 1);
@@ -352,8 +360,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t sK_addr = ptx::smem_u32(sK);
       const uint32_t sV_addr = ptx::smem_u32(sV);
       const uint32_t sQs_addr = ptx::smem_u32(sQs);
-      const uint32_t sPT_addr = ptx::smem_u32(sPT);
-      const uint32_t sDST_addr = ptx::smem_u32(sDST);
       // S^T and dP^T of global step gs into TMEM buffer gs & 1
       auto issue_st = [&](uint32_t gs) -> bool {
         const uint32_t st = gs % NST;
@@ -375,20 +381,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::mma_commit(&bars->s_full[buf]);
         return true;
       };
-      // dV += P^T dO, dK += dS^T Q for global step gs (operands in shared memory)
+      // dV += P^T dO, dK += dS^T Q for global step gs: P^T / dS^T from TMEM
+      // (bf16/fp16 pairs over the first BQ / 2 columns of S^T / dP^T), dO and
+      // Q MN-major from the stage, in steps of 16 queries
       auto issue_acc = [&](uint32_t gs, bool acc) {
         const uint32_t st = gs % NST;
         const uint32_t qa = sQs_addr + st * 2 * QS_BYTES;
         const uint32_t buf = gs & 1u;
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
-          uint64_t apt = ptx::sdesc_sw128(sPT_addr + buf * PT_BYTES + kk * 32u, 16, 1024);
-          uint64_t adst = ptx::sdesc_sw128(sDST_addr + buf * PT_BYTES + kk * 32u, 16, 1024);
           uint64_t bdo = ptx::sdesc_sw128(qa + QS_BYTES + kk * (16 * 128), BQ * 128, 1024);
           uint64_t bq = ptx::sdesc_sw128(qa + kk * (16 * 128), BQ * 128, 1024);
           const uint32_t a = (acc || kk > 0) ? 1u : 0u;
-          ptx::mma_ss(tmem + DV_COL, apt, bdo, IDESC_ACC, a);
-          ptx::mma_ss(tmem + DK_COL, adst, bq, IDESC_ACC, a);
+          ptx::mma_ts(tmem + DV_COL, tmem + ST_COL + buf * BQ + kk * 8, bdo, IDESC_ACC, a);
+          ptx::mma_ts(tmem + DK_COL, tmem + DPT_COL + buf * BQ + kk * 8, bq, IDESC_ACC, a);
         }
       };
       while (ok) {
@@ -416,7 +422,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tc_fence_after();
           }
           issue_acc(gs, s > 0);
-          ptx::mma_commit(&bars->pd_free[buf]);
           ptx::mma_commit(&bars->st_empty[gs % NST]);
           if (s == n - 1) {
             ptx::mma_commit(&bars->acc_ready);
@@ -432,15 +437,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ key rows
-    const int r = threadIdx.x;  // key row in the tile == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t tST0 = tmem + lane_base + ST_COL;
-    const uint32_t tDPT0 = tmem + lane_base + DPT_COL;
+    const int t = warp / 4;             // warpgroup: takes the global steps gs with gs & 1 == t
+    const int r = threadIdx.x - 128 * t;  // key row in the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tST = tmem + lane_base + ST_COL + t * BQ;
+    const uint32_t tDPT = tmem + lane_base + DPT_COL + t * BQ;
     const float sl2 = p.scale_log2;
     uint32_t rs = 0, rph = 0, g = 0, items = 0;
     bool ok = true;
-    // LSE (log2 units) or delta of query c of step s: thread t < BQ loads LSE
-    // of query t, thread BQ + t delta of query t
+    // LSE (log2 units) or delta of query c of step s: thread r < BQ loads LSE
+    // of query r, thread BQ + c delta of query c
     auto load_lsd = [&](const KeyItem &w, int s) -> float {
       const int c = r & (BQ - 1);
       const int h = w.kvh * p.group + s / w.nqt;
@@ -465,65 +471,70 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int kk = w.kt * BK + r;  // sequence-local key
       const bool key_valid = kk < w.Lk;
       const size_t drow = ((size_t)(w.k0 + r) * p.Hkv + w.kvh) * D;
+      // warpgroup 0 writes dV, warpgroup 1 dK
+      uint16_t *out_row = (t == 0 ? bp.dv : bp.dk) + drow;
       if (n == 0) {
-        if (key_valid) {
-          zero_row<D>(bp.dk + drow);
-          zero_row<D>(bp.dv + drow);
-        }
+        if (key_valid) zero_row<D>(out_row);
         continue;
       }
-      float pre = load_lsd(w, 0);
-      for (int s = 0; ok && s < n; ++s) {
+      const int s0 = (int)((t - g) & 1u);  // this warpgroup's first step of the item
+      float pre = s0 < n ? load_lsd(w, s0) : 0.f;
+      for (int s = s0; ok && s < n; s += 2) {
         const uint32_t gs = g + s;
-        const uint32_t buf = gs & 1u;
-        // Exchange of the step's LSE / delta values among the row warps.  The
-        // buffer of parity buf is written again two steps later, only after
-        // every warp has arrived for the step in between, i.e. finished this one.
-        bars->lsd[buf][r / BQ][r & (BQ - 1)] = pre;
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->lsd_full[buf]);
-        if (s + 1 < n) pre = load_lsd(w, s + 1);
-        bool got = wait_bar(&bars->lsd_full[buf], (gs >> 1) & 1u, abort_flag) &&
-                   wait_bar(&bars->s_full[buf], (gs >> 1) & 1u, abort_flag);
+        bool got = wait_bar(&bars->s_full[t], (gs >> 1) & 1u, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        uint32_t sv[BQ], dpv[BQ];
-        tmem_ld_wait<BQ>(tST0 + buf * BQ, sv);
-        tmem_ld_wait<BQ>(tDPT0 + buf * BQ, dpv);
-        // queries of this step that see key kk: qi < Lq (lse = +inf otherwise)
-        // and, with the causal rule, qi >= kk
-        const int qbase = (w.qt0 + s % w.nqt) * BQ;
-        const int cmin = p.causal ? kk - qbase : 0;  // first visible column
-        const float *lse2 = bars->lsd[buf][0];
-        const float *dl = bars->lsd[buf][1];
-        uint32_t ppk[BQ / 2], dpk[BQ / 2];
-#pragma unroll
-        for (int c = 0; c < BQ; c += 2) {
-          float pr[2], ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float x = __uint_as_float(sv[c + e]) * sl2 - lse2[c + e];
-            pr[e] = (key_valid && c + e >= cmin) ? ptx::ex2_approx(x) : 0.f;
-            ds[e] = pr[e] * (__uint_as_float(dpv[c + e]) - dl[c + e]);
-          }
-          ppk[c / 2] = pack2<BF16>(pr[0], pr[1]);
-          dpk[c / 2] = pack2<BF16>(ds[0], ds[1]);
-        }
-        // P^T / dS^T buffer free once the MMAs of step gs - 2 completed
-        got = wait_bar(&bars->pd_free[buf], ((gs >> 1) & 1u) ^ 1u, abort_flag);
+        // Exchange of the step's LSE / delta values among the warpgroup's
+        // warps.  S^T(gs) arriving means the MMA warp saw all four warps'
+        // P^T / dS^T of this warpgroup's previous step, so every warp has
+        // finished reading the previous values and the buffer can be reused.
+        // (S^T(gs) also overwrote the previous step's P^T in TMEM only after
+        // the dV / dK products that read it: the tensor core runs in order.)
+        bars->lsd[t][r / BQ][r & (BQ - 1)] = pre;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->lsd_full[t]);
+        if (s + 2 < n) pre = load_lsd(w, s + 2);
+        got = wait_bar(&bars->lsd_full[t], (gs >> 1) & 1u, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
-        store_sw128_row(sPT + buf * PT_BYTES, r, ppk);
-        store_sw128_row(sDST + buf * PT_BYTES, r, dpk);
-        ptx::fence_proxy_async_smem();
+        // queries of this step that see key kk: qi < Lq (lse = +inf otherwise)
+        // and, with the causal rule, qi >= kk
+        const int qbase = (w.qt0 + s % w.nqt) * BQ;
+        const int cmin = p.causal ? kk - qbase : 0;  // first visible column
+        const float *lse2 = bars->lsd[t][0];
+        const float *dl = bars->lsd[t][1];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t sv[32], dpv[32];
+          tmem_ld_wait<32>(tST + half * 32, sv);
+          tmem_ld_wait<32>(tDPT + half * 32, dpv);
+          uint32_t ppk[16], dpk[16];
+#pragma unroll
+          for (int c2 = 0; c2 < 32; c2 += 2) {
+            float pr[2], ds[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = half * 32 + c2 + e;
+              const float x = __uint_as_float(sv[c2 + e]) * sl2 - lse2[c];
+              pr[e] = (key_valid && c >= cmin) ? ptx::ex2_approx(x) : 0.f;
+              ds[e] = pr[e] * (__uint_as_float(dpv[c2 + e]) - dl[c]);
+            }
+            ppk[c2 / 2] = pack2<BF16>(pr[0], pr[1]);
+            dpk[c2 / 2] = pack2<BF16>(ds[0], ds[1]);
+          }
+          // columns [16 half, 16 half + 16): S^T / dP^T columns already read
+          tmem_st<16>(tST + half * 16, ppk);
+          tmem_st<16>(tDPT + half * 16, dpk);
+        }
+        ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->pd_full[buf]);
+        if (lane == 0) ptx::mbar_arrive(&bars->pd_full[t]);
       }
       if (!ok) break;
       g += n;
@@ -531,8 +542,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ++items;
       if (!__all_sync(0xffffffffu, got)) break;
       ptx::tc_fence_after();
-      store_tmem_row<D, BF16>(tmem + lane_base + DV_COL, 1.f, key_valid, bp.dv + drow);
-      store_tmem_row<D, BF16>(tmem + lane_base + DK_COL, bp.scale, key_valid, bp.dk + drow);
+      store_tmem_row<D, BF16>(tmem + lane_base + (t == 0 ? DV_COL : DK_COL),
+                              t == 0 ? 1.f : bp.scale, key_valid, out_row);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->acc_free);

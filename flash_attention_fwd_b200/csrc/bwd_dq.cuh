@@ -13,8 +13,12 @@
  * dK/dV pass.  This is the query side of the page's backward loop (see
  * bwd_common.cuh); the work items and their order are the forward's.
  *
- * One persistent CTA per SM, 192 threads: warps 0-3 one query row per thread,
- * warp 4 scheduler + TMA producer, warp 5 TMEM owner + MMA issuer.  TMEM:
+ * One persistent CTA per SM, 320 threads: two warpgroups of row threads
+ * (warps 0-3 and 4-7, one query row per thread each) that take the key tiles
+ * in turn — even global tiles to the first, odd to the second, matching the
+ * double-buffered S / dP in TMEM — so one computes while the tensor cores
+ * serve the other; warp 8 scheduler + TMA producer, warp 9 TMEM owner + MMA
+ * issuer.  TMEM:
  * S[2] | dP[2] (BN columns each, double-buffered across key tiles) | dQ (D).
  * The K/V ring holds K(j) and V(j) in turn; V(j) is released after dP(j), K(j)
  * after dQ(j).
@@ -25,12 +29,12 @@
 namespace vattn {
 namespace bwd_dq {
 
-constexpr int NUM_THREADS = 192;
-constexpr int PRODUCER_WARP = 4;
-constexpr int MMA_WARP = 5;
-constexpr int RING_CONSUMERS = 1 + 4;
+constexpr int NUM_THREADS = 320;
+constexpr int PRODUCER_WARP = 8;
+constexpr int MMA_WARP = 9;
+constexpr int RING_CONSUMERS = 1 + 8;
 constexpr int BN = 64;
-constexpr int NSLOT = 8;
+constexpr int NSLOT = 10;
 
 struct Barriers {
   uint64_t full[NSLOT];
@@ -89,7 +93,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&bars->ds_full[i], 4);
     }
     ptx::mbar_init(&bars->dq_ready, 1);
-    ptx::mbar_init(&bars->dq_free, 4);
+    ptx::mbar_init(&bars->dq_free, 8);
     ptx::mbar_init(&bars->drain, 1);
     for (int i = 0; i < ITEM_RING; ++i) {
       ptx::mbar_init(&bars->ring.full[i], 1);
@@ -256,10 +260,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ query rows
-    const int r = threadIdx.x;  // row in the tile == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t tS0 = tmem + lane_base;
-    const uint32_t tDP0 = tmem + lane_base + DP_COL;
+    const int t = warp / 4;               // warpgroup: takes the global tiles gj with gj & 1 == t
+    const int r = threadIdx.x - 128 * t;  // row in the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + t * BN;
+    const uint32_t tDP = tmem + lane_base + DP_COL + t * BN;
     const uint32_t tDQ = tmem + lane_base + DQ_COL;
     const float sl2 = p.scale_log2;
     uint32_t rs = 0, rph = 0;
@@ -280,30 +285,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int qi = w.qi0 + r;
       const bool row_valid = r < w.q_rows;
       const size_t row = (size_t)(w.q0 + r) * p.H + w.hu;  // into [total_q, H]
-      uint16_t *dq_row = bp.dq + row * D;
+      // each warpgroup writes half of the dQ row's columns
+      uint16_t *dq_half = bp.dq + row * D + t * (D / 2);
       float delta = 0.f, lse2 = INFINITY;  // invalid rows: p = exp2(-inf) = 0
       if (row_valid) {
         delta = row_delta<D, BF16>(bp.dout + row * D, bp.o + row * D);
-        bp.delta[row] = delta;
+        if (t == 0) bp.delta[row] = delta;
         lse2 = __ldg(bp.lse + row) * LOG2E;
       }
       if (n == 0) {
-        if (row_valid) zero_row<D>(dq_row);
+        if (row_valid) zero_row<D / 2>(dq_half);
         continue;
       }
       const int hi = key_hi(p, qi, w.Lk);  // visible keys [0, hi)
-      for (int j = 0; ok && j < n; ++j) {
+      for (int j = (int)((t - g) & 1u); ok && j < n; j += 2) {
         const uint32_t gj = g + j;
-        const uint32_t buf = gj & 1u;
-        bool got = wait_bar(&bars->s_full[buf], (gj >> 1) & 1u, abort_flag);
+        bool got = wait_bar(&bars->s_full[t], (gj >> 1) & 1u, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
         uint32_t sv[BN], dpv[BN];
-        tmem_ld_wait<BN>(tS0 + buf * BN, sv);
-        tmem_ld_wait<BN>(tDP0 + buf * BN, dpv);
+        tmem_ld_wait<BN>(tS, sv);
+        tmem_ld_wait<BN>(tDP, dpv);
         const int lim = hi - j * BN;
         uint32_t pk[BN / 2];
 #pragma unroll
@@ -317,11 +322,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           pk[c / 2] = pack2<BF16>(ds[0], ds[1]);
         }
-        tmem_st<BN / 2>(tS0 + buf * BN, pk);
+        tmem_st<BN / 2>(tS, pk);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->ds_full[buf]);
+        if (lane == 0) ptx::mbar_arrive(&bars->ds_full[t]);
       }
       if (!ok) break;
       g += n;
@@ -329,7 +334,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ++items;
       if (!__all_sync(0xffffffffu, got)) break;
       ptx::tc_fence_after();
-      store_tmem_row<D, BF16>(tDQ, bp.scale, row_valid, dq_row);
+      store_tmem_row<D / 2, BF16>(tDQ + t * (D / 2), bp.scale, row_valid, dq_half);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->dq_free);
