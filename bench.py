@@ -103,10 +103,18 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_hash(read=None) -> str:
-    """Hash of every CUDA source of the library (file names sorted)."""
+# Device-code sources of each direction's kernels (the host code does not
+# change a kernel's traffic).
+KERNEL_SOURCES = {
+    "fwd": ("sm100_ptx.cuh", "fwd_common.cuh", "fwd_pair.cuh", "fwd_single.cuh"),
+    "bwd": ("sm100_ptx.cuh", "fwd_common.cuh", "bwd_common.cuh", "bwd_dq.cuh", "bwd_dkdv.cuh"),
+}
+
+
+def kernel_hash(read=None, kind: str = "fwd") -> str:
+    """Hash of the device-code sources of the forward or backward kernels."""
     d = os.path.join(ROOT, KERNEL_DIR)
-    names = sorted(n for n in os.listdir(d) if n.endswith((".cu", ".cuh")))
+    names = sorted(KERNEL_SOURCES[kind])
     h = hashlib.sha256()
     for n in names:
         h.update(n.encode())
@@ -122,7 +130,8 @@ def traffic_for(workload: str):
         with open(path) as f:
             d = json.load(f)
         ent = d.get(workload)
-        if ent and ent.get("kernel_hash") == kernel_hash():
+        kind = "bwd" if workload.endswith(":bwd") else "fwd"
+        if ent and ent.get("kernel_hash") == kernel_hash(kind=kind):
             return ent.get("bytes_per_launch")
     except Exception:
         pass
