@@ -397,6 +397,22 @@ def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist, extra=())
     return e2e_ms, h2d, d2h
 
 
+def hbm_line(case, avg_launch_ms: float, peaks: dict, peak_src: str, traffic_key: str,
+             flops: int):
+    """HBM side of the roofline: algorithmic bytes per launch (Q, K, V read
+    once, O and LSE written once) / launch time against the measured copy
+    bandwidth, and the arithmetic intensity against the ridge point."""
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    nbytes = algorithmic_bytes(case)
+    gbs = nbytes / (avg_launch_ms * 1e-3) / 1e9
+    return {"achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+            "algorithmic_bytes": nbytes, "traffic": traffic_for(traffic_key),
+            "flop_per_byte": round(flops / nbytes, 1),
+            "ridge_flop_per_byte": round(peak * 1e12 / (hbm * 1e9), 1),
+            "peak_source": "%s copy bandwidth" % peak_src}
+
+
 def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk,
          metric=METRIC, cpu_fn=None, launches_per_step=1, traffic_key=None):
     if rank == 0:
@@ -439,6 +455,8 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
                          "traffic": traffic_for(traffic_key or args.workload),
                          "peak_source": "%s burst bf16 (sustained %.1f -> frac %.4f)"
                                         % (peak_src, peak_sus, achieved / peak_sus)},
+            "hbm": hbm_line(case, avg_launch_ms, peaks, peak_src, traffic_key or args.workload,
+                            flops),
             "launch_ms": {"min": round(min(per_launch), 4),
                           "median": round(statistics.median(per_launch), 4),
                           "max": round(max(per_launch), 4)},
