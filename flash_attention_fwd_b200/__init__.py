@@ -39,6 +39,9 @@ EXPORTED_SYMBOLS = (
     "varlen_attn_fwd_v1",
     "varlen_attn_fwd_v2",
     "varlen_attn_fwd_v3",
+    "varlen_attn_fwd_v4",
+    "varlen_attn_fwd_num_splits",
+    "varlen_attn_fwd_workspace_size",
     "varlen_attn_fwd",
     "varlen_attn_strerror",
     "varlen_attn_device_status",
@@ -73,6 +76,15 @@ def _bind(lib):
     lib.varlen_attn_fwd_v3.argtypes = (fwd_args[:15] + [i32, i32, P, P, i32, i32, P]
                                        + fwd_args[15:])
     lib.varlen_attn_fwd_v3.restype = i32
+    # v4: v3's arguments with num_splits, workspace, workspace_bytes after sinks
+    lib.varlen_attn_fwd_v4.argtypes = (fwd_args[:15] + [i32, i32, P, P, i32, i32, P, i32, P,
+                                                        ctypes.c_size_t] + fwd_args[15:])
+    lib.varlen_attn_fwd_v4.restype = i32
+    lib.varlen_attn_fwd_num_splits.argtypes = [i32, i64, i64, i32, i32, i32, i32, i32, i32, i32,
+                                               i32, i32, i32]
+    lib.varlen_attn_fwd_num_splits.restype = i32
+    lib.varlen_attn_fwd_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+    lib.varlen_attn_fwd_workspace_size.restype = ctypes.c_size_t
     lib.varlen_attn_strerror.argtypes = [i32]
     lib.varlen_attn_strerror.restype = ctypes.c_char_p
     lib.varlen_attn_device_status.argtypes = [ctypes.POINTER(ctypes.c_uint), i32]
@@ -132,17 +144,25 @@ def varlen_attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, cu_q_ptr: int, cu_k_
                         lse_ptr: int, stream: int, window_left: int = -1,
                         window_right: int = -1, seqused_k_ptr: int = 0,
                         page_table_ptr: int = 0, page_table_stride: int = 0,
-                        page_size: int = 0, sinks_ptr: int = 0) -> int:
+                        page_size: int = 0, sinks_ptr: int = 0, num_splits: int = 1,
+                        workspace_ptr: int = 0, workspace_bytes: int = 0) -> int:
     """Direct call of the C entry point with integer addresses; returns the
     status code unchanged.  Calls varlen_attn_fwd (v1) unless a window bound,
-    a seqused_k array, a page table or sinks are given; varlen_attn_fwd_v2 for
-    a window / seqused_k, varlen_attn_fwd_v3 for a page table or sinks."""
+    a seqused_k array, a page table, sinks or num_splits != 1 are given;
+    varlen_attn_fwd_v2 for a window / seqused_k, varlen_attn_fwd_v3 for a page
+    table or sinks, varlen_attn_fwd_v4 for a key-range split."""
     lib = load_library()
     V = ctypes.c_void_p
     head = (V(q_ptr), V(k_ptr), V(v_ptr), V(cu_q_ptr), V(cu_k_ptr), int(batch), int(total_q),
             int(total_k), int(max_seqlen_q), int(max_seqlen_k), int(num_heads),
             int(num_kv_heads), int(head_dim), int(bool(causal)), float(scale))
     tail = (int(dtype_code), V(out_ptr), V(lse_ptr), V(stream))
+    if num_splits != 1:
+        return lib.varlen_attn_fwd_v4(*head, int(window_left), int(window_right),
+                                      V(seqused_k_ptr), V(page_table_ptr),
+                                      int(page_table_stride), int(page_size), V(sinks_ptr),
+                                      int(num_splits), V(workspace_ptr), int(workspace_bytes),
+                                      *tail)
     if page_table_ptr or sinks_ptr:
         return lib.varlen_attn_fwd_v3(*head, int(window_left), int(window_right),
                                       V(seqused_k_ptr), V(page_table_ptr),
@@ -163,7 +183,9 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                     window_size_left: int = -1, window_size_right: int = -1,
                     seqused_k: Optional[torch.Tensor] = None,
                     page_table: Optional[torch.Tensor] = None,
-                    sinks: Optional[torch.Tensor] = None
+                    sinks: Optional[torch.Tensor] = None,
+                    num_splits: Optional[int] = None,
+                    workspace: Optional[torch.Tensor] = None
                     ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Packed attention forward on the GPU.
 
@@ -186,6 +208,12 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     ``sinks`` (float32 [H] on the device) adds one logit per query head to
     the softmax normalisation (attention sinks): the row's weights become
     exp(s - m) / (sum exp(s - m) + exp(sinks[h] - m)).
+
+    ``num_splits`` (non-causal calls without a window only): the key range of
+    a row may be computed in up to that many pieces merged by their LSE
+    (varlen_attn_fwd_v4); None lets the library choose, 1 turns it off.  The
+    pieces need a device workspace, allocated here unless ``workspace`` (a
+    uint8 CUDA tensor of at least ``fwd_workspace_size(...)`` bytes) is given.
     """
     if q.dtype not in DTYPE_CODES or k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share dtype bfloat16 or float16")
@@ -243,16 +271,63 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     def addr(t):
         return t.data_ptr() if t is not None and t.numel() else 0
 
+    splits, ws_bytes = 1, 0
+    if not causal and window_size_left < 0 and window_size_right < 0 and num_splits != 1:
+        splits = (fwd_num_splits(B, total_q, total_k, max_seqlen_q, max_seqlen_k, H, Hkv, D,
+                                 paged=paged, device=q.device)
+                  if num_splits is None else int(num_splits))
+        ws_bytes = fwd_workspace_size(total_q, H, D, max_seqlen_k, splits) if splits > 1 else 0
+        if ws_bytes == 0:
+            splits = 1
+        elif workspace is None:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+        elif (not workspace.is_cuda or workspace.dtype != torch.uint8
+              or not workspace.is_contiguous() or workspace.numel() < ws_bytes):
+            raise ValueError("workspace must be a contiguous uint8 CUDA tensor of at least "
+                             "%d bytes" % ws_bytes)
     with torch.cuda.device(q.device):
         rc = varlen_attn_fwd_raw(
             addr(q), addr(k), addr(v), addr(cu_seqlens_q), addr(cu_seqlens_k), B,
             total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), H, Hkv, D, causal,
             0.0 if scale is None else float(scale), DTYPE_CODES[q.dtype], addr(out), addr(lse),
             stream.cuda_stream, int(window_size_left), int(window_size_right), addr(seqused_k),
-            addr(page_table), stride, page_size, addr(sinks))
+            addr(page_table), stride, page_size, addr(sinks), splits,
+            addr(workspace) if splits > 1 else 0, ws_bytes)
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return out, lse
+
+
+_sms = {}
+
+
+def fwd_num_splits(batch: int, total_q: int, total_k: int, max_seqlen_q: int, max_seqlen_k: int,
+                   num_heads: int, num_kv_heads: int, head_dim: int, causal: bool = False,
+                   window_size_left: int = -1, window_size_right: int = -1, paged: bool = False,
+                   device=None, num_sms: Optional[int] = None) -> int:
+    """Key-range piece count the library picks for these sizes
+    (varlen_attn_fwd_num_splits); ``num_sms`` defaults to the device's."""
+    if num_sms is None:
+        dev = torch.device(device if device is not None else "cuda")
+        idx = dev.index if dev.index is not None else torch.cuda.current_device()
+        if idx not in _sms:
+            _sms[idx] = torch.cuda.get_device_properties(idx).multi_processor_count
+        num_sms = _sms[idx]
+    rc = load_library().varlen_attn_fwd_num_splits(
+        int(batch), int(total_q), int(total_k), int(max_seqlen_q), int(max_seqlen_k),
+        int(num_heads), int(num_kv_heads), int(head_dim), int(bool(causal)),
+        int(window_size_left), int(window_size_right), int(bool(paged)), int(num_sms))
+    if rc < 0:
+        raise VarlenAttnError(rc, strerror(rc))
+    return int(rc)
+
+
+def fwd_workspace_size(total_q: int, num_heads: int, head_dim: int, max_seqlen_k: int,
+                       num_splits: int) -> int:
+    """Bytes of device workspace a forward split into at most ``num_splits``
+    pieces needs (0: no split happens)."""
+    return int(load_library().varlen_attn_fwd_workspace_size(
+        int(total_q), int(num_heads), int(head_dim), int(max_seqlen_k), int(num_splits)))
 
 
 def bwd_workspace_size(total_q: int, num_heads: int) -> int:

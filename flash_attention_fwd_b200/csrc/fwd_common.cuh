@@ -59,7 +59,58 @@ struct KParams {
   int num_pages;
   int page_chunk;  // rows per TMA box of a paged K/V tile (divides page_size and the key tile)
   const float *sinks;  // optional [H]: one extra logit per query head in the softmax normalisation
+  // Key-range split (only without the causal rule and without a window): a
+  // work item whose sequence has more than split_tiles key tiles of BM keys is
+  // cut into P = min(ceil(nk / split_tiles), max_parts) pieces of near-equal
+  // tile counts.  Piece i of row `row` (= token * H + head) writes O / l as
+  // float32 to part_o[(i * part_rows + row) * D ...] and its log2-domain LSE to
+  // part_lse[i * part_rows + row]; the combine kernel merges the pieces.
+  int split_tiles;  // 0: no item is split
+  int max_parts;
+  long long part_rows;  // total_q * H
+  float *part_o;
+  float *part_lse;
 };
+
+// Pieces of a key range of nk tiles: P pieces, the first r of base + 1 tiles
+// and the other P - r of base tiles (P = 1, base = nk when it is not split).
+__device__ __forceinline__ void kv_pieces(int nk, int split_tiles, int max_parts, int &P,
+                                          int &base, int &r) {
+  P = (split_tiles > 0 && nk > split_tiles) ? min((nk + split_tiles - 1) / split_tiles, max_parts)
+                                            : 1;
+  if (P < 1) P = 1;
+  base = nk / P;
+  r = nk - base * P;
+}
+
+// Query and key extents of sequence b, clamped into the buffers (so that an
+// inconsistent sequence table can never address memory outside them): queries
+// [qs, qs + lq) of the packed q, keys [ks, ks + lk) of the packed k/v (paged:
+// ks = 0 and lk = the used keys, at most paged_keys).
+__device__ __forceinline__ void seq_extents(const int *cu_q, const int *cu_k,
+                                            const int *seqused_k, bool paged, int paged_keys,
+                                            int total_q, int total_k, int b, int &qs, int &lq,
+                                            int &ks, int &lk) {
+  qs = __ldg(cu_q + b);
+  int qe = __ldg(cu_q + b + 1);
+  qs = min(max(qs, 0), total_q);
+  qe = min(max(qe, qs), total_q);
+  lq = qe - qs;
+  if (paged) {
+    ks = 0;
+    lk = min(max(__ldg(seqused_k + b), 0), paged_keys);
+    return;
+  }
+  ks = __ldg(cu_k + b);
+  int ke = __ldg(cu_k + b + 1);
+  ks = min(max(ks, 0), total_k);
+  ke = min(max(ke, ks), total_k);
+  lk = ke - ks;
+  if (seqused_k) lk = min(lk, max(__ldg(seqused_k + b), 0));
+}
+__device__ __forceinline__ int paged_key_extent(const KParams &p) {
+  return (int)min((long long)p.pt_stride * p.page_size, (long long)INT32_MAX);
+}
 
 // Sink logit of query head h in log2 units (-inf: none).
 __device__ __forceinline__ float sink_log2(const KParams &p, int h) {
@@ -81,6 +132,7 @@ struct WorkItem {
   int q0;       // packed index of the item's first query token
   int q_rows;   // valid query tokens in the item (<= unit_tokens)
   int qi0;      // sequence-local index of the item's first query
+  int part;     // piece of a split key range (-1: the item covers all its keys)
   int k0;       // packed index of the first key of the first visited key tile
   int kofs;     // sequence-local index of that key (a multiple of the key tile)
   int Lk;       // used keys in the sequence
@@ -124,41 +176,31 @@ struct Scheduler {
   long long level_items;  // items in the level
   int cur_b;              // cursor inside the level: first sequence not passed yet
   long long cur_units;    // (sequence, query tile) units before cur_b in this level
+  int split_tiles, max_parts;
 
   __device__ void extents(int b, int &qs, int &lq, int &ks, int &lk) const {
-    qs = __ldg(cu_q + b);
-    int qe = __ldg(cu_q + b + 1);
-    qs = min(max(qs, 0), total_q);
-    qe = min(max(qe, qs), total_q);
-    lq = qe - qs;
-    if (paged) {
-      ks = 0;
-      lk = min(max(__ldg(seqused_k + b), 0), paged_keys);
-      return;
-    }
-    ks = __ldg(cu_k + b);
-    int ke = __ldg(cu_k + b + 1);
-    ks = min(max(ks, 0), total_k);
-    ke = min(max(ke, ks), total_k);
-    lk = ke - ks;
-    if (seqused_k) lk = min(lk, max(__ldg(seqused_k + b), 0));
+    seq_extents(cu_q, cu_k, seqused_k, paged, paged_keys, total_q, total_k, b, qs, lq, ks, lk);
   }
-  // (sequence, query range) units of a sequence at cost level c; nq ranges of
-  // U tokens, nk tiles of BM keys
+  // (sequence, query range[, key piece]) units of a sequence at cost level c;
+  // nq ranges of U tokens, nk tiles of BM keys.  Without the causal rule a
+  // split key range gives each query range P pieces, at levels base + 1 and
+  // base.
   __device__ int units_at(int nq, int nk, int c) const {
-    if (!causal || nk == 0) return (c == nk) ? nq : 0;
+    if (!causal || nk == 0) {
+      int P, base, r;
+      kv_pieces(nk, split_tiles, max_parts, P, base, r);
+      return nq * ((c == base ? P - r : 0) + (r > 0 && c == base + 1 ? r : 0));
+    }
     if (c >= 1 && c < nk) return max(0, min(c * R, nq) - (c - 1) * R);
     if (c == nk) return max(0, nq - (nk - 1) * R);
     return 0;
   }
-  // query range of the k-th unit of a sequence at level c
-  __device__ int tile_of(int nk, int c, int k) const {
-    if (causal && nk > 0) return (min(c, nk) - 1) * R + k;
-    return k;
-  }
   __device__ int top_level(int nq, int nk) const {
     if (nq == 0) return -1;
-    return (causal && nk > 0) ? min(nk, (nq + R - 1) / R) : nk;
+    if (causal && nk > 0) return min(nk, (nq + R - 1) / R);
+    int P, base, r;
+    kv_pieces(nk, split_tiles, max_parts, P, base, r);
+    return r > 0 ? base + 1 : base;
   }
   __device__ long long count_level(int c) const {
     long long u = 0;
@@ -181,7 +223,9 @@ struct Scheduler {
     cu_k = p.cu_k;
     seqused_k = p.seqused_k;
     paged = p.page_table != nullptr;
-    paged_keys = (int)min((long long)p.pt_stride * p.page_size, (long long)INT32_MAX);
+    paged_keys = paged_key_extent(p);
+    split_tiles = p.split_tiles;
+    max_parts = p.max_parts;
     B = p.B;
     HU = p.head_units;
     U = p.unit_tokens;
@@ -253,19 +297,52 @@ struct Scheduler {
         cur_units += before;
         w.b = cur_b;
         const int k = (int)(unit - cur_units);
-        const int qt = tile_of((lk + BM - 1) / BM, level, k);
+        const int nk = (lk + BM - 1) / BM;
+        int qt, t0 = 0, nt = 0;
+        w.part = -1;
+        if (causal && nk > 0) {
+          qt = (min(level, nk) - 1) * R + k;
+        } else {
+          // units of the level: (piece, query range) with the range fastest, so
+          // the query ranges that share a piece's K/V tiles run side by side
+          int P, base, r;
+          kv_pieces(nk, split_tiles, max_parts, P, base, r);
+          const int nq = (lq + U - 1) / U;
+          qt = k % nq;
+          int i = k / nq;
+          if (r > 0 && level == base + 1) {
+            t0 = i * (base + 1);
+            nt = base + 1;
+          } else {
+            i += r;
+            t0 = r * (base + 1) + (i - r) * base;
+            nt = base;
+          }
+          if (P > 1) w.part = i;
+        }
         w.qi0 = qt * U;
         w.q0 = qs + w.qi0;
         w.q_rows = min(U, lq - w.qi0);
         w.Lk = lk;
-        // key tiles spanned by the visible keys of the first and last query
-        const int qa = w.qi0, qb = w.qi0 + w.q_rows - 1;
-        const int lo_a = key_lo(p, qa), hi_b = key_hi(p, qb, lk);
-        w.kofs = (lo_a / BN) * BN;
-        w.k0 = ks + w.kofs;
-        w.n_kv = hi_b > lo_a ? (hi_b - w.kofs + BN - 1) / BN : 0;
-        w.min_hi = key_hi(p, qa, lk) - w.kofs;
-        w.max_lo = key_lo(p, qb) - w.kofs;
+        if (w.part < 0) {
+          // key tiles spanned by the visible keys of the first and last query
+          const int qa = w.qi0, qb = w.qi0 + w.q_rows - 1;
+          const int lo_a = key_lo(p, qa), hi_b = key_hi(p, qb, lk);
+          w.kofs = (lo_a / BN) * BN;
+          w.k0 = ks + w.kofs;
+          w.n_kv = hi_b > lo_a ? (hi_b - w.kofs + BN - 1) / BN : 0;
+          w.min_hi = key_hi(p, qa, lk) - w.kofs;
+          w.max_lo = key_lo(p, qb) - w.kofs;
+        } else {
+          // keys [t0 * BM, min((t0 + nt) * BM, lk)); every row sees all keys
+          // (a split range has no window and no causal rule)
+          const int kend = min((t0 + nt) * BM, lk);
+          w.kofs = t0 * BM;
+          w.k0 = ks + w.kofs;
+          w.n_kv = (kend - w.kofs + BN - 1) / BN;
+          w.min_hi = lk - w.kofs;
+          w.max_lo = -w.kofs;
+        }
         return true;
       }
       cur_b += 32;
@@ -689,6 +766,36 @@ __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, floa
     }
   }
   if (row_valid) *lse_ptr = any ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+}
+
+// Epilogue of one row of a piece of a split key range: O / l as float32 and
+// the piece's LSE in log2 units (m + log2 l; -inf and O = 0 when the piece has
+// no visible key for the row).  Sinks are left to the combine.
+template <int D>
+__device__ __forceinline__ void epilogue_part(uint32_t tO, float m, float l, bool row_valid,
+                                              float *part_o_row, float *part_lse, uint64_t *o_free,
+                                              int lane) {
+  const bool any = l > 0.f;
+  const float inv_l = any ? 1.f / l : 0.f;
+#pragma unroll
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    uint32_t o[32];
+    tmem_ld_wait<32>(tO + c0, o);
+    if (c0 + 32 == D) {
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(o_free);
+    }
+    if (row_valid) {
+      float4 *dst = reinterpret_cast<float4 *>(part_o_row + c0);
+#pragma unroll
+      for (int v4 = 0; v4 < 8; ++v4)
+        dst[v4] = make_float4(__uint_as_float(o[4 * v4]) * inv_l, __uint_as_float(o[4 * v4 + 1]) * inv_l,
+                              __uint_as_float(o[4 * v4 + 2]) * inv_l,
+                              __uint_as_float(o[4 * v4 + 3]) * inv_l);
+    }
+  }
+  if (row_valid) *part_lse = any ? m + log2f(l) : -INFINITY;
 }
 
 // A query row of an item without visible keys: O = 0, LSE = the sink logit

@@ -493,8 +493,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      epilogue_row<D, BF16>(tO, m, l, sink_log2(p, h), row_valid, orow_ptr, p.lse + orow,
-                            &bars->o_free[t], lane);
+      if (w.part < 0)
+        epilogue_row<D, BF16>(tO, m, l, sink_log2(p, h), row_valid, orow_ptr, p.lse + orow,
+                              &bars->o_free[t], lane);
+      else
+        epilogue_part<D>(tO, m, l, row_valid, p.part_o + ((size_t)w.part * p.part_rows + orow) * D,
+                         p.part_lse + (size_t)w.part * p.part_rows + orow, &bars->o_free[t], lane);
     }
     end_of_kernel();
   }

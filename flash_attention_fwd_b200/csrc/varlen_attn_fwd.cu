@@ -29,6 +29,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include "fwd_combine.cuh"
 #include "fwd_common.cuh"
 #include "fwd_pair.cuh"
 #include "fwd_single.cuh"
@@ -130,6 +131,104 @@ static int launch_pair(const CUtensorMap &tq, const CUtensorMap &tk, const CUten
 
 static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+template <int D, bool BF16>
+static int launch_combine(const KParams &kp, int sms, cudaStream_t s) {
+  const long long blocks = (kp.part_rows + combine::ROWS_PER_CTA - 1) / combine::ROWS_PER_CTA;
+  const int grid = (int)(blocks < (long long)sms * 16 ? blocks : (long long)sms * 16);
+  combine::combine_kernel<D, BF16><<<grid < 1 ? 1 : grid, combine::NUM_THREADS, 0, s>>>(kp);
+  return cudaGetLastError() == cudaSuccess ? VARLEN_OK : VARLEN_ERR_LAUNCH;
+}
+
+// Which kernel serves a call, and how it cuts the queries into work items.
+struct FwdLayout {
+  bool use_pair;    // pair kernel (two query tiles per item sharing K/V)
+  int pack_log2;    // GQA packing (see KParams::pack_log2)
+  int head_units;   // head units per (sequence, token range)
+  int unit_tokens;  // query tokens per work item
+};
+static FwdLayout fwd_layout(int max_seqlen_q, int num_heads, int num_kv_heads, int D) {
+  FwdLayout L;
+  const int group = num_heads / num_kv_heads;
+  // Query-head pairs share a key/value head when the group size is even;
+  // the pair kernel then covers D = 64 and 128 (TMEM holds 2 x (S + O)).
+  L.use_pair = (group % 2 == 0) && (D == 64 || D == 128);
+  // GQA packing: a tile's 128 rows = (128 / group) tokens x the group's query
+  // heads.  It pays when query sequences are short next to a 128-row tile
+  // (most rows of a per-head tile would be empty); group must be a power of
+  // two dividing 128.
+  L.pack_log2 = 0;
+  if (L.use_pair && (group & (group - 1)) == 0 && group <= BM) {
+    const bool short_q = (long long)max_seqlen_q * 2 <= BM;
+    if (PAIR_PACK_POLICY == 1 || (PAIR_PACK_POLICY == 2 && short_q))
+      while ((1 << L.pack_log2) < group) ++L.pack_log2;
+  }
+  L.head_units = L.pack_log2 ? num_kv_heads : (L.use_pair ? num_heads / 2 : num_heads);
+  L.unit_tokens = L.pack_log2 ? 2 * (BM >> L.pack_log2) : BM;
+  return L;
+}
+
+// Key tiles per piece and the largest piece count when a call asks for at
+// most num_splits pieces per key range (no split: num_splits <= 1, a causal
+// rule or a window, or no sequence long enough to be cut).
+static void split_plan(int num_splits, int max_seqlen_k, bool masked, int &split_tiles,
+                       int &max_parts) {
+  split_tiles = 0;
+  max_parts = 1;
+  if (num_splits <= 1 || masked || max_seqlen_k <= 0) return;
+  const int nk_max = (int)(((long long)max_seqlen_k + BM - 1) / BM);
+  const int S = (nk_max + num_splits - 1) / num_splits;
+  if (S < 1 || nk_max <= S) return;
+  split_tiles = S;
+  max_parts = (nk_max + S - 1) / S;
+}
+
+// Piece count chosen when the caller leaves it to the library.  A piece is a
+// work item of its own (Q load, pipeline start, epilogue) and the merge is a
+// second launch over float32 partials of every row, so a split pays only when
+// the work items alone cannot fill the GPU (fewer than 3/4 as many items as
+// SMs): then each key range is cut into up to 16 pieces of at least 16 key
+// tiles, so that the pieces of the few long items spread over all SMs in
+// several rounds that the cost-ordered dealing evens out.  Measured on B200:
+// 8 single-query sequences x 8 KV heads x 32k keys, 0.61 ms unsplit, 0.27 ms
+// in 16 pieces; 208 short-query items over up to 63 key tiles (the
+// short-query / long-KV batch), every split slower than none.
+static int auto_num_splits(int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
+                           int max_seqlen_k, int num_heads, int num_kv_heads, int D, bool masked,
+                           bool paged, int sms) {
+  (void)total_k;
+  (void)paged;
+  if (masked || batch <= 0 || max_seqlen_k <= 0 || max_seqlen_q <= 0 || sms <= 0) return 1;
+  const FwdLayout L = fwd_layout(max_seqlen_q, num_heads, num_kv_heads, D);
+  const double nk_max = ceil((double)max_seqlen_k / BM);
+  const double q_mean = fmin((double)total_q / batch, (double)max_seqlen_q);
+  const double items = (double)batch * fmax(1.0, ceil(q_mean / L.unit_tokens)) * L.head_units;
+  if (items >= 0.75 * sms) return 1;
+  const double ns = fmin(16.0, floor(nk_max / 16.0));
+  return ns < 2.0 ? 1 : (ns > combine::MAX_PARTS ? combine::MAX_PARTS : (int)ns);
+}
+
+static size_t split_workspace_bytes(int64_t total_q, int num_heads, int D, int max_parts) {
+  return (size_t)max_parts * (size_t)total_q * (size_t)num_heads * (size_t)(D + 1) * 4u;
+}
+
+static int device_sms(DeviceInfo *&dev_out) {
+  int dev_id = 0;
+  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= 64) return VARLEN_ERR_LAUNCH;
+  DeviceInfo &dev = g_dev[dev_id];
+  if (dev.sms == 0) {
+    int sms = 0, mj = 0, mn = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id) != cudaSuccess ||
+        cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, dev_id) != cudaSuccess ||
+        cudaDeviceGetAttribute(&mn, cudaDevAttrComputeCapabilityMinor, dev_id) != cudaSuccess)
+      return VARLEN_ERR_LAUNCH;
+    dev.major = mj;
+    dev.minor = mn;
+    dev.sms = sms;
+  }
+  dev_out = &dev;
+  return VARLEN_OK;
+}
+
 }  // namespace vattn
 
 using namespace vattn;
@@ -151,8 +250,9 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
                     int max_seqlen_q, int max_seqlen_k, int num_heads, int num_kv_heads,
                     int head_dim, int causal, float scale, int window_left, int window_right,
                     const int32_t *seqused_k, const int32_t *page_table, int page_table_stride,
-                    int page_size, const float *sinks, varlen_dtype_t dtype, void *out,
-                    float *lse, varlen_stream_t stream) {
+                    int page_size, const float *sinks, int num_splits, void *workspace,
+                    size_t workspace_bytes, varlen_dtype_t dtype, void *out, float *lse,
+                    varlen_stream_t stream) {
   const bool paged = page_table != nullptr;
   // ---- host-side validation: nothing is launched or touched on error
   if (dtype != VARLEN_BF16 && dtype != VARLEN_FP16) return VARLEN_ERR_DTYPE;
@@ -175,22 +275,12 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   if (!aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4) ||
       !aligned(seqused_k, 4) || !aligned(page_table, 4) || !aligned(sinks, 4))
     return VARLEN_ERR_ALIGN;
+  if (num_splits < 0 || num_splits > combine::MAX_PARTS) return VARLEN_ERR_SHAPE;
   if (batch == 0 || total_q == 0) return VARLEN_OK;
 
-  int dev_id = 0;
-  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= 64)
-    return VARLEN_ERR_LAUNCH;
-  DeviceInfo &dev = g_dev[dev_id];
-  if (dev.sms == 0) {
-    int sms = 0, mj = 0, mn = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id) != cudaSuccess ||
-        cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, dev_id) != cudaSuccess ||
-        cudaDeviceGetAttribute(&mn, cudaDevAttrComputeCapabilityMinor, dev_id) != cudaSuccess)
-      return VARLEN_ERR_LAUNCH;
-    dev.major = mj;
-    dev.minor = mn;
-    dev.sms = sms;
-  }
+  DeviceInfo *devp = nullptr;
+  if (const int rc = device_sms(devp)) return rc;
+  DeviceInfo &dev = *devp;
   if (dev.major != 10 || dev.minor != 0) return VARLEN_ERR_ARCH;
 
   EncodeTiledFn enc = get_encode_fn();
@@ -198,19 +288,9 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   const bool bf16 = dtype == VARLEN_BF16;
   const int D = head_dim;
   const int group = num_heads / num_kv_heads;
-  // Query-head pairs share a key/value head when the group size is even;
-  // the pair kernel then covers D = 64 and 128 (TMEM holds 2 x (S + O)).
-  const bool use_pair = (group % 2 == 0) && (D == 64 || D == 128);
-  // GQA packing: a tile's 128 rows = (128 / group) tokens x the group's query
-  // heads.  It pays when query sequences are short next to a 128-row tile
-  // (most rows of a per-head tile would be empty); group must be a power of
-  // two dividing 128.
-  int pack_log2 = 0;
-  if (use_pair && (group & (group - 1)) == 0 && group <= BM) {
-    const bool short_q = (long long)max_seqlen_q * 2 <= BM;
-    if (PAIR_PACK_POLICY == 1 || (PAIR_PACK_POLICY == 2 && short_q))
-      while ((1 << pack_log2) < group) ++pack_log2;
-  }
+  const FwdLayout layout = fwd_layout(max_seqlen_q, num_heads, num_kv_heads, D);
+  const bool use_pair = layout.use_pair;
+  const int pack_log2 = layout.pack_log2;
   const int BN = use_pair ? pair::BN : (D == 256 ? single::Cfg<256>::BN : single::Cfg<128>::BN);
   alignas(64) CUtensorMap tq, tk, tv;
   memset(&tk, 0, sizeof tk);
@@ -236,8 +316,8 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   kp.H = num_heads;
   kp.Hkv = num_kv_heads;
   kp.group = group;
-  kp.head_units = pack_log2 ? num_kv_heads : (use_pair ? num_heads / 2 : num_heads);
-  kp.unit_tokens = pack_log2 ? 2 * (BM >> pack_log2) : BM;
+  kp.head_units = layout.head_units;
+  kp.unit_tokens = layout.unit_tokens;
   kp.pack_log2 = pack_log2;
   kp.total_q = (int)total_q;
   kp.total_k = (int)total_k;
@@ -260,33 +340,67 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   kp.num_pages = paged ? (int)(total_k / page_size) : 0;
   kp.page_chunk = chunk;
   kp.sinks = sinks;
+  // Key-range split (non-causal, windowless calls): pieces merged by the
+  // combine kernel through the caller's workspace.
+  const bool masked = kp.win_left >= 0 || kp.win_right >= 0;
+  if (num_splits == 0)
+    num_splits = auto_num_splits(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads,
+                                 num_kv_heads, D, masked, paged, dev.sms);
+  split_plan(num_splits, max_seqlen_k, masked, kp.split_tiles, kp.max_parts);
+  kp.part_rows = (long long)total_q * num_heads;
+  kp.part_o = nullptr;
+  kp.part_lse = nullptr;
+  if (kp.split_tiles > 0) {
+    const size_t need = split_workspace_bytes(total_q, num_heads, D, kp.max_parts);
+    if (!workspace || !aligned(workspace, 16) || workspace_bytes < need)
+      return VARLEN_ERR_WORKSPACE;
+    kp.part_o = static_cast<float *>(workspace);
+    kp.part_lse = kp.part_o + (size_t)kp.max_parts * (size_t)kp.part_rows * D;
+  }
 
   // Upper bound of work items from max_seqlen_q; at least one CTA so that an
   // understated bound never drops work (the CTAs loop over all items).
   long long max_items =
-      (long long)batch * ((max_seqlen_q + kp.unit_tokens - 1) / kp.unit_tokens) * kp.head_units;
+      (long long)batch * ((max_seqlen_q + kp.unit_tokens - 1) / kp.unit_tokens) * kp.head_units *
+      kp.max_parts;
   int grid = dev.sms;
   if (max_items >= 1 && max_items < grid) grid = (int)max_items;
   if (grid < 1) grid = 1;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int rc;
   if (use_pair) {
     if (D == 64)
-      return bf16 ? launch_pair<64, true>(tq, tk, tv, kp, grid, s, dev, 0)
-                  : launch_pair<64, false>(tq, tk, tv, kp, grid, s, dev, 1);
-    return bf16 ? launch_pair<128, true>(tq, tk, tv, kp, grid, s, dev, 2)
+      rc = bf16 ? launch_pair<64, true>(tq, tk, tv, kp, grid, s, dev, 0)
+                : launch_pair<64, false>(tq, tk, tv, kp, grid, s, dev, 1);
+    else
+      rc = bf16 ? launch_pair<128, true>(tq, tk, tv, kp, grid, s, dev, 2)
                 : launch_pair<128, false>(tq, tk, tv, kp, grid, s, dev, 3);
+  } else {
+    switch (D) {
+      case 64:
+        rc = bf16 ? launch_single<64, true>(tq, tk, tv, kp, grid, s, dev, 4)
+                  : launch_single<64, false>(tq, tk, tv, kp, grid, s, dev, 5);
+        break;
+      case 128:
+        rc = bf16 ? launch_single<128, true>(tq, tk, tv, kp, grid, s, dev, 6)
+                  : launch_single<128, false>(tq, tk, tv, kp, grid, s, dev, 7);
+        break;
+      default:
+        rc = bf16 ? launch_single<256, true>(tq, tk, tv, kp, grid, s, dev, 8)
+                  : launch_single<256, false>(tq, tk, tv, kp, grid, s, dev, 9);
+    }
   }
+  if (rc != VARLEN_OK || kp.split_tiles == 0) return rc;
   switch (D) {
     case 64:
-      return bf16 ? launch_single<64, true>(tq, tk, tv, kp, grid, s, dev, 4)
-                  : launch_single<64, false>(tq, tk, tv, kp, grid, s, dev, 5);
+      return bf16 ? launch_combine<64, true>(kp, dev.sms, s) : launch_combine<64, false>(kp, dev.sms, s);
     case 128:
-      return bf16 ? launch_single<128, true>(tq, tk, tv, kp, grid, s, dev, 6)
-                  : launch_single<128, false>(tq, tk, tv, kp, grid, s, dev, 7);
+      return bf16 ? launch_combine<128, true>(kp, dev.sms, s)
+                  : launch_combine<128, false>(kp, dev.sms, s);
     default:
-      return bf16 ? launch_single<256, true>(tq, tk, tv, kp, grid, s, dev, 8)
-                  : launch_single<256, false>(tq, tk, tv, kp, grid, s, dev, 9);
+      return bf16 ? launch_combine<256, true>(kp, dev.sms, s)
+                  : launch_combine<256, false>(kp, dev.sms, s);
   }
 }
 
@@ -298,7 +412,7 @@ extern "C" int varlen_attn_fwd_v1(const void *q, const void *k, const void *v,
                                   float *lse, varlen_stream_t stream) {
   return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                   max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, -1, -1, nullptr,
-                  nullptr, 0, 0, nullptr, dtype, out, lse, stream);
+                  nullptr, 0, 0, nullptr, 1, nullptr, 0, dtype, out, lse, stream);
 }
 
 extern "C" int varlen_attn_fwd_v2(const void *q, const void *k, const void *v,
@@ -310,7 +424,8 @@ extern "C" int varlen_attn_fwd_v2(const void *q, const void *k, const void *v,
                                   float *lse, varlen_stream_t stream) {
   return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                   max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, window_left,
-                  window_right, seqused_k, nullptr, 0, 0, nullptr, dtype, out, lse, stream);
+                  window_right, seqused_k, nullptr, 0, 0, nullptr, 1, nullptr, 0, dtype, out, lse,
+                  stream);
 }
 
 extern "C" int varlen_attn_fwd_v3(const void *q, const void *k, const void *v,
@@ -324,8 +439,52 @@ extern "C" int varlen_attn_fwd_v3(const void *q, const void *k, const void *v,
                                   varlen_stream_t stream) {
   return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
                   max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, window_left,
-                  window_right, seqused_k, page_table, page_table_stride, page_size, sinks, dtype,
-                  out, lse, stream);
+                  window_right, seqused_k, page_table, page_table_stride, page_size, sinks, 1,
+                  nullptr, 0, dtype, out, lse, stream);
+}
+
+extern "C" int varlen_attn_fwd_v4(const void *q, const void *k, const void *v,
+                                  const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                  int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
+                                  int max_seqlen_k, int num_heads, int num_kv_heads, int head_dim,
+                                  int causal, float scale, int window_left, int window_right,
+                                  const int32_t *seqused_k, const int32_t *page_table,
+                                  int page_table_stride, int page_size, const float *sinks,
+                                  int num_splits, void *workspace, size_t workspace_bytes,
+                                  varlen_dtype_t dtype, void *out, float *lse,
+                                  varlen_stream_t stream) {
+  return fwd_impl(q, k, v, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
+                  max_seqlen_k, num_heads, num_kv_heads, head_dim, causal, scale, window_left,
+                  window_right, seqused_k, page_table, page_table_stride, page_size, sinks,
+                  num_splits, workspace, workspace_bytes, dtype, out, lse, stream);
+}
+
+extern "C" int varlen_attn_fwd_num_splits(int batch, int64_t total_q, int64_t total_k,
+                                          int max_seqlen_q, int max_seqlen_k, int num_heads,
+                                          int num_kv_heads, int head_dim, int causal,
+                                          int window_left, int window_right, int paged,
+                                          int num_sms) {
+  if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 ||
+      num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+      (head_dim != 64 && head_dim != 128 && head_dim != 256))
+    return VARLEN_ERR_SHAPE;
+  if (num_sms <= 0) {
+    DeviceInfo *dev = nullptr;
+    if (const int rc = device_sms(dev)) return rc;
+    num_sms = dev->sms;
+  }
+  const bool masked = causal || window_left >= 0 || window_right >= 0;
+  return auto_num_splits(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads,
+                         num_kv_heads, head_dim, masked, paged != 0, num_sms);
+}
+
+extern "C" size_t varlen_attn_fwd_workspace_size(int64_t total_q, int num_heads, int head_dim,
+                                                 int max_seqlen_k, int num_splits) {
+  if (total_q <= 0 || num_heads <= 0 || head_dim <= 0 || num_splits > combine::MAX_PARTS)
+    return 0;
+  int split_tiles, max_parts;
+  split_plan(num_splits, max_seqlen_k, false, split_tiles, max_parts);
+  return split_tiles > 0 ? split_workspace_bytes(total_q, num_heads, head_dim, max_parts) : 0;
 }
 
 extern "C" int varlen_attn_fwd(const void *q, const void *k, const void *v,
@@ -361,7 +520,8 @@ extern "C" const char *varlen_attn_strerror(int code) {
     case VARLEN_ERR_ARCH:
       return "current device is not compute capability 10.0 (sm_100a build)";
     case VARLEN_ERR_WORKSPACE:
-      return "workspace missing or smaller than varlen_attn_bwd_workspace_size()";
+      return "workspace missing, not 16-byte aligned, or smaller than "
+             "varlen_attn_fwd_workspace_size() / varlen_attn_bwd_workspace_size()";
     default:
       return "unknown status code";
   }
@@ -379,7 +539,7 @@ extern "C" int varlen_attn_device_status(unsigned int *status, int clear) {
   return VARLEN_OK;
 }
 
-extern "C" int varlen_attn_abi_version(void) { return 4; }
+extern "C" int varlen_attn_abi_version(void) { return 5; }
 
 // Backward entry points (same translation unit: one device status word).
 #include "bwd_host.cuh"

@@ -60,7 +60,7 @@ typedef enum {
 #define VARLEN_ERR_LAUNCH (-5)      /* the CUDA launch itself failed (see varlen_attn_strerror) */
 #define VARLEN_ERR_DEVICE (-6)      /* device-side status word set (see varlen_attn_device_status) */
 #define VARLEN_ERR_ARCH (-7)        /* current device is not compute capability 10.0 (B200/B100 class) */
-#define VARLEN_ERR_WORKSPACE (-8)   /* backward: workspace NULL or smaller than varlen_attn_bwd_workspace_size */
+#define VARLEN_ERR_WORKSPACE (-8)   /* workspace NULL, misaligned or smaller than the *_workspace_size */
 
 /*
  * varlen_attn_fwd_v1 — packed attention forward, output written in place.
@@ -203,6 +203,74 @@ int varlen_attn_fwd_v3(const void *q, const void *k, const void *v,
                        int page_table_stride, int page_size, const float *sinks,
                        varlen_dtype_t dtype, void *out, float *lse, varlen_stream_t stream);
 
+/*
+ * varlen_attn_fwd_v4 — varlen_attn_fwd_v3 plus a split of long key ranges
+ * (same operation and results up to rounding; a new symbol under the
+ * versioned-entry-point rule of PyTorch pull request #176015).
+ *
+ * Without a causal rule and without a window, a query row's softmax over the
+ * keys of its sequence may be computed in pieces: the key range is cut into
+ * at most num_splits ranges of near-equal length, each range gives a partial
+ * result (O_i normalised by its own sum, and lse_i), and a second kernel
+ * merges them exactly as the softmax over the union of the ranges:
+ *   M = max(max_i lse_i, sink),  L = sum_i exp(lse_i - M) + exp(sink - M),
+ *   out = sum_i exp(lse_i - M) / L * O_i,  lse = M + ln L
+ * (sink terms only with sinks).  Short-query / long-key batches then spread
+ * over all SMs instead of leaving a few long work items to a few of them.
+ *
+ *   num_splits   0: the library chooses (varlen_attn_fwd_num_splits); 1: no
+ *                split (exactly v3); 2..32: at most that many pieces per key
+ *                range: pieces hold up to S = ceil(ceil(max_seqlen_k / 128) /
+ *                num_splits) tiles of 128 keys, and a sequence of at most S
+ *                tiles is not cut.  Ignored (no split) with causal or a window.
+ *                Outside [0, 32]: VARLEN_ERR_SHAPE.
+ *   workspace, workspace_bytes   device buffer (16-byte aligned) of at least
+ *                varlen_attn_fwd_workspace_size(total_q, num_heads, head_dim,
+ *                max_seqlen_k, n) bytes, n the piece count in force (for
+ *                num_splits = 0: the value varlen_attn_fwd_num_splits returns
+ *                for the same arguments).  Used only when a split happens
+ *                (NULL is fine otherwise); contents on entry do not matter
+ *                and are scratch afterwards.  Missing, misaligned or too
+ *                small when needed: VARLEN_ERR_WORKSPACE, nothing launched.
+ *
+ * With a split, two kernels run on `stream` in order (attention, then the
+ * merge); the workspace must stay allocated until both have finished.
+ * Everything else is as in v3.
+ */
+int varlen_attn_fwd_v4(const void *q, const void *k, const void *v,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       int batch, int64_t total_q, int64_t total_k,
+                       int max_seqlen_q, int max_seqlen_k,
+                       int num_heads, int num_kv_heads, int head_dim,
+                       int causal, float scale, int window_left, int window_right,
+                       const int32_t *seqused_k, const int32_t *page_table,
+                       int page_table_stride, int page_size, const float *sinks,
+                       int num_splits, void *workspace, size_t workspace_bytes,
+                       varlen_dtype_t dtype, void *out, float *lse, varlen_stream_t stream);
+
+/*
+ * Piece count varlen_attn_fwd_v4 uses for num_splits = 0 with these
+ * arguments (paged: non-zero when a page table is given; num_sms <= 0: the
+ * current device's SM count, which needs a CUDA device).  Host only; returns
+ * >= 1, or a negative code for arguments v4 would reject with
+ * VARLEN_ERR_SHAPE (or VARLEN_ERR_LAUNCH when the device query fails).
+ */
+int varlen_attn_fwd_num_splits(int batch, int64_t total_q, int64_t total_k,
+                               int max_seqlen_q, int max_seqlen_k, int num_heads,
+                               int num_kv_heads, int head_dim, int causal,
+                               int window_left, int window_right, int paged, int num_sms);
+
+/*
+ * Bytes of workspace varlen_attn_fwd_v4 needs with at most num_splits pieces
+ * per key range (num_splits >= 2) for a non-causal call without a window;
+ * 0 when no split happens (num_splits <= 1, or max_seqlen_k too short to be
+ * cut) or for invalid sizes.  Host only.  Layout (float32): the pieces'
+ * O / l rows [pieces][total_q * num_heads][head_dim], then their lse
+ * [pieces][total_q * num_heads].
+ */
+size_t varlen_attn_fwd_workspace_size(int64_t total_q, int num_heads, int head_dim,
+                                      int max_seqlen_k, int num_splits);
+
 /* Static, human-readable description of a status code.  Never NULL. */
 const char *varlen_attn_strerror(int code);
 
@@ -293,7 +361,7 @@ int varlen_attn_bwd_noalloc(const void *dout, const void *q, const void *k, cons
                             int causal, float scale, varlen_dtype_t dtype,
                             void *dq, void *dk, void *dv, varlen_stream_t stream);
 
-/* Library ABI version: 4 for this header (v2, v3 and the backward added; v1 unchanged). */
+/* Library ABI version: 5 for this header (v2, v3, v4 and the backward added; v1 unchanged). */
 int varlen_attn_abi_version(void);
 
 #ifdef __cplusplus

@@ -21,10 +21,12 @@ O_MAX, O_MEAN, LSE_MAX = 1.5e-2, 2e-3, 5e-3
 GUARD = 3
 
 
-def run_gpu(case, scale=None, guard=GUARD, max_q=None, max_k=None, mask=None, paged=None):
+def run_gpu(case, scale=None, guard=GUARD, max_q=None, max_k=None, mask=None, paged=None,
+            num_splits=None):
     """Runs the CUDA forward with NaN-filled outputs inside guard rows.
     ``paged`` (a workloads.PagedKV) replaces the packed K/V by its page cache,
     page table and key counts (mask's seqused_k, if any, wins).
+    ``num_splits``: key-range pieces (None: the library's choice).
     Returns (out float64 [Tq,H,D], lse float64 [Tq,H], raw out, raw lse)."""
     import flash_attention_fwd_b200 as fa
     mask = mask or {}
@@ -59,7 +61,7 @@ def run_gpu(case, scale=None, guard=GUARD, max_q=None, max_k=None, mask=None, pa
                        scale if scale is not None else case.scale, out=out, lse=lse,
                        window_size_left=mask.get("window_left", -1),
                        window_size_right=mask.get("window_right", -1), seqused_k=used_t,
-                       page_table=table, sinks=sinks_t)
+                       page_table=table, sinks=sinks_t, num_splits=num_splits)
     torch.cuda.synchronize()
     ob, lb = out_buf.cpu(), lse_buf.cpu()
     assert torch.all(ob[:guard] == canary) and torch.all(ob[guard + Tq:] == canary), \

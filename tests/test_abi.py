@@ -28,7 +28,7 @@ def test_library_loads_and_exports_every_symbol():
     raw = ctypes.CDLL(fa.LIB_PATH)
     for name in header_functions():
         assert hasattr(raw, name), name
-    assert lib.varlen_attn_abi_version() == 4
+    assert lib.varlen_attn_abi_version() == 5
 
 
 def test_library_is_built_for_sm100a():
@@ -91,6 +91,11 @@ PAGED = dict(page_table_ptr=0x90000, page_table_stride=2, page_size=16, total_k=
     (dict(PAGED, num_heads=5), -2),
     (dict(sinks_ptr=0x90002), -4),           # sinks need 4-byte alignment
     (dict(sinks_ptr=0x90000, head_dim=48), -2),
+    # the v4 entry point (key-range split): the piece count must be in [0, 32]
+    (dict(num_splits=33, causal=False), -2),
+    (dict(num_splits=-2, causal=False), -2),
+    (dict(num_splits=4, num_heads=5), -2),
+    (dict(num_splits=0, q_ptr=0x10004), -4),
 ])
 def test_host_validation_rejects(change, code):
     args = dict(BASE)
@@ -111,6 +116,48 @@ def test_empty_problems_are_noops_without_device():
     args = dict(BASE)
     args.update(PAGED, total_q=0, q_ptr=0, out_ptr=0, lse_ptr=0)
     assert fa.varlen_attn_fwd_raw(**args) == 0
+
+
+def test_v4_empty_problem_is_a_noop_without_workspace():
+    args = dict(BASE)
+    args.update(batch=0, num_splits=8, causal=False)
+    assert fa.varlen_attn_fwd_raw(**args) == 0
+
+
+def test_split_heuristic_and_workspace_size():
+    # the short-query / long-KV batch (32 sequences, 1267 queries, 145,046
+    # keys, H=32, Hkv=4, D=128) has about 200 work items: no split on 148 SMs
+    shortq = (32, 1267, 145046, 64, 7954, 32, 4, 128)
+    assert fa.fwd_num_splits(*shortq, num_sms=148) == 1
+    # ... but with many more SMs than items, pieces fill them
+    assert fa.fwd_num_splits(*shortq, num_sms=1000) > 1
+    # decode-like: 8 sequences of one query, 8 KV heads (64 items), 32k keys
+    dec = (8, 8, 8 * 32768, 1, 32768, 32, 8, 128)
+    n = fa.fwd_num_splits(*dec, num_sms=148)
+    assert n == 16  # 256 key tiles: 16 pieces of 16
+    # never with a causal rule or a window, never pieces under 16 key tiles
+    assert fa.fwd_num_splits(*dec, causal=True, num_sms=148) == 1
+    assert fa.fwd_num_splits(*dec, window_size_left=100, num_sms=148) == 1
+    assert fa.fwd_num_splits(*dec, window_size_right=0, num_sms=148) == 1
+    assert fa.fwd_num_splits(8, 8, 8 * 2048, 1, 2048, 32, 8, 128, num_sms=148) == 1
+    assert fa.fwd_num_splits(8, 8, 8 * 4096, 1, 4096, 32, 8, 128, num_sms=148) == 2
+    # long prefill: plenty of items, no split
+    assert fa.fwd_num_splits(16, 65536, 65536, 24865, 24865, 64, 8, 128, num_sms=148) == 1
+    # one sequence, one KV head: at most 16 pieces
+    assert fa.fwd_num_splits(1, 1, 1 << 20, 1, 1 << 20, 8, 1, 128, num_sms=148) == 16
+    with pytest.raises(fa.VarlenAttnError):
+        fa.fwd_num_splits(2, 10, 10, 5, 5, 5, 2, 128, num_sms=148)
+    # workspace: pieces x rows x (D + 1) float32; max_seqlen_k = 7954 is 63 key
+    # tiles: 4 pieces of up to 16 tiles
+    assert fa.fwd_workspace_size(1267, 32, 128, 7954, 4) == 4 * 1267 * 32 * 129 * 4
+    # 63 tiles in at most 5 pieces: 13 tiles a piece, 5 pieces
+    assert fa.fwd_workspace_size(1267, 32, 128, 7954, 5) == 5 * 1267 * 32 * 129 * 4
+    # 63 tiles in at most 32 pieces: 2 tiles a piece -> 32 pieces
+    assert fa.fwd_workspace_size(10, 4, 64, 7954, 32) == 32 * 10 * 4 * 65 * 4
+    # no split: one piece asked for, or a key range of one tile
+    assert fa.fwd_workspace_size(1267, 32, 128, 7954, 1) == 0
+    assert fa.fwd_workspace_size(1267, 32, 128, 128, 8) == 0
+    assert fa.fwd_workspace_size(1267, 32, 128, 7954, 33) == 0
 
 
 def test_product_module_does_not_import_oracle():

@@ -18,6 +18,11 @@ five benchmark configurations of the varlen attention forward:
   wide      4 sequences of 4096, H=Hkv=16, D=256, fp16, Q/K ~ N(0, 3^2),
             V ~ N(0, 1), causal
 
+and, beyond them, variants for the window / used-key / paged / sink forms
+and one long-KV decode batch (8 single-query sequences, k_len uniform-int
+[16384, 32768], H=32, Hkv=8: fewer work items than SMs, the case for the
+key-range split).
+
 Length recipe: numpy ``default_rng(seed)`` (PCG64).  Tensor recipe:
 ``torch.Generator('cpu').manual_seed(seed)``, fp32 ``randn`` drawn in the
 order Q [Tq,H,D], K [Tk,Hkv,D], V [Tk,Hkv,D], multiplied by sigma, then cast
@@ -86,6 +91,12 @@ WORKLOADS = {
                           description="GQA prefill lengths with one attention-sink logit per "
                                       "query head (uniform in [-2, 4]), H=32, Hkv=8, D=128, bf16, "
                                       "causal"),
+    # Long-KV decode: one query token per sequence against long ragged key
+    # ranges; 64 work items (one per sequence and KV head) for 148 SMs.
+    "decode": Workload("decode", 6, 32, 8, 128, "bf16", False,
+                       description="long-KV decode: 8 sequences of 1 query token, k_len "
+                                   "uniform-int [16384, 32768], H=32, Hkv=8, D=128, bf16, "
+                                   "non-causal"),
     # Profiling case only (not a benchmark configuration): the long ragged
     # prefill lengths with a quarter of its heads, so that a many-pass profiler
     # capture stays small while its inputs still exceed the L2 cache.
@@ -132,6 +143,10 @@ def seqlens(name: str):
     if name == "wide":
         q = [4096] * 4
         return q, list(q)
+    if name == "decode":
+        rng = np.random.default_rng(w.seed)
+        k = [int(x) for x in rng.integers(16384, 32769, 8)]
+        return [1] * 8, k
     raise KeyError(name)
 
 
