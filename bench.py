@@ -107,6 +107,7 @@ def load_peaks():
 # change a kernel's traffic).
 KERNEL_SOURCES = {
     "fwd": ("sm100_ptx.cuh", "fwd_common.cuh", "fwd_pair.cuh", "fwd_single.cuh"),
+    "combine": ("fwd_common.cuh", "fwd_combine.cuh"),
     "bwd": ("sm100_ptx.cuh", "fwd_common.cuh", "bwd_common.cuh", "bwd_dq.cuh", "bwd_dkdv.cuh"),
 }
 

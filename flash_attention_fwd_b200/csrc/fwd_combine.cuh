@@ -77,15 +77,31 @@ __global__ void __launch_bounds__(NUM_THREADS) combine_kernel(const KParams p) {
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int i = 0; i < P; ++i) {
-      const float wi = __shfl_sync(0xffffffffu, wgt, i) * inv_L;
-      const float *src = p.part_o + ((size_t)i * rows + row) * D + lane * E;
-      if (wi == 0.f) continue;
+    // UNROLL pieces at a time: their loads are all issued before the first
+    // is used, so the latency of the partials is paid once per group
+    constexpr int UNROLL = 4;
+    const float *src0 = p.part_o + (size_t)row * D + lane * E;
+    for (int i0 = 0; i0 < P; i0 += UNROLL) {
+      float2 x[UNROLL][E / 2];
+      float wi[UNROLL];
 #pragma unroll
-      for (int e = 0; e < E; e += 2) {
-        const float2 x = __ldcg(reinterpret_cast<const float2 *>(src + e));
-        acc[e] += wi * x.x;
-        acc[e + 1] += wi * x.y;
+      for (int u = 0; u < UNROLL; ++u) {
+        const int i = i0 + u;
+        wi[u] = __shfl_sync(0xffffffffu, wgt, i & 31) * inv_L;
+        const float *src = src0 + (size_t)i * rows * D;
+#pragma unroll
+        for (int e = 0; e < E; e += 2)
+          x[u][e / 2] = i < P ? __ldcg(reinterpret_cast<const float2 *>(src + e))
+                              : make_float2(0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        if (i0 + u >= P) wi[u] = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+          acc[e] += wi[u] * x[u][e / 2].x;
+          acc[e + 1] += wi[u] * x[u][e / 2].y;
+        }
       }
     }
     uint32_t pk[E / 2];
