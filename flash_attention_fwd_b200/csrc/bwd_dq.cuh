@@ -1,6 +1,6 @@
 /*
  * bwd_dq.cuh — backward, dQ pass: one 128-row query tile (one query head) per
- * work item, streaming the sequence's visible key tiles of BN = 64 keys:
+ * work item, streaming the sequence's visible key tiles of BN = 96 keys:
  *
  *   S(j)  = Q K(j)^T                      tcgen05, into TMEM
  *   dP(j) = dO V(j)^T                     tcgen05, into TMEM
@@ -19,9 +19,12 @@
  * double-buffered S / dP in TMEM — so one computes while the tensor cores
  * serve the other; warp 8 scheduler + TMA producer, warp 9 TMEM owner + MMA
  * issuer.  TMEM:
- * S[2] | dP[2] (BN columns each, double-buffered across key tiles) | dQ (D).
- * The K/V ring holds K(j) and V(j) in turn; V(j) is released after dP(j), K(j)
- * after dQ(j).
+ * S[2] | dP[2] (BN columns each, double-buffered across key tiles) | dQ (D),
+ * 4 * 96 + 128 = 512 columns at D = 128.  (The S and dP products take about
+ * as long per instruction at N = 96 as at N = 64, so the wider tile does half
+ * again as much work per instruction; N = 128 would not fit.)  The row
+ * threads read S and dP in 32-column pieces.  The K/V ring holds K(j) and
+ * V(j) in turn; V(j) is released after dP(j), K(j) after dQ(j).
  */
 #pragma once
 #include "bwd_common.cuh"
@@ -33,8 +36,8 @@ constexpr int NUM_THREADS = 320;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int RING_CONSUMERS = 1 + 8;
-constexpr int BN = 64;
-constexpr int NSLOT = 10;
+constexpr int BN = 96;
+constexpr int NSLOT = 6;
 
 struct Barriers {
   uint64_t full[NSLOT];
@@ -306,23 +309,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         ptx::tc_fence_after();
-        uint32_t sv[BN], dpv[BN];
-        tmem_ld_wait<BN>(tS, sv);
-        tmem_ld_wait<BN>(tDP, dpv);
         const int lim = hi - j * BN;
-        uint32_t pk[BN / 2];
+        // 32 keys at a time: dS of keys [c0, c0 + 32) goes to packed columns
+        // [c0 / 2, c0 / 2 + 16) of S, which were read by an earlier piece
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          float ds[2];
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t sv[32], dpv[32];
+          tmem_ld_wait<32>(tS + c0, sv);
+          tmem_ld_wait<32>(tDP + c0, dpv);
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const float x = __uint_as_float(sv[c + e]) * sl2 - lse2;
-            const float pr = (c + e < lim) ? ptx::ex2_approx(x) : 0.f;
-            ds[e] = pr * (__uint_as_float(dpv[c + e]) - delta);
+          for (int c = 0; c < 32; c += 2) {
+            float ds[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float x = __uint_as_float(sv[c + e]) * sl2 - lse2;
+              const float pr = (c0 + c + e < lim) ? ptx::ex2_approx(x) : 0.f;
+              ds[e] = pr * (__uint_as_float(dpv[c + e]) - delta);
+            }
+            pk[c / 2] = pack2<BF16>(ds[0], ds[1]);
           }
-          pk[c / 2] = pack2<BF16>(ds[0], ds[1]);
+          tmem_st<16>(tS + c0 / 2, pk);
         }
-        tmem_st<BN / 2>(tS, pk);
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
