@@ -149,7 +149,7 @@ __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, i
   const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
   const float negm = exp_offset(m);
   const uint64_t negm_2 = ptx::f2_pack(negm, negm);
-  float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
+  uint64_t sum_ab = ptx::f2_pack(0.f, 0.f), sum_cd = ptx::f2_pack(0.f, 0.f);
 #pragma unroll
   for (int c0 = 0; c0 < BN; c0 += 32) {
     uint32_t pk[16];
@@ -159,15 +159,11 @@ __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, i
       const uint64_t x2 = ptx::f2_fma(ptx::f2_pack(s[c], s[c + 1]), sl2_2, negm_2);
       float x0, x1;
       ptx::f2_unpack(x2, x0, x1);
-      pk[i] = pack2<BF16>(ptx::ex2_approx(x0), ptx::ex2_approx(x1));
-      // the rounded P values (what the PV MMA sees) go into the row sum
-      if (i & 1) {
-        sc = ptx::add_lo16<BF16>(pk[i], sc);
-        sd = ptx::add_hi16<BF16>(pk[i], sd);
-      } else {
-        sa = ptx::add_lo16<BF16>(pk[i], sa);
-        sb = ptx::add_hi16<BF16>(pk[i], sb);
-      }
+      const float e0 = ptx::ex2_approx(x0), e1 = ptx::ex2_approx(x1);
+      pk[i] = pack2<BF16>(e0, e1);
+      // row sum of the unrounded values, two keys per packed add
+      uint64_t &acc = (i & 1) ? sum_cd : sum_ab;
+      acc = ptx::f2_add(acc, ptx::f2_pack(e0, e1));
     }
     ptx::tmem_st_x16(tS + c0 / 2, pk);
     if ((c0 + 32) % CHUNK_KEYS == 0) {
@@ -175,6 +171,9 @@ __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, i
       chunk_ready(c0 / CHUNK_KEYS);
     }
   }
+  float sa, sb, sc, sd;
+  ptx::f2_unpack(sum_ab, sa, sb);
+  ptx::f2_unpack(sum_cd, sc, sd);
   l = l * alpha + ((sa + sb) + (sc + sd));
 }
 
