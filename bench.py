@@ -318,19 +318,21 @@ def run_gpu(args, rank: int, world: int):
         rows_k = k.shape[0] * k.shape[1] if table_t is not None else k.shape[0]
         splits = fa.fwd_num_splits(case.B, case.Tq, rows_k, case.max_q, case.max_k, case.H,
                                    case.Hkv, case.D, paged=table_t is not None, device=dev)
-        nbytes = (fa.fwd_workspace_size(case.Tq, case.H, case.D, case.max_k, splits)
-                  if splits > 1 else 0)
+        nbytes = fa.fwd_workspace_size(case.Tq, case.H, case.Hkv, case.D, case.max_q,
+                                       case.max_k, splits)
         if nbytes:
             ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
         else:
             splits = 1
     args.num_splits = splits
+    args.workspace_bytes = nbytes if ws is not None else 0
 
     def step():
         fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, case.causal, case.scale,
                            out=out, lse=lse, stream=stream, window_size_left=wl,
                            window_size_right=wr, seqused_k=used_t, page_table=table_t,
-                           sinks=sinks_t, num_splits=splits, workspace=ws)
+                           sinks=sinks_t, num_splits=None if ws is not None else 1,
+                           workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -369,7 +371,7 @@ def run_gpu(args, rank: int, world: int):
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
         dist.barrier()
     emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk,
-         launches_per_step=2 if splits > 1 else 1)
+         launches_per_step=2 if ws is not None else 1)
     if dist:
         dist.destroy_process_group()
 
@@ -464,6 +466,7 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
                 "page_size": workloads.WORKLOADS[args.workload].page_size or None,
                 "sinks": "sinks" in case.mask,
                 "num_splits": getattr(args, "num_splits", 1),
+                "workspace_bytes": getattr(args, "workspace_bytes", 0),
                 "l2": "no flush: inputs (%.0f MB) exceed the 126 MB L2"
                       % (algorithmic_bytes(case) / 1e6),
                 "parallelism": "dp%d (one independent batch per GPU)" % world},

@@ -83,7 +83,7 @@ def _bind(lib):
     lib.varlen_attn_fwd_num_splits.argtypes = [i32, i64, i64, i32, i32, i32, i32, i32, i32, i32,
                                                i32, i32, i32]
     lib.varlen_attn_fwd_num_splits.restype = i32
-    lib.varlen_attn_fwd_workspace_size.argtypes = [i64, i32, i32, i32, i32]
+    lib.varlen_attn_fwd_workspace_size.argtypes = [i64, i32, i32, i32, i32, i32, i32]
     lib.varlen_attn_fwd_workspace_size.restype = ctypes.c_size_t
     lib.varlen_attn_strerror.argtypes = [i32]
     lib.varlen_attn_strerror.restype = ctypes.c_char_p
@@ -148,16 +148,17 @@ def varlen_attn_fwd_raw(q_ptr: int, k_ptr: int, v_ptr: int, cu_q_ptr: int, cu_k_
                         workspace_ptr: int = 0, workspace_bytes: int = 0) -> int:
     """Direct call of the C entry point with integer addresses; returns the
     status code unchanged.  Calls varlen_attn_fwd (v1) unless a window bound,
-    a seqused_k array, a page table, sinks or num_splits != 1 are given;
-    varlen_attn_fwd_v2 for a window / seqused_k, varlen_attn_fwd_v3 for a page
-    table or sinks, varlen_attn_fwd_v4 for a key-range split."""
+    a seqused_k array, a page table, sinks, num_splits != 1 or a workspace are
+    given; varlen_attn_fwd_v2 for a window / seqused_k, varlen_attn_fwd_v3 for
+    a page table or sinks, varlen_attn_fwd_v4 for a key-range split or a
+    workspace."""
     lib = load_library()
     V = ctypes.c_void_p
     head = (V(q_ptr), V(k_ptr), V(v_ptr), V(cu_q_ptr), V(cu_k_ptr), int(batch), int(total_q),
             int(total_k), int(max_seqlen_q), int(max_seqlen_k), int(num_heads),
             int(num_kv_heads), int(head_dim), int(bool(causal)), float(scale))
     tail = (int(dtype_code), V(out_ptr), V(lse_ptr), V(stream))
-    if num_splits != 1:
+    if num_splits != 1 or workspace_ptr:
         return lib.varlen_attn_fwd_v4(*head, int(window_left), int(window_right),
                                       V(seqused_k_ptr), V(page_table_ptr),
                                       int(page_table_stride), int(page_size), V(sinks_ptr),
@@ -276,7 +277,7 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         splits = (fwd_num_splits(B, total_q, total_k, max_seqlen_q, max_seqlen_k, H, Hkv, D,
                                  paged=paged, device=q.device)
                   if num_splits is None else int(num_splits))
-        ws_bytes = fwd_workspace_size(total_q, H, D, max_seqlen_k, splits) if splits > 1 else 0
+        ws_bytes = fwd_workspace_size(total_q, H, Hkv, D, max_seqlen_q, max_seqlen_k, splits)
         if ws_bytes == 0:
             splits = 1
         elif workspace is None:
@@ -292,7 +293,7 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             0.0 if scale is None else float(scale), DTYPE_CODES[q.dtype], addr(out), addr(lse),
             stream.cuda_stream, int(window_size_left), int(window_size_right), addr(seqused_k),
             addr(page_table), stride, page_size, addr(sinks), splits,
-            addr(workspace) if splits > 1 else 0, ws_bytes)
+            addr(workspace) if ws_bytes else 0, ws_bytes)
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return out, lse
@@ -322,12 +323,14 @@ def fwd_num_splits(batch: int, total_q: int, total_k: int, max_seqlen_q: int, ma
     return int(rc)
 
 
-def fwd_workspace_size(total_q: int, num_heads: int, head_dim: int, max_seqlen_k: int,
-                       num_splits: int) -> int:
-    """Bytes of device workspace a forward split into at most ``num_splits``
-    pieces needs (0: no split happens)."""
+def fwd_workspace_size(total_q: int, num_heads: int, num_kv_heads: int, head_dim: int,
+                       max_seqlen_q: int, max_seqlen_k: int, num_splits: int) -> int:
+    """Bytes of device workspace a non-causal, windowless forward with at most
+    ``num_splits`` key-range pieces needs (0: none; see
+    varlen_attn_fwd_workspace_size)."""
     return int(load_library().varlen_attn_fwd_workspace_size(
-        int(total_q), int(num_heads), int(head_dim), int(max_seqlen_k), int(num_splits)))
+        int(total_q), int(num_heads), int(num_kv_heads), int(head_dim), int(max_seqlen_q),
+        int(max_seqlen_k), int(num_splits)))
 
 
 def bwd_workspace_size(total_q: int, num_heads: int) -> int:

@@ -18,6 +18,9 @@
  * The sink term (a per-head extra logit in the normalisation) enters once,
  * here, not in the pieces.
  *
+ * With replicated rows (KParams::rep) every key piece of a row comes in rep
+ * copies over interleaved key subsets, each a piece of its own here.
+ *
  * One warp per row (token, head); lane i reads piece i's LSE (at most 32
  * pieces), and lane c holds columns [c * D/32, (c + 1) * D/32) of O.  Rows of
  * sequences that are not split were written by the attention kernel and are
@@ -60,7 +63,9 @@ __global__ void __launch_bounds__(NUM_THREADS) combine_kernel(const KParams p) {
                 ks, lk);
     if (tok < qs || tok >= qs + lq) continue;  // not a row of any sequence
     int P, base, r;
-    kv_pieces((lk + BM - 1) / BM, p.split_tiles, p.max_parts, P, base, r);
+    const int nk = (lk + BM - 1) / BM;
+    kv_pieces(nk, p.split_tiles, p.max_parts, P, base, r);
+    if (nk > 0 && p.rep > 1) P *= p.rep;  // every key piece in rep interleaved copies
     if (P <= 1) continue;  // written whole by the attention kernel
     const float lse_i = lane < P ? __ldcg(p.part_lse + (size_t)lane * rows + row) : -INFINITY;
     float M = lse_i;

@@ -67,6 +67,12 @@ struct KParams {
   // part_lse[i * part_rows + row]; the combine kernel merges the pieces.
   int split_tiles;  // 0: no item is split
   int max_parts;
+  // Replicated rows (pair kernel, GQA-packed, rep = 4; 1 otherwise): an item
+  // holds at most 32 query rows; tile A carries four copies of them, one per
+  // TMEM lane quarter, copy c keeps keys [32c, 32c + 32) of every key tile,
+  // and each copy is a piece of its own for the combine kernel (piece index
+  // part * rep + c).  Tile B is not used.
+  int rep;
   long long part_rows;  // total_q * H
   float *part_o;
   float *part_lse;

@@ -177,7 +177,90 @@ __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, i
   l = l * alpha + ((sa + sb) + (sc + sd));
 }
 
-template <int D, bool BF16>
+// Softmax of one S tile in the replicated-rows form (KParams::rep = 4): the
+// thread holds row copy `copy` (its warp's TMEM lane quarter) and keeps keys
+// [32 copy, 32 copy + 32) of the tile.  It reads those 32 scores, writes their
+// P values to packed columns [16 copy, 16 copy + 16) and zeros to the other 48
+// packed columns of its row, so that the PV product sums, in this row copy,
+// over the copy's keys alone; the running max, sum and O rescale are per copy.
+// Both P pieces are signalled once the row is written.
+template <int D, bool BF16, class ChunkReady>
+__device__ __forceinline__ void softmax_tile_rep(uint32_t tS, uint32_t tO, int copy, int j,
+                                                 float sl2, bool need_mask, int lo, int hi,
+                                                 float &m, float &l, ChunkReady &&chunk_ready) {
+  uint32_t sr[32];
+  tmem_ld_wait<32>(tS + 32 * copy, sr);
+  float s[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(sr[c]);
+  if (need_mask) {
+    const int k0 = 32 * copy;
+#pragma unroll
+    for (int c = 0; c < 32; ++c)
+      if (k0 + c < lo || k0 + c >= hi) s[c] = -INFINITY;
+  }
+  float mx0 = s[0], mx1 = s[1];
+#pragma unroll
+  for (int c = 2; c < 32; c += 4) {
+    mx0 = ptx::fmax3(mx0, s[c], s[c + 1]);
+    mx1 = ptx::fmax3(mx1, s[c + 2], s[c + 3]);
+  }
+  const float mx = fmaxf(mx0, mx1) * sl2;
+  float alpha = 1.f;
+  bool need = false;
+  update_max(j, mx, m, alpha, need);
+  if (__any_sync(0xffffffffu, need)) {
+    const uint64_t a2 = ptx::f2_pack(alpha, alpha);
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += 16) {
+      uint32_t o[16];
+      tmem_ld_wait<16>(tO + c0, o);
+#pragma unroll
+      for (int c = 0; c < 16; c += 2) {
+        float o0, o1;
+        ptx::f2_unpack(
+            ptx::f2_mul(ptx::f2_pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), a2), o0,
+            o1);
+        o[c] = __float_as_uint(o0);
+        o[c + 1] = __float_as_uint(o1);
+      }
+      tmem_st<16>(tO + c0, o);
+    }
+  }
+  const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+  const float negm = exp_offset(m);
+  const uint64_t negm_2 = ptx::f2_pack(negm, negm);
+  uint64_t sum_ab = ptx::f2_pack(0.f, 0.f), sum_cd = ptx::f2_pack(0.f, 0.f);
+  uint32_t pk[16], zr[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint64_t x2 = ptx::f2_fma(ptx::f2_pack(s[2 * i], s[2 * i + 1]), sl2_2, negm_2);
+    float x0, x1;
+    ptx::f2_unpack(x2, x0, x1);
+    const float e0 = ptx::ex2_approx(x0), e1 = ptx::ex2_approx(x1);
+    pk[i] = pack2<BF16>(e0, e1);
+    uint64_t &acc = (i & 1) ? sum_cd : sum_ab;
+    acc = ptx::f2_add(acc, ptx::f2_pack(e0, e1));
+    zr[i] = 0u;
+  }
+  // copy is the same for the whole warp: each branch stores a fixed array
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    if (v == copy)
+      ptx::tmem_st_x16(tS + 16 * v, pk);
+    else
+      ptx::tmem_st_x16(tS + 16 * v, zr);
+  }
+  ptx::tmem_st_wait();
+#pragma unroll
+  for (int c = 0; c < NCHUNK; ++c) chunk_ready(c);
+  float sa, sb, sc, sd;
+  ptx::f2_unpack(sum_ab, sa, sb);
+  ptx::f2_unpack(sum_cd, sc, sd);
+  l = l * alpha + ((sa + sb) + (sc + sd));
+}
+
+template <int D, bool BF16, bool REP>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const KParams p) {
@@ -203,6 +286,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int pack = p.pack_log2;
+  // replicated rows (compiled separately, so the plain kernel keeps its code)
+  constexpr int rep = REP ? 4 : 1;
+  constexpr int NT = REP ? 1 : 2;  // query tiles in use
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSLOT; ++s) {
@@ -263,6 +349,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // tokens of all query heads of kv_h; otherwise tile t = head 2u + t
       auto load_q = [&](const WorkItem &w) -> bool {
         if (!wait_bar(&bars->q_empty, (q_count & 1u) ^ 1u, abort_flag)) return false;
+        if constexpr (REP) {
+          // replicated rows: tile A = four copies of the item's 32 rows
+          ptx::mbar_arrive_expect_tx(&bars->q_full, Q_BYTES);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int db = 0; db < DB; ++db)
+              ptx::tma_load_3d(sQ + db * (BM * 128) + c * (32 * 128), &tm_q, &bars->q_full,
+                               db * 64, w.hu << pack, w.q0);
+          ++q_count;
+          return true;
+        }
         ptx::mbar_arrive_expect_tx(&bars->q_full, 2 * Q_BYTES);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -361,10 +459,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tc_fence_after();
         uint32_t ks;
         if (!(ok = take_slot(ks))) break;
-        issue_s(0, ks, 0, IDESC_S_FULL);
-        ptx::mma_commit(&bars->s_full[0]);
-        issue_s(1, ks, 0, IDESC_S_FULL);
-        ptx::mma_commit(&bars->s_full[1]);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          issue_s(t, ks, 0, IDESC_S_FULL);
+          ptx::mma_commit(&bars->s_full[t]);
+        }
         ptx::mma_commit(&bars->empty[ks]);
         if (n == 1) ptx::mma_commit(&bars->q_empty);
         for (int j = 0; ok && j < n; ++j) {
@@ -372,7 +471,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const bool more = j + 1 < n;
           uint32_t ks_next = 0, vs = 0;
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
+          for (int t = 0; t < NT; ++t) {
             if (S_SPLIT) {
               // upper half of S_t(j+1) while the softmax works on S_t(j)
               if (!(ok = wait_bar(&bars->s_loaded[t], par, abort_flag))) break;
@@ -397,13 +496,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             if (!ok) break;
             if (j == n - 1) ptx::mma_commit(&bars->o_ready[t]);
-            if (t == 1) ptx::mma_commit(&bars->empty[vs]);
+            if (t == NT - 1) ptx::mma_commit(&bars->empty[vs]);
             if (more) {
               // lower half of S_t(j+1): columns 0..63 that P_t(j) occupied
               // (the whole of S_t(j+1) without the split)
               issue_s(t, ks_next, 0, S_SPLIT ? IDESC_S_HALF : IDESC_S_FULL);
               ptx::mma_commit(&bars->s_full[t]);
-              if (t == 1) {
+              if (t == NT - 1) {
                 ptx::mma_commit(&bars->empty[ks_next]);
                 if (j + 1 == n - 1) ptx::mma_commit(&bars->q_empty);
               }
@@ -431,9 +530,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tS = tmem + lane_base + t * BN;
     const uint32_t tO = tmem + lane_base + O_COL0 + t * D;
     const float sl2 = p.scale_log2;
+    // replicated rows: copy = lane quarter, the copy's row = the lane
+    const int copy = warp % 4;
+    const int rr = rep > 1 ? lane : r;
     // row -> (token offset in the item, query head offset)
-    const int tok_off = pack ? t * (BM >> pack) + (r >> pack) : r;
-    const int head_off = pack ? (r & ((1 << pack) - 1)) : t;
+    const int tok_off = pack ? (rep > 1 ? 0 : t * (BM >> pack)) + (rr >> pack) : r;
+    const int head_off = pack ? (rr & ((1 << pack) - 1)) : t;
     uint32_t rs = 0, rph = 0;
     uint32_t g = 0, items = 0;
     bool ok = true;
@@ -453,6 +555,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         rph ^= 1u;
       }
       if (w.hu < 0) break;
+      if (t >= NT) continue;  // tile B is idle with replicated rows
       const int n = w.n_kv;
       const int h = (pack ? (w.hu << pack) : 2 * w.hu) + head_off;
       const int qi = w.qi0 + tok_off;
@@ -460,7 +563,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const size_t orow = (size_t)(w.q0 + tok_off) * p.H + h;
       uint16_t *orow_ptr = reinterpret_cast<uint16_t *>(p.out) + orow * D;
       if (n == 0) {
-        if (row_valid) empty_row<D>(orow_ptr, p.lse + orow, sink_log2(p, h));
+        if (row_valid && (rep == 1 || copy == 0))
+          empty_row<D>(orow_ptr, p.lse + orow, sink_log2(p, h));
         continue;
       }
       // visible keys of this row, relative to the first visited key tile
@@ -475,13 +579,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         ptx::tc_fence_after();
-        softmax_tile_chunked<D, BF16>(
-            tS, tO, j, sl2, j * BN < w.max_lo || (j + 1) * BN > w.min_hi, lo - j * BN,
-            hi - j * BN, m, l,
-            [&]() {
-              if (S_SPLIT) arrive(&bars->s_loaded[t]);
-            },
-            [&](int c) { arrive(&bars->p_chunk[t][c]); });
+        const bool need_mask = j * BN < w.max_lo || (j + 1) * BN > w.min_hi;
+        if constexpr (REP)
+          softmax_tile_rep<D, BF16>(tS, tO, copy, j, sl2, need_mask, lo - j * BN, hi - j * BN, m,
+                                    l, [&](int c) { arrive(&bars->p_chunk[t][c]); });
+        else
+          softmax_tile_chunked<D, BF16>(
+              tS, tO, j, sl2, need_mask, lo - j * BN, hi - j * BN, m, l,
+              [&]() {
+                if (S_SPLIT) arrive(&bars->s_loaded[t]);
+              },
+              [&](int c) { arrive(&bars->p_chunk[t][c]); });
       }
       if (!ok) break;
       g += n;
@@ -492,12 +600,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
-      if (w.part < 0)
+      if (w.part < 0 && rep == 1) {
         epilogue_row<D, BF16>(tO, m, l, sink_log2(p, h), row_valid, orow_ptr, p.lse + orow,
                               &bars->o_free[t], lane);
-      else
-        epilogue_part<D>(tO, m, l, row_valid, p.part_o + ((size_t)w.part * p.part_rows + orow) * D,
-                         p.part_lse + (size_t)w.part * p.part_rows + orow, &bars->o_free[t], lane);
+      } else {
+        // a piece of the row: the key-range piece, and with replicated rows
+        // the copy within it
+        const size_t piece = (size_t)(w.part < 0 ? 0 : w.part) * rep + (rep > 1 ? copy : 0);
+        epilogue_part<D>(tO, m, l, row_valid, p.part_o + (piece * p.part_rows + orow) * D,
+                         p.part_lse + piece * p.part_rows + orow, &bars->o_free[t], lane);
+      }
     }
     end_of_kernel();
   }

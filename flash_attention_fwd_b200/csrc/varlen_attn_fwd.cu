@@ -125,8 +125,13 @@ static int launch_pair(const CUtensorMap &tq, const CUtensorMap &tk, const CUten
                        const KParams &kp, int grid, cudaStream_t s, DeviceInfo &dev, int slot) {
   constexpr size_t smem = pair::smem_bytes<D>();
   static_assert(smem <= 232448, "shared memory budget");
-  return launch_kernel(pair::fwd_kernel<D, BF16>, smem, pair::NUM_THREADS, tq, tk, tv, kp, grid,
-                       s, dev.attr_set[slot], (int)pair::REG_LAUNCH);
+  // replicated rows: its own instantiation, attribute slots 18..21 (the
+  // forward uses 0..9, the backward 10..17)
+  if (kp.rep > 1)
+    return launch_kernel(pair::fwd_kernel<D, BF16, true>, smem, pair::NUM_THREADS, tq, tk, tv, kp,
+                         grid, s, dev.attr_set[slot + 18], (int)pair::REG_LAUNCH);
+  return launch_kernel(pair::fwd_kernel<D, BF16, false>, smem, pair::NUM_THREADS, tq, tk, tv, kp,
+                       grid, s, dev.attr_set[slot], (int)pair::REG_LAUNCH);
 }
 
 static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -145,8 +150,10 @@ struct FwdLayout {
   int pack_log2;    // GQA packing (see KParams::pack_log2)
   int head_units;   // head units per (sequence, token range)
   int unit_tokens;  // query tokens per work item
+  int rep;          // replicated rows (see KParams::rep): 4, or 1
 };
-static FwdLayout fwd_layout(int max_seqlen_q, int num_heads, int num_kv_heads, int D) {
+static FwdLayout fwd_layout(int max_seqlen_q, int num_heads, int num_kv_heads, int D,
+                            bool rep = false) {
   FwdLayout L;
   const int group = num_heads / num_kv_heads;
   // Query-head pairs share a key/value head when the group size is even;
@@ -164,7 +171,23 @@ static FwdLayout fwd_layout(int max_seqlen_q, int num_heads, int num_kv_heads, i
   }
   L.head_units = L.pack_log2 ? num_kv_heads : (L.use_pair ? num_heads / 2 : num_heads);
   L.unit_tokens = L.pack_log2 ? 2 * (BM >> L.pack_log2) : BM;
+  L.rep = 1;
+  if (rep && L.pack_log2 > 0) {  // replicated rows: 32 rows (32 >> pack tokens) per item
+    L.rep = 4;
+    L.unit_tokens = 32 >> L.pack_log2;
+  }
   return L;
+}
+
+// The replicated-rows form (KParams::rep) applies to GQA-packed calls whose
+// items have at most 32 query rows (max_seqlen_q x H / Hkv <= 32) and whose
+// key ranges reach 8 tiles, so that the merge launch pays; without a causal
+// rule or a window, and only when the caller gives a workspace.
+static bool rep_eligible(int max_seqlen_q, int max_seqlen_k, int num_heads, int num_kv_heads,
+                         int D) {
+  const FwdLayout L = fwd_layout(max_seqlen_q, num_heads, num_kv_heads, D);
+  return L.pack_log2 > 0 && L.pack_log2 <= 5 && ((long long)max_seqlen_q << L.pack_log2) <= 32 &&
+         max_seqlen_k >= 8 * BM;
 }
 
 // Key tiles per piece and the largest piece count when a call asks for at
@@ -194,11 +217,11 @@ static void split_plan(int num_splits, int max_seqlen_k, bool masked, int &split
 // short-query / long-KV batch), every split slower than none.
 static int auto_num_splits(int batch, int64_t total_q, int64_t total_k, int max_seqlen_q,
                            int max_seqlen_k, int num_heads, int num_kv_heads, int D, bool masked,
-                           bool paged, int sms) {
+                           bool paged, int sms, bool rep) {
   (void)total_k;
   (void)paged;
   if (masked || batch <= 0 || max_seqlen_k <= 0 || max_seqlen_q <= 0 || sms <= 0) return 1;
-  const FwdLayout L = fwd_layout(max_seqlen_q, num_heads, num_kv_heads, D);
+  const FwdLayout L = fwd_layout(max_seqlen_q, num_heads, num_kv_heads, D, rep);
   const double nk_max = ceil((double)max_seqlen_k / BM);
   const double q_mean = fmin((double)total_q / batch, (double)max_seqlen_q);
   const double items = (double)batch * fmax(1.0, ceil(q_mean / L.unit_tokens)) * L.head_units;
@@ -288,15 +311,28 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   const bool bf16 = dtype == VARLEN_BF16;
   const int D = head_dim;
   const int group = num_heads / num_kv_heads;
-  const FwdLayout layout = fwd_layout(max_seqlen_q, num_heads, num_kv_heads, D);
+  // Window bounds in canonical form: a bound that no query of the buffers can
+  // reach is dropped (this also keeps qi - left and qi + right + 1 in range),
+  // and the causal rule is the right bound 0.
+  // (a sequence has at most total_k keys, or page_table_stride pages of keys when paged: pages
+  // may be shared, so a paged sequence can hold more keys than the cache has rows)
+  const int64_t key_extent = paged ? (int64_t)page_table_stride * page_size : total_k;
+  int win_left = (window_left >= 0 && (int64_t)window_left < total_q) ? window_left : -1;
+  int win_right = (window_right >= 0 && (int64_t)window_right < key_extent) ? window_right : -1;
+  if (causal) win_right = 0;
+  const bool masked = win_left >= 0 || win_right >= 0;
+  const bool rep = !masked && workspace != nullptr &&
+                   rep_eligible(max_seqlen_q, max_seqlen_k, num_heads, num_kv_heads, D);
+  const FwdLayout layout = fwd_layout(max_seqlen_q, num_heads, num_kv_heads, D, rep);
   const bool use_pair = layout.use_pair;
   const int pack_log2 = layout.pack_log2;
   const int BN = use_pair ? pair::BN : (D == 256 ? single::Cfg<256>::BN : single::Cfg<128>::BN);
   alignas(64) CUtensorMap tq, tk, tv;
   memset(&tk, 0, sizeof tk);
   memset(&tv, 0, sizeof tv);
-  if (!encode_qkv_map(enc, &tq, q, bf16, total_q, num_heads, D, BM >> pack_log2,
-                      1 << pack_log2))
+  // a query box is one tile of 128 rows, or one copy of 32 rows with replicated rows
+  if (!encode_qkv_map(enc, &tq, q, bf16, total_q, num_heads, D,
+                      (layout.rep > 1 ? 32 : BM) >> pack_log2, 1 << pack_log2))
     return VARLEN_ERR_LAUNCH;
   // paged: a key tile is fetched as boxes of `chunk` rows, which divide both
   // the page and the tile, so that no box crosses a page
@@ -325,37 +361,32 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   const float sc = (scale > 0.f) ? scale : 1.0f / sqrtf((float)D);  // NaN fails "> 0"
   kp.scale_log2 = sc * 1.4426950408889634f;
   kp.seqused_k = seqused_k;
-  // Window bounds in canonical form: a bound that no query of the buffers can
-  // reach is dropped (this also keeps qi - left and qi + right + 1 in range),
-  // and the causal rule is the right bound 0.
-  // (a sequence has at most total_k keys, or page_table_stride pages of keys when paged: pages
-  // may be shared, so a paged sequence can hold more keys than the cache has rows)
-  const int64_t key_extent = paged ? (int64_t)page_table_stride * page_size : total_k;
-  kp.win_left = (window_left >= 0 && (int64_t)window_left < total_q) ? window_left : -1;
-  kp.win_right = (window_right >= 0 && (int64_t)window_right < key_extent) ? window_right : -1;
-  if (causal) kp.win_right = 0;
+  kp.win_left = win_left;
+  kp.win_right = win_right;
   kp.page_table = page_table;
   kp.pt_stride = paged ? page_table_stride : 0;
   kp.page_size = paged ? page_size : 0;
   kp.num_pages = paged ? (int)(total_k / page_size) : 0;
   kp.page_chunk = chunk;
   kp.sinks = sinks;
-  // Key-range split (non-causal, windowless calls): pieces merged by the
-  // combine kernel through the caller's workspace.
-  const bool masked = kp.win_left >= 0 || kp.win_right >= 0;
+  // Key-range split (non-causal, windowless calls) and replicated rows:
+  // pieces merged by the combine kernel through the caller's workspace.
+  kp.rep = layout.rep;
   if (num_splits == 0)
     num_splits = auto_num_splits(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads,
-                                 num_kv_heads, D, masked, paged, dev.sms);
+                                 num_kv_heads, D, masked, paged, dev.sms, rep);
+  if (num_splits > combine::MAX_PARTS / kp.rep) num_splits = combine::MAX_PARTS / kp.rep;
   split_plan(num_splits, max_seqlen_k, masked, kp.split_tiles, kp.max_parts);
   kp.part_rows = (long long)total_q * num_heads;
   kp.part_o = nullptr;
   kp.part_lse = nullptr;
-  if (kp.split_tiles > 0) {
-    const size_t need = split_workspace_bytes(total_q, num_heads, D, kp.max_parts);
+  if (kp.split_tiles > 0 || kp.rep > 1) {
+    const int slots = kp.max_parts * kp.rep;
+    const size_t need = split_workspace_bytes(total_q, num_heads, D, slots);
     if (!workspace || !aligned(workspace, 16) || workspace_bytes < need)
       return VARLEN_ERR_WORKSPACE;
     kp.part_o = static_cast<float *>(workspace);
-    kp.part_lse = kp.part_o + (size_t)kp.max_parts * (size_t)kp.part_rows * D;
+    kp.part_lse = kp.part_o + (size_t)slots * (size_t)kp.part_rows * D;
   }
 
   // Upper bound of work items from max_seqlen_q; at least one CTA so that an
@@ -391,7 +422,7 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
                   : launch_single<256, false>(tq, tk, tv, kp, grid, s, dev, 9);
     }
   }
-  if (rc != VARLEN_OK || kp.split_tiles == 0) return rc;
+  if (rc != VARLEN_OK || (kp.split_tiles == 0 && kp.rep == 1)) return rc;
   switch (D) {
     case 64:
       return bf16 ? launch_combine<64, true>(kp, dev.sms, s) : launch_combine<64, false>(kp, dev.sms, s);
@@ -474,17 +505,28 @@ extern "C" int varlen_attn_fwd_num_splits(int batch, int64_t total_q, int64_t to
     num_sms = dev->sms;
   }
   const bool masked = causal || window_left >= 0 || window_right >= 0;
-  return auto_num_splits(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads,
-                         num_kv_heads, head_dim, masked, paged != 0, num_sms);
+  const bool rep =
+      !masked && rep_eligible(max_seqlen_q, max_seqlen_k, num_heads, num_kv_heads, head_dim);
+  const int n = auto_num_splits(batch, total_q, total_k, max_seqlen_q, max_seqlen_k, num_heads,
+                                num_kv_heads, head_dim, masked, paged != 0, num_sms, rep);
+  return rep && n > combine::MAX_PARTS / 4 ? combine::MAX_PARTS / 4 : n;
 }
 
-extern "C" size_t varlen_attn_fwd_workspace_size(int64_t total_q, int num_heads, int head_dim,
+extern "C" size_t varlen_attn_fwd_workspace_size(int64_t total_q, int num_heads,
+                                                 int num_kv_heads, int head_dim, int max_seqlen_q,
                                                  int max_seqlen_k, int num_splits) {
-  if (total_q <= 0 || num_heads <= 0 || head_dim <= 0 || num_splits > combine::MAX_PARTS)
+  if (total_q <= 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 ||
+      (head_dim != 64 && head_dim != 128 && head_dim != 256) || max_seqlen_q < 0 ||
+      num_splits < 1 || num_splits > combine::MAX_PARTS)
     return 0;
+  const int rep =
+      rep_eligible(max_seqlen_q, max_seqlen_k, num_heads, num_kv_heads, head_dim) ? 4 : 1;
+  if (num_splits > combine::MAX_PARTS / rep) num_splits = combine::MAX_PARTS / rep;
   int split_tiles, max_parts;
   split_plan(num_splits, max_seqlen_k, false, split_tiles, max_parts);
-  return split_tiles > 0 ? split_workspace_bytes(total_q, num_heads, head_dim, max_parts) : 0;
+  return (split_tiles > 0 || rep > 1)
+             ? split_workspace_bytes(total_q, num_heads, head_dim, max_parts * rep)
+             : 0;
 }
 
 extern "C" int varlen_attn_fwd(const void *q, const void *k, const void *v,

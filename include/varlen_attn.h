@@ -219,23 +219,33 @@ int varlen_attn_fwd_v3(const void *q, const void *k, const void *v,
  * over all SMs instead of leaving a few long work items to a few of them.
  *
  *   num_splits   0: the library chooses (varlen_attn_fwd_num_splits); 1: no
- *                split (exactly v3); 2..32: at most that many pieces per key
+ *                key-range split (with a NULL workspace exactly v3); 2..32: at
+ *                most that many pieces per key
  *                range: pieces hold up to S = ceil(ceil(max_seqlen_k / 128) /
  *                num_splits) tiles of 128 keys, and a sequence of at most S
  *                tiles is not cut.  Ignored (no split) with causal or a window.
  *                Outside [0, 32]: VARLEN_ERR_SHAPE.
  *   workspace, workspace_bytes   device buffer (16-byte aligned) of at least
- *                varlen_attn_fwd_workspace_size(total_q, num_heads, head_dim,
- *                max_seqlen_k, n) bytes, n the piece count in force (for
- *                num_splits = 0: the value varlen_attn_fwd_num_splits returns
- *                for the same arguments).  Used only when a split happens
- *                (NULL is fine otherwise); contents on entry do not matter
- *                and are scratch afterwards.  Missing, misaligned or too
- *                small when needed: VARLEN_ERR_WORKSPACE, nothing launched.
+ *                varlen_attn_fwd_workspace_size(total_q, num_heads,
+ *                num_kv_heads, head_dim, max_seqlen_q, max_seqlen_k, n)
+ *                bytes, n the piece count in force (for num_splits = 0: the
+ *                value varlen_attn_fwd_num_splits returns for the same
+ *                arguments), or NULL (no split then needs none, and rows are
+ *                not replicated).  Contents on entry do not matter and are
+ *                scratch afterwards.  Missing, misaligned or too small when
+ *                needed: VARLEN_ERR_WORKSPACE, nothing launched.
  *
- * With a split, two kernels run on `stream` in order (attention, then the
- * merge); the workspace must stay allocated until both have finished.
- * Everything else is as in v3.
+ * Replicated rows: when a workspace is given, the call is non-causal without
+ * a window, H / Hkv is a power of two of at least 2, every sequence's query
+ * rows fit in 32 (max_seqlen_q * H / Hkv <= 32: decode-like calls) and
+ * max_seqlen_k >= 1024, the library also computes each row as four pieces
+ * over interleaved key subsets (a quarter of the exponentials per thread),
+ * merged the same way; then at most 8 key-range pieces are used.
+ * varlen_attn_fwd_workspace_size accounts for both.
+ *
+ * With a split or replicated rows, two kernels run on `stream` in order
+ * (attention, then the merge); the workspace must stay allocated until both
+ * have finished.  Everything else is as in v3.
  */
 int varlen_attn_fwd_v4(const void *q, const void *k, const void *v,
                        const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
@@ -261,15 +271,16 @@ int varlen_attn_fwd_num_splits(int batch, int64_t total_q, int64_t total_k,
                                int window_left, int window_right, int paged, int num_sms);
 
 /*
- * Bytes of workspace varlen_attn_fwd_v4 needs with at most num_splits pieces
- * per key range (num_splits >= 2) for a non-causal call without a window;
- * 0 when no split happens (num_splits <= 1, or max_seqlen_k too short to be
- * cut) or for invalid sizes.  Host only.  Layout (float32): the pieces'
- * O / l rows [pieces][total_q * num_heads][head_dim], then their lse
+ * Bytes of workspace varlen_attn_fwd_v4 needs for a non-causal call without a
+ * window with these sizes and at most num_splits (>= 1) pieces per key range;
+ * 0 when it needs none (no split and no replicated rows, see below) or for
+ * invalid sizes.  Host only.  Layout (float32): the pieces' O / l rows
+ * [pieces][total_q * num_heads][head_dim], then their lse
  * [pieces][total_q * num_heads].
  */
-size_t varlen_attn_fwd_workspace_size(int64_t total_q, int num_heads, int head_dim,
-                                      int max_seqlen_k, int num_splits);
+size_t varlen_attn_fwd_workspace_size(int64_t total_q, int num_heads, int num_kv_heads,
+                                      int head_dim, int max_seqlen_q, int max_seqlen_k,
+                                      int num_splits);
 
 /* Static, human-readable description of a status code.  Never NULL. */
 const char *varlen_attn_strerror(int code);

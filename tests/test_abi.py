@@ -134,7 +134,10 @@ def test_split_heuristic_and_workspace_size():
     # decode-like: 8 sequences of one query, 8 KV heads (64 items), 32k keys
     dec = (8, 8, 8 * 32768, 1, 32768, 32, 8, 128)
     n = fa.fwd_num_splits(*dec, num_sms=148)
-    assert n == 16  # 256 key tiles: 16 pieces of 16
+    assert n == 8  # 256 key tiles: 16 pieces of 16, capped at 8 with replicated rows
+    # without replicated rows (8 query heads per KV head -> 8 rows, but
+    # max_seqlen_q = 5 -> 40 rows > 32): 16
+    assert fa.fwd_num_splits(8, 40, 8 * 32768, 5, 32768, 64, 8, 128, num_sms=148) == 16
     # never with a causal rule or a window, never pieces under 16 key tiles
     assert fa.fwd_num_splits(*dec, causal=True, num_sms=148) == 1
     assert fa.fwd_num_splits(*dec, window_size_left=100, num_sms=148) == 1
@@ -143,21 +146,33 @@ def test_split_heuristic_and_workspace_size():
     assert fa.fwd_num_splits(8, 8, 8 * 4096, 1, 4096, 32, 8, 128, num_sms=148) == 2
     # long prefill: plenty of items, no split
     assert fa.fwd_num_splits(16, 65536, 65536, 24865, 24865, 64, 8, 128, num_sms=148) == 1
-    # one sequence, one KV head: at most 16 pieces
-    assert fa.fwd_num_splits(1, 1, 1 << 20, 1, 1 << 20, 8, 1, 128, num_sms=148) == 16
+    # one sequence, one KV head (8 rows, replicated): at most 8 pieces
+    assert fa.fwd_num_splits(1, 1, 1 << 20, 1, 1 << 20, 8, 1, 128, num_sms=148) == 8
     with pytest.raises(fa.VarlenAttnError):
         fa.fwd_num_splits(2, 10, 10, 5, 5, 5, 2, 128, num_sms=148)
     # workspace: pieces x rows x (D + 1) float32; max_seqlen_k = 7954 is 63 key
-    # tiles: 4 pieces of up to 16 tiles
-    assert fa.fwd_workspace_size(1267, 32, 128, 7954, 4) == 4 * 1267 * 32 * 129 * 4
+    # tiles: 4 pieces of up to 16 tiles (H/Hkv = 8, max_seqlen_q = 64: 512
+    # rows per item, no replicated rows)
+    assert fa.fwd_workspace_size(1267, 32, 4, 128, 64, 7954, 4) == 4 * 1267 * 32 * 129 * 4
     # 63 tiles in at most 5 pieces: 13 tiles a piece, 5 pieces
-    assert fa.fwd_workspace_size(1267, 32, 128, 7954, 5) == 5 * 1267 * 32 * 129 * 4
-    # 63 tiles in at most 32 pieces: 2 tiles a piece -> 32 pieces
-    assert fa.fwd_workspace_size(10, 4, 64, 7954, 32) == 32 * 10 * 4 * 65 * 4
-    # no split: one piece asked for, or a key range of one tile
-    assert fa.fwd_workspace_size(1267, 32, 128, 7954, 1) == 0
-    assert fa.fwd_workspace_size(1267, 32, 128, 128, 8) == 0
-    assert fa.fwd_workspace_size(1267, 32, 128, 7954, 33) == 0
+    assert fa.fwd_workspace_size(1267, 32, 4, 128, 64, 7954, 5) == 5 * 1267 * 32 * 129 * 4
+    # 63 tiles in at most 32 pieces: 2 tiles a piece -> 32 pieces (D = 64, no GQA packing)
+    assert fa.fwd_workspace_size(10, 4, 4, 64, 5, 7954, 32) == 32 * 10 * 4 * 65 * 4
+    # no split and no replicated rows: nothing
+    assert fa.fwd_workspace_size(1267, 32, 4, 128, 64, 7954, 1) == 0
+    assert fa.fwd_workspace_size(1267, 32, 4, 128, 64, 128, 8) == 0
+    assert fa.fwd_workspace_size(1267, 32, 4, 128, 64, 7954, 33) == 0
+    assert fa.fwd_workspace_size(1267, 32, 4, 128, 64, 7954, 0) == 0
+    # replicated rows (1 query x 4 heads per KV head, keys >= 1024): 4 copies of
+    # each key piece, at most 8 key pieces
+    assert fa.fwd_workspace_size(8, 32, 8, 128, 1, 4096, 1) == 4 * 8 * 32 * 129 * 4
+    assert fa.fwd_workspace_size(8, 32, 8, 128, 1, 4096, 2) == 8 * 8 * 32 * 129 * 4
+    assert fa.fwd_workspace_size(8, 32, 8, 128, 1, 32768, 16) == 32 * 8 * 32 * 129 * 4
+    # ... not for 8 query tokens x 8 heads (64 rows), nor for short key ranges
+    assert fa.fwd_workspace_size(64, 32, 4, 128, 8, 4096, 1) == 0
+    assert fa.fwd_workspace_size(8, 32, 8, 128, 1, 1000, 1) == 0
+    # the auto piece count with replicated rows stays within 8
+    assert fa.fwd_num_splits(8, 8, 8 * 32768, 1, 32768, 32, 8, 128, num_sms=148) <= 8
 
 
 def test_product_module_does_not_import_oracle():

@@ -167,7 +167,7 @@ def test_split_auto_choice_decode_batch():
 def test_split_workspace_errors():
     import flash_attention_fwd_b200 as fa
     case = workloads.make_case(LQ, LK, 16, 2, 128, "bf16", False, seed=1120)
-    need = fa.fwd_workspace_size(case.q.shape[0], 16, 128, case.max_k, 4)
+    need = fa.fwd_workspace_size(case.q.shape[0], 16, 2, 128, case.max_q, case.max_k, 4)
     assert need > 0
     dev = torch.device("cuda", 0)
     args = (case.q.to(dev), case.k.to(dev), case.v.to(dev), case.cu_q.to(dev),
@@ -189,3 +189,81 @@ def test_split_workspace_errors():
             **base)
         assert rc == -8
     torch.cuda.synchronize()
+
+
+# ---- replicated rows: decode-like calls (at most 32 query rows per KV head)
+# The pair kernel puts four copies of an item's <= 32 rows in the four TMEM
+# lane quarters and gives copy c keys [32c, 32c + 32) of every key tile; the
+# copies are merged like key-range pieces.  Eligible: non-causal, no window,
+# H/Hkv a power of two >= 2, max_seqlen_q * H/Hkv <= 32, max_seqlen_k >= 1024,
+# and a workspace (the binding passes one unless num_splits=1).
+
+DEC_LK = [5000, 1025, 0, 3000, 17, 2048, 1999, 40]
+
+
+@pytest.mark.parametrize("H,Hkv,max_q", [(4, 2, 16), (32, 8, 8), (16, 2, 4), (32, 2, 2),
+                                         (32, 1, 1)])
+def test_rep_group_sizes(H, Hkv, max_q):
+    gen = np.random.default_rng(1200 + H + Hkv)
+    lq = [int(x) for x in gen.integers(1, max_q + 1, len(DEC_LK))]
+    lq[1] = max_q
+    case = workloads.make_case(lq, DEC_LK, H, Hkv, 128, "bf16", False, seed=1201 + H)
+    full_check(case)
+
+
+@pytest.mark.parametrize("splits", [None, 2, 3, 8, 32])
+@pytest.mark.parametrize("D,dtype", [(128, "bf16"), (64, "fp16"), (128, "fp16")])
+def test_rep_with_key_pieces(D, dtype, splits):
+    lq = [1, 2, 1, 4, 3, 1, 2, 1]
+    case = workloads.make_case(lq, DEC_LK, 32, 8, D, dtype, False, seed=1210 + D)
+    full_check(case, num_splits=splits)
+
+
+def test_rep_empty_query_and_key_sequences():
+    lq = [1, 0, 2, 1, 0, 3]
+    lk = [0, 3000, 1500, 0, 0, 2000]
+    case = workloads.make_case(lq, lk, 32, 8, 128, "bf16", False, seed=1220)
+    out, lse = full_check(case)
+    cu = case.cu_q.tolist()
+    assert np.all(out[cu[0]:cu[1]] == 0.0) and np.all(np.isneginf(lse[cu[0]:cu[1]]))
+
+
+def test_rep_with_sinks_and_seqused_k():
+    lq = [1, 2, 1, 4, 3, 1, 2, 1]
+    case = workloads.make_case(lq, DEC_LK, 32, 8, 128, "bf16", False, seed=1230)
+    sinks = np.random.default_rng(1231).uniform(-2.0, 4.0, 32).astype(np.float32).tolist()
+    used = [4000, 1025, 0, 1, 17, 1100, 33, 40]
+    full_check(case, mask=dict(sinks=sinks, seqused_k=used))
+
+
+@pytest.mark.parametrize("page_size", [16, 64])
+def test_rep_paged(page_size):
+    lq = [1, 2, 1, 4, 3, 1, 2, 1]
+    case = workloads.make_case(lq, DEC_LK, 32, 8, 128, "bf16", False, seed=1240 + page_size)
+    paged = workloads.to_paged(case, page_size, seed=1241)
+    full_check(case, paged=paged, num_splits=4)
+
+
+def test_rep_understated_max_seqlen_k():
+    lq = [1, 2, 1, 4, 3, 1, 2, 1]
+    case = workloads.make_case(lq, DEC_LK, 32, 8, 128, "bf16", False, seed=1250)
+    full_check(case, max_k=1024, num_splits=2)
+
+
+def test_rep_equals_plain_path_up_to_rounding():
+    lq = [1, 2, 1, 4, 3, 1, 2, 1]
+    case = workloads.make_case(lq, DEC_LK, 32, 8, 128, "fp16", False, seed=1260)
+    o1, l1, _, _ = run_gpu(case, num_splits=1)      # no workspace: the plain kernel path
+    o2, l2, _, _ = run_gpu(case, num_splits=None)   # replicated rows (+ key pieces)
+    fin = np.isfinite(l1)
+    assert np.array_equal(fin, np.isfinite(l2))
+    assert np.abs(o1 - o2).max() <= 4e-3
+    assert np.abs(l1[fin] - l2[fin]).max() <= 1e-4
+
+
+def test_rep_deterministic():
+    lq = [1, 2, 1, 4, 3, 1, 2, 1]
+    case = workloads.make_case(lq, DEC_LK, 32, 8, 128, "bf16", False, seed=1270)
+    _, _, a_o, a_l = run_gpu(case)
+    _, _, b_o, b_l = run_gpu(case)
+    assert torch.equal(a_o, b_o) and torch.equal(a_l, b_l)
