@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(NUM_THREADS) combine_kernel(const KParams p) {
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
     // UNROLL pieces at a time: their loads are all issued before the first
     // is used, so the latency of the partials is paid once per group
-    constexpr int UNROLL = 4;
+    constexpr int UNROLL = E <= 4 ? 8 : 4;
     const float *src0 = p.part_o + (size_t)row * D + lane * E;
     for (int i0 = 0; i0 < P; i0 += UNROLL) {
       float2 x[UNROLL][E / 2];

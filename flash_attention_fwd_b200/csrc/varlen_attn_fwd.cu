@@ -211,7 +211,8 @@ static void split_plan(int num_splits, int max_seqlen_k, bool masked, int &split
 // the work items alone cannot fill the GPU (fewer than 3/4 as many items as
 // SMs): then each key range is cut into up to 16 pieces of at least 16 key
 // tiles, so that the pieces of the few long items spread over all SMs in
-// several rounds that the cost-ordered dealing evens out.  Measured on B200:
+// several rounds that the cost-ordered dealing evens out (replicated-row
+// calls: see below).  Measured on B200:
 // 8 single-query sequences x 8 KV heads x 32k keys, 0.61 ms unsplit, 0.27 ms
 // in 16 pieces; 208 short-query items over up to 63 key tiles (the
 // short-query / long-KV batch), every split slower than none.
@@ -225,6 +226,17 @@ static int auto_num_splits(int batch, int64_t total_q, int64_t total_k, int max_
   const double nk_max = ceil((double)max_seqlen_k / BM);
   const double q_mean = fmin((double)total_q / batch, (double)max_seqlen_q);
   const double items = (double)batch * fmax(1.0, ceil(q_mean / L.unit_tokens)) * L.head_units;
+  if (rep) {
+    // replicated rows: items are short and the merge is cheap (few rows), so
+    // pieces of about 32 key tiles even out ragged key ranges unless there are
+    // plenty of items (measured: 64 ragged 1k-16k sequences, 512 items,
+    // 0.441 ms in one piece, 0.397 ms in 4)
+    // (pieces of 16 tiles when the items alone leave SMs idle)
+    if (items >= 4.0 * sms) return 1;
+    const double tiles = items < 0.75 * sms ? 16.0 : 32.0;
+    const double ns = fmin((double)(combine::MAX_PARTS / 4), floor(nk_max / tiles));
+    return ns < 2.0 ? 1 : (int)ns;
+  }
   if (items >= 0.75 * sms) return 1;
   const double ns = fmin(16.0, floor(nk_max / 16.0));
   return ns < 2.0 ? 1 : (ns > combine::MAX_PARTS ? combine::MAX_PARTS : (int)ns);

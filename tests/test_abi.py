@@ -171,8 +171,11 @@ def test_split_heuristic_and_workspace_size():
     # ... not for 8 query tokens x 8 heads (64 rows), nor for short key ranges
     assert fa.fwd_workspace_size(64, 32, 4, 128, 8, 4096, 1) == 0
     assert fa.fwd_workspace_size(8, 32, 8, 128, 1, 1000, 1) == 0
-    # the auto piece count with replicated rows stays within 8
-    assert fa.fwd_num_splits(8, 8, 8 * 32768, 1, 32768, 32, 8, 128, num_sms=148) <= 8
+    # the auto piece count with replicated rows: about 32 key tiles a piece, at
+    # most 8 pieces, none with plenty of items
+    assert fa.fwd_num_splits(8, 8, 8 * 32768, 1, 32768, 32, 8, 128, num_sms=148) == 8
+    assert fa.fwd_num_splits(64, 64, 64 * 8000, 1, 16384, 32, 8, 128, num_sms=148) == 4
+    assert fa.fwd_num_splits(512, 512, 512 * 8000, 1, 16384, 32, 8, 128, num_sms=148) == 1
 
 
 def test_product_module_does_not_import_oracle():
