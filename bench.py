@@ -107,6 +107,9 @@ def timed_steps(step, steps, stream, dev, flush: bool):
     # one untimed step first: the GPU has idled while the clock sampler started
     step()
     torch.cuda.synchronize()
+    # keep the GPU busy for about a millisecond while the host queues the first
+    # steps, so that no step waits for the host between its events
+    torch.cuda._sleep(2_000_000)
     for i in range(steps):
         if buf is not None:
             buf.zero_()
@@ -368,12 +371,17 @@ def run_gpu(args, rank: int, world: int):
     args.num_splits = splits
     args.workspace_bytes = nbytes if ws is not None else 0
 
-    def step():
+    def step_on(q, k, v, cq, ck, used_t, table_t, sinks_t, out, lse):
         fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, case.causal, case.scale,
                            out=out, lse=lse, stream=stream, window_size_left=wl,
                            window_size_right=wr, seqused_k=used_t, page_table=table_t,
                            sinks=sinks_t, num_splits=None if ws is not None else 1,
                            workspace=ws)
+
+    set0 = (q, k, v, cq, ck, used_t, table_t, sinks_t)
+
+    def step():
+        step_on(*set0, out, lse)
 
     for _ in range(args.warmup):
         step()
@@ -399,9 +407,19 @@ def run_gpu(args, rank: int, world: int):
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
     else:
-        e2e_ms, h2d, d2h = run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist,
-                                   extra=[t for t in (used_t, table_t, sinks_t)
-                                          if t is not None])
+        ins0 = [t for t in set0 if t is not None]
+        host_in = [pinned(t) for t in ins0]
+        for h, d in zip(host_in, ins0):
+            h.copy_(d)
+        set1 = tuple(None if t is None else torch.empty_like(t) for t in set0)
+        outs = [(out, lse), (torch.empty_like(out), torch.empty_like(lse))]
+        sets = [set0, set1]
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+        e2e_ms = pipelined_e2e(
+            lambda b: step_on(*sets[b], *outs[b]),
+            [[t for t in st if t is not None] for st in sets], host_in, outs,
+            [[pinned(t) for t in o] for o in outs], max(2, min(args.steps, 6)), stream, dist)
 
     if dist:
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
@@ -412,44 +430,64 @@ def run_gpu(args, rank: int, world: int):
         dist.destroy_process_group()
 
 
-def run_e2e(args, case, q, k, v, cq, ck, out, lse, step, stream, dist, extra=()):
+def pipelined_e2e(run_step, dev_in, host_in, dev_out, host_out, steps, stream, dist):
+    """End-to-end time per step through the public API: every step copies all
+    of its inputs from pinned host memory to the device, runs the call and
+    copies all of its results back.  Two device buffer sets take the steps in
+    turn, with the host-to-device and device-to-host copies on streams of
+    their own, so that the copies of one step overlap the call of the other
+    (as a serving loop would run them); a set is refilled only once its
+    previous call has read it, and rewritten only once its results have left.
+    run_step(b) runs the call on buffer set b on `stream`.  Returns ms per
+    step (device time from the first copy to the last result)."""
     import torch
-    hq, hk, hv = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
-    hcq = case.cu_q.pin_memory()
-    hck = case.cu_k.pin_memory() if ck is not None else None
-    ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    hx = [t.cpu().pin_memory() for t in extra]  # further inputs (seqused_k)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcq, hck, *hx) if t is not None)
-    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    dev = stream.device
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+    used = [False, False]
 
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        cq.copy_(hcq, non_blocking=True)
-        if ck is not None:
-            ck.copy_(hck, non_blocking=True)
-        for d, h in zip(extra, hx):
-            d.copy_(h, non_blocking=True)
-        step()
-        ho.copy_(out, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
+    def one(i):
+        b = i % 2
+        if used[b]:
+            h2d_s.wait_event(comp_done[b])
+        with torch.cuda.stream(h2d_s):
+            for d, h in zip(dev_in[b], host_in):
+                d.copy_(h, non_blocking=True)
+        h2d_done[b].record(h2d_s)
+        stream.wait_event(h2d_done[b])
+        if used[b]:
+            stream.wait_event(d2h_done[b])
+        run_step(b)
+        comp_done[b].record(stream)
+        d2h_s.wait_event(comp_done[b])
+        with torch.cuda.stream(d2h_s):
+            for h, d in zip(host_out[b], dev_out[b]):
+                h.copy_(d, non_blocking=True)
+        d2h_done[b].record(d2h_s)
+        used[b] = True
 
-    e2e_steps = max(1, min(args.steps, 5))
-    e2e_step()
+    one(0)
+    one(1)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    h2d_s.wait_event(e0)
+    d2h_s.wait_event(e0)
+    for i in range(steps):
+        one(i)
+    stream.wait_event(d2h_done[(steps - 1) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    return e2e_ms, h2d, d2h
+    return e0.elapsed_time(e1) / steps
+
+
+def pinned(t):
+    import torch
+    return torch.empty(t.shape, dtype=t.dtype).pin_memory()
 
 
 def hbm_line(case, avg_launch_ms: float, peaks: dict, peak_src: str, traffic_key: str,
@@ -518,7 +556,11 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
                           "max": round(max(per_launch), 4)},
             "e2e": {"value": round(whole_job_tflops(world, flops, e2e_ms), 3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": round(e2e_ms, 3)},
+                    "ms_per_step": round(e2e_ms, 3),
+                    "schedule": "every step copies all its inputs from pinned host memory and "
+                                "reads all its results back; two device buffer sets take the "
+                                "steps in turn, the copies on streams of their own overlapping "
+                                "the other set's call"},
             "gpu_launches": args.steps * launches_per_step,
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -608,9 +650,14 @@ def run_gpu_bwd(args, rank: int, world: int):
                      device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step_on(dout, q, k, v, out, lse, cq, ck, dq, dk, dv):
         fa.varlen_attn_bwd(dout, q, k, v, out, lse, cq, ck, case.max_q, case.max_k, case.causal,
                            case.scale, dq=dq, dk=dk, dv=dv, workspace=ws, stream=stream)
+
+    set0 = (dout, q, k, v, out, lse, cq, ck)
+
+    def step():
+        step_on(*set0, dq, dk, dv)
 
     for _ in range(args.warmup):
         step()
@@ -634,31 +681,16 @@ def run_gpu_bwd(args, rank: int, world: int):
 
     e2e_ms, h2d, d2h = float("nan"), 0, 0
     if not args.no_e2e:
-        host_in = [t.cpu().pin_memory() for t in (dout, q, k, v, out, lse, cq, ck)]
-        dev_in = [dout, q, k, v, out, lse, cq, ck]
-        host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+        host_in = [pinned(t) for t in set0]
+        for h, d in zip(host_in, set0):
+            h.copy_(d)
+        sets = [set0, tuple(torch.empty_like(t) for t in set0)]
+        outs = [(dq, dk, dv), tuple(torch.empty_like(t) for t in (dq, dk, dv))]
         h2d = sum(t.numel() * t.element_size() for t in host_in)
-        d2h = sum(t.numel() * t.element_size() for t in host_out)
-
-        def e2e_step():
-            for d_, h_ in zip(dev_in, host_in):
-                d_.copy_(h_, non_blocking=True)
-            step()
-            for h_, d_ in zip(host_out, (dq, dk, dv)):
-                h_.copy_(d_, non_blocking=True)
-
-        e2e_step()
-        torch.cuda.synchronize()
-        if dist:
-            dist.barrier()
-        n = max(1, min(args.steps, 5))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n
+        d2h = sum(t.numel() * t.element_size() for t in outs[0])
+        e2e_ms = pipelined_e2e(lambda b: step_on(*sets[b], *outs[b]), [list(st) for st in sets],
+                               host_in, outs, [[pinned(t) for t in o] for o in outs],
+                               max(2, min(args.steps, 6)), stream, dist)
     if dist:
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
         dist.barrier()
