@@ -174,3 +174,26 @@ def test_short_queries_gqa_packed_fp16(D):
     lk = [900, 129, 64, 1, 300]
     case = workloads.make_case(lq, lk, 16, 2, D, "fp16", True, seed=120 + D)
     full_check(case)
+
+
+@pytest.mark.parametrize("splits", [1, 3, None])
+def test_sequence_table_past_the_buffers_is_clamped(splits):
+    # the last sequence claims 500 more queries and 1000 more keys than the
+    # buffers hold; the kernels clamp every extent to the buffers (total_q,
+    # total_k), so the result is that of the table cut at the buffer ends, and
+    # nothing outside them is read or written (guard rows intact)
+    import dataclasses
+    # (query lengths, max_seqlen_q passed): per-head pairs, GQA-packed, and
+    # decode-like rows (replicated rows with a workspace)
+    for lq, max_q, H, Hkv in (([40, 1, 200], 700, 8, 2), ([40, 1, 200], 700, 32, 8),
+                              ([4, 1, 8], 8, 32, 8)):
+        lk = [300, 5, 1700]
+        case = workloads.make_case(lq, lk, H, Hkv, 128, "bf16", False, seed=1500 + H + max_q)
+        ref_out, ref_lse = oracle.run_case(case)
+        cq = case.cu_q.clone()
+        ck = case.cu_k.clone()
+        cq[-1] += 500
+        ck[-1] += 1000
+        bad = dataclasses.replace(case, cu_q=cq, cu_k=ck)
+        out, lse, _, _ = run_gpu(bad, max_q=max_q, max_k=2700, num_splits=splits)
+        check_close(out, lse, ref_out, ref_lse, "table past the buffers")
