@@ -280,16 +280,18 @@ def time_oracle(case, seconds: float, nthreads: int | None = None):
     about ``seconds`` of CPU work.  Returns (TFLOP/s, rows, flops, secs)."""
     import oracle
     nthreads = nthreads or oracle.default_threads()
-    rows, fl = oracle_sample_rows(case, 256, seed=98)
-    t0 = time.perf_counter()
-    oracle.run_case_rows(case, rows, nthreads=nthreads, **case.mask)
-    rate = fl / max(time.perf_counter() - t0, 1e-6)
-    avg_row = fl / max(len(rows), 1)
-    n = int(max(64, min(2_000_000, seconds * rate / max(avg_row, 1))))
-    rows, fl = oracle_sample_rows(case, n, seed=99)
-    t0 = time.perf_counter()
-    oracle.run_case_rows(case, rows, nthreads=nthreads, **case.mask)
-    dt = time.perf_counter() - t0
+    # a small run sizes the sample; it is rescaled from the measured time
+    # until a run reaches 60 % of the target (a small run underestimates the
+    # rate: fixed costs per call), at most three runs
+    n = 256
+    for attempt in range(3):
+        rows, fl = oracle_sample_rows(case, n, seed=98 + attempt)
+        t0 = time.perf_counter()
+        oracle.run_case_rows(case, rows, nthreads=nthreads, **case.mask)
+        dt = time.perf_counter() - t0
+        if dt >= 0.6 * seconds or n >= 2_000_000:
+            break
+        n = int(max(64, min(2_000_000, n * seconds / max(dt, 1e-3))))
     return fl / dt / 1e12, len(rows), fl, dt, nthreads
 
 
