@@ -348,9 +348,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     if (lane == 0) {
       // Drain: every copy issued has landed before the CTA exits.
-      if (kv_count > 0) wait_bar(&bars->kv_full, (kv_count - 1) & 1u, abort_flag);
+      if (kv_count > 0) drain_wait(&bars->kv_full, (kv_count - 1) & 1u);
       for (uint32_t k = (gs > NST ? gs - NST : 0); k < gs; ++k)
-        wait_bar(&bars->st_full[k % NST], (k / NST) & 1u, abort_flag);
+        drain_wait(&bars->st_full[k % NST], (k / NST) & 1u);
     }
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++items;
       }
       ptx::mma_commit(&bars->drain);
-      wait_bar(&bars->drain, 0, abort_flag);
+      drain_wait(&bars->drain, 0);
     }
   } else {
     // ------------------------------------------------------------ key rows

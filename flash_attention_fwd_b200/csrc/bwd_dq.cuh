@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     if (lane == 0) {
       kv.drain();
-      if (q_count > 0) wait_bar(&bars->q_full, (q_count - 1) & 1u, abort_flag);
+      if (q_count > 0) drain_wait(&bars->q_full, (q_count - 1) & 1u);
     }
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ++items;
       }
       ptx::mma_commit(&bars->drain);
-      wait_bar(&bars->drain, 0, abort_flag);
+      drain_wait(&bars->drain, 0);
     }
   } else {
     // ------------------------------------------------------------ query rows

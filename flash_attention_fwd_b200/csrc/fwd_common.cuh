@@ -383,6 +383,23 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait of the end-of-kernel drains: the copies and MMAs a CTA issued
+// must finish before it exits or frees TMEM, after an abort too, so this wait
+// does not stop at the abort flag; it gives up only after WAIT_TIMEOUT_NS
+// (status bit STATUS_TIMEOUT).  Every drain waits on work already issued,
+// which always completes.
+__device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0 && ptx::globaltimer_ns() - t0 > WAIT_TIMEOUT_NS) {
+      atomicOr(&g_device_status, STATUS_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Producer side of the K/V shared-memory ring: NSLOT slots of one BN-key tile
 // (D / 64 swizzled 128-byte column blocks) each, slot s guarded by full[s]
@@ -520,7 +537,7 @@ struct KVProducer {
   // lane 0: every copy issued has landed (before the CTA exits)
   __device__ void drain() {
     for (int i = 0; i < NSLOT; ++i)
-      if (fills[i] > 0) wait_bar(&full[i], (fills[i] - 1) & 1u, abort_flag);
+      if (fills[i] > 0) drain_wait(&full[i], (fills[i] - 1) & 1u);
   }
 };
 

@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) {
         // Drain: every copy this warp issued has landed before the CTA exits.
         kv.drain();
-        if (q_count > 0) wait_bar(&bars->q_full, (q_count - 1) & 1u, abort_flag);
+        if (q_count > 0) drain_wait(&bars->q_full, (q_count - 1) & 1u);
       }
     }
   } else if (warp == MMA_WARP) {
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
       ptx::mma_commit(&bars->drain);
-      wait_bar(&bars->drain, 0, abort_flag);
+      drain_wait(&bars->drain, 0);
     }
   } else {
     // ------------------------------------------------------------ softmax WG
