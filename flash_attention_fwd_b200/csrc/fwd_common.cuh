@@ -73,6 +73,12 @@ struct KParams {
   // and each copy is a piece of its own for the combine kernel (piece index
   // part * rep + c).  Tile B is not used.
   int rep;
+  // Folded causal units (single kernel, query ranges of BM tokens, Lq = Lk, no
+  // window): query ranges u and nq - 1 - u of a sequence form one unit of
+  // nq + 1 key tiles, handed to one CTA as two consecutive work items (the
+  // second reads K/V the first just brought into L2); an odd nq leaves the
+  // middle range on its own.
+  int fold;
   long long part_rows;  // total_q * H
   float *part_o;
   float *part_lse;
@@ -183,6 +189,9 @@ struct Scheduler {
   int cur_b;              // cursor inside the level: first sequence not passed yet
   long long cur_units;    // (sequence, query tile) units before cur_b in this level
   int split_tiles, max_parts;
+  int fold;               // KParams::fold
+  bool pending;           // the second range of a folded unit is still to be handed out
+  WorkItem pend;
 
   __device__ void extents(int b, int &qs, int &lq, int &ks, int &lk) const {
     seq_extents(cu_q, cu_k, seqused_k, paged, paged_keys, total_q, total_k, b, qs, lq, ks, lk);
@@ -191,7 +200,10 @@ struct Scheduler {
   // nq ranges of U tokens, nk tiles of BM keys.  Without the causal rule a
   // split key range gives each query range P pieces, at levels base + 1 and
   // base.
-  __device__ int units_at(int nq, int nk, int c) const {
+  // folded: the sequence is cut into folded units (fold, causal, Lq = Lk)
+  __device__ bool folded(int lq, int lk) const { return fold && causal && lq == lk && lq > 0; }
+  __device__ int units_at(int nq, int nk, int c, bool fd = false) const {
+    if (fd) return (c == nq + 1 ? nq / 2 : 0) + ((nq & 1) && c == (nq + 1) / 2 ? 1 : 0);
     if (!causal || nk == 0) {
       int P, base, r;
       kv_pieces(nk, split_tiles, max_parts, P, base, r);
@@ -201,8 +213,9 @@ struct Scheduler {
     if (c == nk) return max(0, nq - (nk - 1) * R);
     return 0;
   }
-  __device__ int top_level(int nq, int nk) const {
+  __device__ int top_level(int nq, int nk, bool fd = false) const {
     if (nq == 0) return -1;
+    if (fd) return nq >= 2 ? nq + 1 : 1;
     if (causal && nk > 0) return min(nk, (nq + R - 1) / R);
     int P, base, r;
     kv_pieces(nk, split_tiles, max_parts, P, base, r);
@@ -215,7 +228,7 @@ struct Scheduler {
       if (b < B) {
         int qs, lq, ks, lk;
         extents(b, qs, lq, ks, lk);
-        v = units_at((lq + U - 1) / U, (lk + BM - 1) / BM, c);
+        v = units_at((lq + U - 1) / U, (lk + BM - 1) / BM, c, folded(lq, lk));
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -232,6 +245,8 @@ struct Scheduler {
     paged_keys = paged_key_extent(p);
     split_tiles = p.split_tiles;
     max_parts = p.max_parts;
+    fold = p.fold;
+    pending = false;
     B = p.B;
     HU = p.head_units;
     U = p.unit_tokens;
@@ -249,7 +264,7 @@ struct Scheduler {
       if (b < B) {
         int qs, lq, ks, lk;
         extents(b, qs, lq, ks, lk);
-        top = max(top, top_level((lq + U - 1) / U, (lk + BM - 1) / BM));
+        top = max(top, top_level((lq + U - 1) / U, (lk + BM - 1) / BM, folded(lq, lk)));
       }
     }
 #pragma unroll
@@ -261,7 +276,30 @@ struct Scheduler {
     cur_units = 0;
   }
 
+  // the query range qt of a sequence whose keys are not split: its queries
+  // and the key tiles spanned by their visible keys
+  __device__ void fill_range(WorkItem &w, const KParams &p, int qt, int qs, int lq, int ks,
+                             int lk) const {
+    w.part = -1;
+    w.qi0 = qt * U;
+    w.q0 = qs + w.qi0;
+    w.q_rows = min(U, lq - w.qi0);
+    w.Lk = lk;
+    const int qa = w.qi0, qb = w.qi0 + w.q_rows - 1;
+    const int lo_a = key_lo(p, qa), hi_b = key_hi(p, qb, lk);
+    w.kofs = (lo_a / BN) * BN;
+    w.k0 = ks + w.kofs;
+    w.n_kv = hi_b > lo_a ? (hi_b - w.kofs + BN - 1) / BN : 0;
+    w.min_hi = key_hi(p, qa, lk) - w.kofs;
+    w.max_lo = key_lo(p, qb) - w.kofs;
+  }
+
   __device__ bool next(WorkItem &w, const KParams &p) {
+    if (pending) {
+      pending = false;
+      w = pend;
+      return true;
+    }
     const long long idx = round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
     ++round;
     while (level >= 0 && idx >= level_base + level_items) {
@@ -282,7 +320,7 @@ struct Scheduler {
       int qs = 0, lq = 0, ks = 0, lk = 0, u = 0;
       if (b < B) {
         extents(b, qs, lq, ks, lk);
-        u = units_at((lq + U - 1) / U, (lk + BM - 1) / BM, level);
+        u = units_at((lq + U - 1) / U, (lk + BM - 1) / BM, level, folded(lq, lk));
       }
       int incl = u;
 #pragma unroll
@@ -306,7 +344,18 @@ struct Scheduler {
         const int nk = (lk + BM - 1) / BM;
         int qt, t0 = 0, nt = 0;
         w.part = -1;
-        if (causal && nk > 0) {
+        if (folded(lq, lk)) {
+          // folded unit: ranges k and nq - 1 - k, or the middle range alone
+          const int nq = (lq + U - 1) / U;
+          if (level == nq + 1 && nq >= 2) {
+            qt = k;
+            pend = w;
+            fill_range(pend, p, nq - 1 - k, qs, lq, ks, lk);
+            pending = true;
+          } else {
+            qt = (nq - 1) / 2;
+          }
+        } else if (causal && nk > 0) {
           qt = (min(level, nk) - 1) * R + k;
         } else {
           // units of the level: (piece, query range) with the range fastest, so
@@ -326,20 +375,13 @@ struct Scheduler {
           }
           if (P > 1) w.part = i;
         }
-        w.qi0 = qt * U;
-        w.q0 = qs + w.qi0;
-        w.q_rows = min(U, lq - w.qi0);
-        w.Lk = lk;
         if (w.part < 0) {
-          // key tiles spanned by the visible keys of the first and last query
-          const int qa = w.qi0, qb = w.qi0 + w.q_rows - 1;
-          const int lo_a = key_lo(p, qa), hi_b = key_hi(p, qb, lk);
-          w.kofs = (lo_a / BN) * BN;
-          w.k0 = ks + w.kofs;
-          w.n_kv = hi_b > lo_a ? (hi_b - w.kofs + BN - 1) / BN : 0;
-          w.min_hi = key_hi(p, qa, lk) - w.kofs;
-          w.max_lo = key_lo(p, qb) - w.kofs;
+          fill_range(w, p, qt, qs, lq, ks, lk);
         } else {
+          w.qi0 = qt * U;
+          w.q0 = qs + w.qi0;
+          w.q_rows = min(U, lq - w.qi0);
+          w.Lk = lk;
           // keys [t0 * BM, min((t0 + nt) * BM, lk)); every row sees all keys
           // (a split range has no window and no causal rule)
           const int kend = min((t0 + nt) * BM, lk);

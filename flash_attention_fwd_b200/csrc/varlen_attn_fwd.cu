@@ -375,6 +375,10 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   kp.seqused_k = seqused_k;
   kp.win_left = win_left;
   kp.win_right = win_right;
+  // folded causal units for the single kernel (one query tile per item): the
+  // query tiles of a sequence would otherwise run in different cost rounds, and
+  // with no GQA sharing their K/V prefixes leave the L2 in between
+  kp.fold = (!use_pair && causal && win_left < 0 && layout.unit_tokens == BM) ? 1 : 0;
   kp.page_table = page_table;
   kp.pt_stride = paged ? page_table_stride : 0;
   kp.page_size = paged ? page_size : 0;
