@@ -212,9 +212,12 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 
     ``num_splits`` (non-causal calls without a window only): the key range of
     a row may be computed in up to that many pieces merged by their LSE
-    (varlen_attn_fwd_v4); None lets the library choose, 1 turns it off.  The
-    pieces need a device workspace, allocated here unless ``workspace`` (a
-    uint8 CUDA tensor of at least ``fwd_workspace_size(...)`` bytes) is given.
+    (varlen_attn_fwd_v4), and decode-like calls (at most 32 query rows per
+    KV head) in replicated rows, four copies over interleaved key subsets
+    merged the same way; None lets the library choose, 1 turns both off.
+    The pieces need a device workspace, allocated here unless ``workspace``
+    (a uint8 CUDA tensor of at least ``fwd_workspace_size(...)`` bytes) is
+    given.
     """
     if q.dtype not in DTYPE_CODES or k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share dtype bfloat16 or float16")
