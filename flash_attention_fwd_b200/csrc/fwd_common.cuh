@@ -453,7 +453,11 @@ __device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
 // box never crosses a page); lane c of the warp looks up the page of box c.
 // A box past the sequence's used keys, or whose page-table entry is out of
 // range, is read at a row beyond the buffer, which the TMA fills with zeros.
-template <int BN, int D, int NSLOT>
+//
+// With SPLIT > 1 a slot holds one D-wide column slice of a key tile (the
+// tensor's head dim is SPLIT * D) and a tile takes SPLIT consecutive slots,
+// slice 0 first.
+template <int BN, int D, int NSLOT, int SPLIT = 1>
 struct KVProducer {
   static constexpr int DB = D / 64;
   static constexpr uint32_t KV_BYTES = BN * D * 2;
@@ -483,15 +487,23 @@ struct KVProducer {
       phase ^= 1u;
     }
   }
-  // lane 0: key rows [row, row + BN) of a packed k/v
-  __device__ bool load_packed(const CUtensorMap *tm, int kv_h, int row) {
+  // lane 0: key rows [row, row + BN) of a packed k/v (columns [col0, col0 + D)
+  // of the tensor; col0 a multiple of 64)
+  __device__ bool load_packed(const CUtensorMap *tm, int kv_h, int row, int col0 = 0) {
     if (!wait_bar(&empty[slot], phase ^ 1u, abort_flag)) return false;
     uint8_t *dst = sKV + slot * KV_BYTES;
     ptx::mbar_arrive_expect_tx(&full[slot], KV_BYTES);
 #pragma unroll
     for (int db = 0; db < DB; ++db)
-      ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &full[slot], db * 64, kv_h, row, pol);
+      ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &full[slot], col0 + db * 64, kv_h, row,
+                            pol);
     advance();
+    return true;
+  }
+  __device__ bool tile_packed(const CUtensorMap *tm, int kv_h, int row) {
+#pragma unroll
+    for (int s = 0; s < SPLIT; ++s)
+      if (!load_packed(tm, kv_h, row, s * D)) return false;
     return true;
   }
   // paged: source row of box `lane` of the key tile that starts at key0
@@ -514,7 +526,7 @@ struct KVProducer {
   // Lane 0 waits for the slot and posts the byte count first, so the lanes'
   // copies (one warp instruction per column block) complete into a phase
   // that already expects them.
-  __device__ bool load_paged(const CUtensorMap *tm, int kv_h, int my_row, int ch) {
+  __device__ bool load_paged(const CUtensorMap *tm, int kv_h, int my_row, int ch, int col0 = 0) {
     bool ok = true;
     if (lane == 0) {
       ok = wait_bar(&empty[slot], phase ^ 1u, abort_flag);
@@ -526,9 +538,16 @@ struct KVProducer {
       uint8_t *dst = sKV + slot * KV_BYTES + lane * ch * 128;
 #pragma unroll
       for (int db = 0; db < DB; ++db)
-        ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &full[slot], db * 64, kv_h, my_row, pol);
+        ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &full[slot], col0 + db * 64, kv_h,
+                              my_row, pol);
     }
     advance();
+    return true;
+  }
+  __device__ bool tile_paged(const CUtensorMap *tm, int kv_h, int my_row, int ch) {
+#pragma unroll
+    for (int s = 0; s < SPLIT; ++s)
+      if (!load_paged(tm, kv_h, my_row, ch, s * D)) return false;
     return true;
   }
   // Whole warp: the K/V tiles of one item in the order the MMA warp consumes
@@ -541,18 +560,18 @@ struct KVProducer {
     if (p.page_table == nullptr) {
       bool ok = true;
       if (lane == 0) {
-        ok = load_packed(tm_k, kv_h, w.k0) && load_q();
-        if (ok && n >= 2) ok = load_packed(tm_k, kv_h, w.k0 + BN);
+        ok = tile_packed(tm_k, kv_h, w.k0) && load_q();
+        if (ok && n >= 2) ok = tile_packed(tm_k, kv_h, w.k0 + BN);
         for (int j = 0; ok && j < n; ++j) {
-          ok = load_packed(tm_v, kv_h, w.k0 + j * BN);
-          if (ok && j + 2 < n) ok = load_packed(tm_k, kv_h, w.k0 + (j + 2) * BN);
+          ok = tile_packed(tm_v, kv_h, w.k0 + j * BN);
+          if (ok && j + 2 < n) ok = tile_packed(tm_k, kv_h, w.k0 + (j + 2) * BN);
         }
       }
       return __shfl_sync(0xffffffffu, ok, 0);
     }
     const int ch = p.page_chunk;
     int r0 = chunk_row(p, w, w.kofs), r1 = 0;
-    bool ok = load_paged(tm_k, kv_h, r0, ch);
+    bool ok = tile_paged(tm_k, kv_h, r0, ch);
     if (ok) {
       bool q = true;
       if (lane == 0) q = load_q();
@@ -560,18 +579,18 @@ struct KVProducer {
     }
     if (ok && n >= 2) {
       r1 = chunk_row(p, w, w.kofs + BN);
-      ok = load_paged(tm_k, kv_h, r1, ch);
+      ok = tile_paged(tm_k, kv_h, r1, ch);
     }
     for (int j = 0; ok && j < n; ++j) {
       // look up K(j+2) before waiting for V(j)'s slot, so that the two overlap
       const int rn = (j + 2 < n) ? chunk_row(p, w, w.kofs + (j + 2) * BN) : 0;
-      ok = load_paged(tm_v, kv_h, (j & 1) ? r1 : r0, ch);
+      ok = tile_paged(tm_v, kv_h, (j & 1) ? r1 : r0, ch);
       if (ok && j + 2 < n) {
         if (j & 1)
           r1 = rn;
         else
           r0 = rn;
-        ok = load_paged(tm_k, kv_h, rn, ch);
+        ok = tile_paged(tm_k, kv_h, rn, ch);
       }
     }
     return ok;

@@ -2,8 +2,13 @@
  * fwd_single.cuh — attention forward, one 128-row query tile per work item.
  *
  * Used for head dim 256 (TMEM holds one tile's O of 256 columns plus two S
- * buffers of 64 key columns) and for head layouts without query-head pairs
+ * buffers of 128 key columns) and for head layouts without query-head pairs
  * sharing a key/value head (H / Hkv odd, e.g. plain multi-head attention).
+ *
+ * At head dim 256 a 128-key K or V tile (64 KB) is staged as two 128-column
+ * slices in consecutive ring slots of 32 KB: S = Q K^T runs at N = 128 (an
+ * N = 64 MMA takes as long as an N = 128 one) and PV as two N = 128 products
+ * into the two column halves of O.
  *
  * One persistent CTA per SM, 192 threads:
  *   warps 0-3  softmax warpgroup (thread t = query row t = TMEM lane t)
@@ -26,18 +31,19 @@ constexpr int MMA_WARP = 5;
 
 template <int D>
 struct Cfg;
-// BN = keys per tile, NSLOT = K/V shared-memory ring depth.
+// BN = keys per tile, NSLOT = K/V shared-memory ring depth, SPLIT = column
+// slices of a K/V tile (one ring slot each).
 template <>
 struct Cfg<64> {
-  static constexpr int BN = 128, NSLOT = 8;
+  static constexpr int BN = 128, NSLOT = 8, SPLIT = 1;
 };
 template <>
 struct Cfg<128> {
-  static constexpr int BN = 128, NSLOT = 6;
+  static constexpr int BN = 128, NSLOT = 6, SPLIT = 1;
 };
 template <>
 struct Cfg<256> {
-  static constexpr int BN = 64, NSLOT = 4;
+  static constexpr int BN = 128, NSLOT = 5, SPLIT = 2;
 };
 
 struct Barriers {
@@ -53,9 +59,12 @@ struct Barriers {
 
 template <int D>
 constexpr size_t smem_bytes() {
-  return (size_t)BM * D * 2 + (size_t)Cfg<D>::NSLOT * Cfg<D>::BN * D * 2 + sizeof(Barriers) +
-         1024;
+  return (size_t)BM * D * 2 + (size_t)Cfg<D>::NSLOT * Cfg<D>::BN * (D / Cfg<D>::SPLIT) * 2 +
+         sizeof(Barriers) + 1024;
 }
+static_assert(smem_bytes<256>() <= 232448 && smem_bytes<128>() <= 232448 &&
+                  smem_bytes<64>() <= 232448,
+              "shared memory per block");
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -63,15 +72,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                const __grid_constant__ CUtensorMap tm_v, const KParams p) {
   constexpr int BN = Cfg<D>::BN;
   constexpr int NSLOT = Cfg<D>::NSLOT;
-  constexpr int DB = D / 64;  // 128-byte swizzle blocks along D
+  constexpr int SPLIT = Cfg<D>::SPLIT;
+  constexpr int DS = D / SPLIT;  // columns of a K/V slice (one ring slot)
+  constexpr int DB = D / 64;     // 128-byte swizzle blocks along D
   constexpr uint32_t Q_BYTES = BM * D * 2;
-  constexpr uint32_t KV_BYTES = BN * D * 2;
+  constexpr uint32_t KV_BYTES = BN * DS * 2;
   // TMEM columns: S buffer b at [b*BN, (b+1)*BN), P aliases its first BN/2
   // columns, O accumulator at [2*BN, 2*BN + D).
   constexpr uint32_t O_COL = 2 * BN;
   static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
   constexpr uint32_t IDESC_S = ptx::idesc_f16(BM, BN, BF16, false);
-  constexpr uint32_t IDESC_PV = ptx::idesc_f16(BM, D, BF16, true);
+  constexpr uint32_t IDESC_PV = ptx::idesc_f16(BM, DS, BF16, true);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -129,7 +140,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       sched.init(p);
       uint32_t rs = 0, rph = 0, q_count = 0;
       bool ok = true;
-      KVProducer<BN, D, NSLOT> kv;
+      KVProducer<BN, DS, NSLOT, SPLIT> kv;
       kv.init(sKV, bars->full, bars->empty, abort_flag);
       // Q tile of an item (lane 0)
       auto load_q = [&](const WorkItem &w) -> bool {
@@ -176,35 +187,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       const uint32_t sQ_addr = ptx::smem_u32(sQ);
       const uint32_t sKV_addr = ptx::smem_u32(sKV);
-      auto take_slot = [&](uint32_t &s_out) -> bool {
-        s_out = slot;
-        if (!wait_bar(&bars->full[slot], phase, abort_flag)) return false;
-        ptx::tc_fence_after();
-        if (++slot == NSLOT) {
-          slot = 0;
-          phase ^= 1u;
+      // the SPLIT ring slots of the next K or V tile
+      auto take_tile = [&](uint32_t (&s_out)[SPLIT]) -> bool {
+#pragma unroll
+        for (int i = 0; i < SPLIT; ++i) {
+          s_out[i] = slot;
+          if (!wait_bar(&bars->full[slot], phase, abort_flag)) return false;
+          if (++slot == NSLOT) {
+            slot = 0;
+            phase ^= 1u;
+          }
         }
+        ptx::tc_fence_after();
         return true;
       };
-      // S[buf] = Q K^T over D in steps of 16 (K-major A and B, 128B swizzle)
-      auto issue_s = [&](uint32_t buf, uint32_t kslot) {
-        const uint32_t kbase = sKV_addr + kslot * KV_BYTES;
+      auto release_tile = [&](const uint32_t (&s_in)[SPLIT]) {
+#pragma unroll
+        for (int i = 0; i < SPLIT; ++i) ptx::mma_commit(&bars->empty[s_in[i]]);
+      };
+      // S[buf] = Q K^T over D in steps of 16 (K-major A and B, 128B swizzle);
+      // step kk reads slice kk / (DS / 16) of the K tile
+      auto issue_s = [&](uint32_t buf, const uint32_t (&ks)[SPLIT]) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk % 4) * 32u;  // 16 elements = 32 bytes inside a swizzle row
+          const int ki = kk % (DS / 16);        // step inside the slice
+          const uint32_t off = (ki % 4) * 32u;  // 16 elements = 32 bytes inside a swizzle row
+          const uint32_t kbase = sKV_addr + ks[kk / (DS / 16)] * KV_BYTES;
           uint64_t a = ptx::sdesc_sw128(sQ_addr + (kk / 4) * (BM * 128) + off, 16, 1024);
-          uint64_t bdesc = ptx::sdesc_sw128(kbase + (kk / 4) * (BN * 128) + off, 16, 1024);
+          uint64_t bdesc = ptx::sdesc_sw128(kbase + (ki / 4) * (BN * 128) + off, 16, 1024);
           ptx::mma_ss(tmem + buf * BN, a, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
-      // O += P V over the BN keys in steps of 16 (P from TMEM, V MN-major)
-      auto issue_pv = [&](uint32_t buf, uint32_t vslot, bool acc) {
-        const uint32_t vbase = sKV_addr + vslot * KV_BYTES;
+      // O += P V over the BN keys in steps of 16 (P from TMEM, V MN-major);
+      // slice i of V feeds O's columns [i * DS, (i + 1) * DS)
+      auto issue_pv = [&](uint32_t buf, const uint32_t (&vs)[SPLIT], bool acc) {
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
-          ptx::mma_ts(tmem + O_COL, tmem + buf * BN + kk * 8, bdesc, IDESC_PV,
-                      (acc || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int i = 0; i < SPLIT; ++i) {
+            const uint32_t vbase = sKV_addr + vs[i] * KV_BYTES;
+            uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
+            ptx::mma_ts(tmem + O_COL + i * DS, tmem + buf * BN + kk * 8, bdesc, IDESC_PV,
+                        (acc || kk > 0) ? 1u : 0u);
+          }
         }
       };
       while (ok) {
@@ -221,12 +246,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!wait_bar(&bars->q_full, items & 1u, abort_flag)) break;
         ptx::tc_fence_after();
         for (int jj = 0; ok && jj < 2 && jj < n; ++jj) {
-          uint32_t ks;
-          if (!(ok = take_slot(ks))) break;
+          uint32_t ks[SPLIT];
+          if (!(ok = take_tile(ks))) break;
           const uint32_t buf = (g + jj) & 1u;
           issue_s(buf, ks);
           ptx::mma_commit(&bars->s_full[buf]);
-          ptx::mma_commit(&bars->empty[ks]);
+          release_tile(ks);
           if (jj == n - 1) ptx::mma_commit(&bars->q_empty);
         }
         for (int j = 0; ok && j < n; ++j) {
@@ -238,18 +263,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!(ok = wait_bar(&bars->o_free, (items - 1) & 1u, abort_flag))) break;
             ptx::tc_fence_after();
           }
-          uint32_t vs;
-          if (!(ok = take_slot(vs))) break;
+          uint32_t vs[SPLIT];
+          if (!(ok = take_tile(vs))) break;
           issue_pv(buf, vs, j > 0);
-          ptx::mma_commit(&bars->empty[vs]);
+          release_tile(vs);
           ptx::mma_commit(&bars->pv_done);
           if (j == n - 1) ptx::mma_commit(&bars->o_ready);
           if (j + 2 < n) {
-            uint32_t ks;
-            if (!(ok = take_slot(ks))) break;
+            uint32_t ks[SPLIT];
+            if (!(ok = take_tile(ks))) break;
             issue_s(buf, ks);
             ptx::mma_commit(&bars->s_full[buf]);
-            ptx::mma_commit(&bars->empty[ks]);
+            release_tile(ks);
             if (j + 2 == n - 1) ptx::mma_commit(&bars->q_empty);
           }
         }
