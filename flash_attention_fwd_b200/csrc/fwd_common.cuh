@@ -815,11 +815,13 @@ __device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, fl
 // row gets O / (l + 2^(sink-m)) and LSE = M + log2 l' without overflow.  A
 // row that saw no visible key (l = 0; O is then 0 too) gets O = 0 and
 // LSE = the sink, or -inf without one.  Arrives on o_free (one arrival per
-// warp) as soon as O has been read.
+// warp) as soon as O has been read.  D is the number of columns this thread
+// writes (a column slice of the row when several threads share it; only one
+// of them writes the LSE).
 template <int D, bool BF16>
 __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, float sink_l2,
                                              bool row_valid, uint16_t *orow_ptr, float *lse_ptr,
-                                             uint64_t *o_free, int lane) {
+                                             uint64_t *o_free, int lane, bool write_lse = true) {
   float o_scale = 1.f;
   if (sink_l2 != -INFINITY) {
     const float M = fmaxf(m, sink_l2);
@@ -849,7 +851,8 @@ __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, floa
         dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
     }
   }
-  if (row_valid) *lse_ptr = any ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  if (row_valid && write_lse)
+    *lse_ptr = any ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
 }
 
 // Epilogue of one row of a piece of a split key range: O / l as float32 and
@@ -858,7 +861,7 @@ __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, floa
 template <int D>
 __device__ __forceinline__ void epilogue_part(uint32_t tO, float m, float l, bool row_valid,
                                               float *part_o_row, float *part_lse, uint64_t *o_free,
-                                              int lane) {
+                                              int lane, bool write_lse = true) {
   const bool any = l > 0.f;
   const float inv_l = any ? 1.f / l : 0.f;
 #pragma unroll
@@ -879,7 +882,7 @@ __device__ __forceinline__ void epilogue_part(uint32_t tO, float m, float l, boo
                               __uint_as_float(o[4 * v4 + 3]) * inv_l);
     }
   }
-  if (row_valid) *part_lse = any ? m + log2f(l) : -INFINITY;
+  if (row_valid && write_lse) *part_lse = any ? m + log2f(l) : -INFINITY;
 }
 
 // A query row of an item without visible keys: O = 0, LSE = the sink logit

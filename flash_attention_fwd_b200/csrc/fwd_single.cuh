@@ -10,13 +10,24 @@
  * N = 64 MMA takes as long as an N = 128 one) and PV as two N = 128 products
  * into the two column halves of O.
  *
- * One persistent CTA per SM, 192 threads:
- *   warps 0-3  softmax warpgroup (thread t = query row t = TMEM lane t)
- *   warp 4     TMA producer: Q tile, K/V tiles through a shared-memory ring
- *   warp 5     TMEM owner and MMA issuer
+ * One persistent CTA per SM, 320 threads:
+ *   warps 0-3  softmax, key columns [0, BN/2) of every S tile
+ *   warps 4-7  softmax, key columns [BN/2, BN)
+ *              (thread t of either warpgroup = query row t = TMEM lane t, and
+ *              column half of O: [0, D/2) or [D/2, D))
+ *   warp 8     TMA producer: Q tile, K/V tiles through a shared-memory ring
+ *   warp 9     TMEM owner and MMA issuer
  * S is double-buffered in TMEM so that S(j+1) = Q K(j+1)^T runs on the tensor
  * cores while the softmax warps work on S(j); the MMA order per key tile is
  * S(0), S(1), then PV(j), S(j+2) for j = 0, 1, ...
+ *
+ * The two threads of a row share its running max: per tile each publishes its
+ * half's max in shared memory and both continue with the larger one, so both
+ * take the same rescaling decisions and their P halves carry one scale.  The
+ * packed P of key c goes to column BN/4 + c/2, so the first half's P lands in
+ * columns [BN/4, BN/2) and the second's in [BN/2, 3BN/4): each inside the S
+ * columns that its own warps read, never over S that the other half has
+ * still to load.
  */
 #pragma once
 #include "fwd_common.cuh"
@@ -24,10 +35,11 @@
 namespace vattn {
 namespace single {
 
-constexpr int NUM_THREADS = 192;
-constexpr int PRODUCER_WARP = 4;
-constexpr int RING_CONSUMERS = 1 + 4;  // MMA thread + one arrival per softmax warp
-constexpr int MMA_WARP = 5;
+constexpr int NUM_THREADS = 320;
+constexpr int SOFTMAX_WARPS = 8;
+constexpr int PRODUCER_WARP = 8;
+constexpr int RING_CONSUMERS = 1 + SOFTMAX_WARPS;  // MMA thread + one arrival per softmax warp
+constexpr int MMA_WARP = 9;
 
 template <int D>
 struct Cfg;
@@ -52,10 +64,135 @@ struct Barriers {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2];
   uint64_t pv_done, o_ready, o_free, drain;
+  uint64_t xf[4], xr[4];  // row-pair exchange, per TMEM lane quarter: value written / read
+  float xch[2][BM];       // exchanged value of row r from column half h
   ItemRing ring;
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// Exchange of one float between the two threads of a row (one per column
+// half; warps w and w + 4 cover the same TMEM lanes).  Each swap publishes v
+// in its slot and returns the partner's.  xf completes when both have written,
+// xr when both have read, and a slot is rewritten only after xr of the
+// previous swap, so one slot per thread suffices.  Waits are bounded; false
+// when one gave up (warp-uniform).
+struct RowSwap {
+  float *mine;
+  const volatile float *other;
+  uint64_t *xf, *xr;
+  volatile int *abort_flag;
+  uint32_t n;
+  int lane;
+  __device__ void init(float *a, const float *b, uint64_t *f, uint64_t *rd, int ln,
+                       volatile int *abort) {
+    mine = a;
+    other = b;
+    xf = f;
+    xr = rd;
+    lane = ln;
+    abort_flag = abort;
+    n = 0;
+  }
+  __device__ bool swap(float v, float &out) {
+    if (n > 0 && !__all_sync(0xffffffffu, wait_bar(xr, (n - 1) & 1u, abort_flag))) return false;
+    *mine = v;
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(xf);
+    if (!__all_sync(0xffffffffu, wait_bar(xf, n & 1u, abort_flag))) return false;
+    out = *other;
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(xr);
+    ++n;
+    return true;
+  }
+};
+
+// Softmax of one key tile over this thread's half of its columns (HB keys,
+// S at tS, packed P to tP, O columns [0, DC) at tO) for one row; the row's
+// max over the whole tile comes from the swap with the other half.  Running
+// state and rescaling as in softmax_tile: m (log2 units, possibly stale by up
+// to RESCALE_THRESHOLD) is the same in both halves, l is this half's sum of
+// the rounded P values.  Returns false when a wait gave up.
+template <int HB, int DC, bool BF16, class WaitO>
+__device__ __forceinline__ bool softmax_half(uint32_t tS, uint32_t tP, uint32_t tO, int j,
+                                             float sl2, bool need_mask, int lo, int hi, float &m,
+                                             float &l, RowSwap &xs, WaitO &&wait_o) {
+  uint32_t sr[HB];
+  tmem_ld_wait<HB>(tS, sr);
+  float s[HB];
+#pragma unroll
+  for (int c = 0; c < HB; ++c) s[c] = __uint_as_float(sr[c]);
+  if (need_mask) {
+#pragma unroll
+    for (int c = 0; c < HB; ++c)
+      if (c < lo || c >= hi) s[c] = -INFINITY;
+  }
+  float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+  for (int c = 4; c + 8 <= HB; c += 8) {
+    mx0 = ptx::fmax3(mx0, s[c], s[c + 1]);
+    mx1 = ptx::fmax3(mx1, s[c + 2], s[c + 3]);
+    mx2 = ptx::fmax3(mx2, s[c + 4], s[c + 5]);
+    mx3 = ptx::fmax3(mx3, s[c + 6], s[c + 7]);
+  }
+  mx0 = ptx::fmax3(mx0, s[HB - 4], s[HB - 3]);
+  mx1 = ptx::fmax3(mx1, s[HB - 2], s[HB - 1]);
+  const float mh = fmaxf(ptx::fmax3(mx0, mx1, mx2), mx3);
+  float mo;
+  if (!xs.swap(mh, mo)) return false;
+  const float mx = fmaxf(mh, mo) * sl2;
+  float alpha = 1.f;
+  bool need = false;
+  update_max(j, mx, m, alpha, need);
+  const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
+  const float negm = exp_offset(m);
+  const uint64_t negm_2 = ptx::f2_pack(negm, negm);
+  float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
+#pragma unroll
+  for (int c0 = 0; c0 < HB; c0 += 32) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = c0 + 2 * i;
+      const uint64_t x2 = ptx::f2_fma(ptx::f2_pack(s[c], s[c + 1]), sl2_2, negm_2);
+      float x0, x1;
+      ptx::f2_unpack(x2, x0, x1);
+      pk[i] = pack2<BF16>(ptx::ex2_approx(x0), ptx::ex2_approx(x1));
+      if (i & 1) {
+        sc = ptx::add_lo16<BF16>(pk[i], sc);
+        sd = ptx::add_hi16<BF16>(pk[i], sd);
+      } else {
+        sa = ptx::add_lo16<BF16>(pk[i], sa);
+        sb = ptx::add_hi16<BF16>(pk[i], sb);
+      }
+    }
+    ptx::tmem_st_x16(tP + c0 / 2, pk);
+  }
+  l = l * alpha + ((sa + sb) + (sc + sd));
+  if (__any_sync(0xffffffffu, need)) {
+    if (!__all_sync(0xffffffffu, wait_o())) return false;
+    ptx::tc_fence_after();
+    const uint64_t a2 = ptx::f2_pack(alpha, alpha);
+#pragma unroll
+    for (int c0 = 0; c0 < DC; c0 += 32) {
+      uint32_t o[32];
+      tmem_ld_wait<32>(tO + c0, o);
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        float o0, o1;
+        ptx::f2_unpack(
+            ptx::f2_mul(ptx::f2_pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), a2), o0,
+            o1);
+        o[c] = __float_as_uint(o0);
+        o[c + 1] = __float_as_uint(o1);
+      }
+      tmem_st<32>(tO + c0, o);
+    }
+  }
+  ptx::tmem_st_wait();
+  return true;
+}
 
 template <int D>
 constexpr size_t smem_bytes() {
@@ -77,8 +214,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr int DB = D / 64;     // 128-byte swizzle blocks along D
   constexpr uint32_t Q_BYTES = BM * D * 2;
   constexpr uint32_t KV_BYTES = BN * DS * 2;
-  // TMEM columns: S buffer b at [b*BN, (b+1)*BN), P aliases its first BN/2
-  // columns, O accumulator at [2*BN, 2*BN + D).
+  // TMEM columns: S buffer b at [b*BN, (b+1)*BN), P aliases its columns
+  // [BN/4, 3*BN/4), O accumulator at [2*BN, 2*BN + D).
+  constexpr uint32_t P_COL = BN / 4;
   constexpr uint32_t O_COL = 2 * BN;
   static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
   constexpr uint32_t IDESC_S = ptx::idesc_f16(BM, BN, BF16, false);
@@ -104,11 +242,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::mbar_init(&bars->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars->s_full[i], 1);
-      ptx::mbar_init(&bars->p_full[i], 4);
+      ptx::mbar_init(&bars->p_full[i], SOFTMAX_WARPS);
     }
     ptx::mbar_init(&bars->pv_done, 1);
     ptx::mbar_init(&bars->o_ready, 1);
-    ptx::mbar_init(&bars->o_free, 4);
+    ptx::mbar_init(&bars->o_free, SOFTMAX_WARPS);
+    for (int i = 0; i < 4; ++i) {
+      ptx::mbar_init(&bars->xf[i], 2);
+      ptx::mbar_init(&bars->xr[i], 2);
+    }
     ptx::mbar_init(&bars->drain, 1);
     for (int i = 0; i < ITEM_RING; ++i) {
       ptx::mbar_init(&bars->ring.full[i], 1);
@@ -227,7 +369,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < SPLIT; ++i) {
             const uint32_t vbase = sKV_addr + vs[i] * KV_BYTES;
             uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
-            ptx::mma_ts(tmem + O_COL + i * DS, tmem + buf * BN + kk * 8, bdesc, IDESC_PV,
+            ptx::mma_ts(tmem + O_COL + i * DS, tmem + buf * BN + P_COL + kk * 8, bdesc, IDESC_PV,
                         (acc || kk > 0) ? 1u : 0u);
           }
         }
@@ -286,11 +428,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       drain_wait(&bars->drain, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax WG
-    const int r = threadIdx.x;  // row in the tile == TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t tS0 = tmem + lane_base;
-    const uint32_t tO = tmem + lane_base + O_COL;
+    // ------------------------------------------------------------ softmax
+    constexpr int HB = BN / 2;  // key columns per half
+    constexpr int DC = D / 2;   // O columns per half
+    const int h = threadIdx.x / BM;  // column half
+    const int r = threadIdx.x % BM;  // row in the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS0 = tmem + lane_base + h * HB;
+    const uint32_t tP0 = tmem + lane_base + P_COL + h * (HB / 2);
+    const uint32_t tO = tmem + lane_base + O_COL + h * DC;
+    RowSwap xs;
+    xs.init(&bars->xch[h][r], &bars->xch[h ^ 1][r], &bars->xf[warp & 3], &bars->xr[warp & 3],
+            lane, abort_flag);
     const float sl2 = p.scale_log2;
     uint32_t rs = 0, rph = 0;
     uint32_t g = 0, items = 0;
@@ -312,12 +461,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const size_t orow = (size_t)(w.q0 + r) * p.H + w.hu;  // row index into [total_q, H]
       uint16_t *orow_ptr = reinterpret_cast<uint16_t *>(p.out) + orow * D;
       if (n == 0) {
-        if (row_valid) empty_row<D>(orow_ptr, p.lse + orow, sink_log2(p, w.hu));
+        if (row_valid && h == 0) empty_row<D>(orow_ptr, p.lse + orow, sink_log2(p, w.hu));
         continue;
       }
-      // visible keys of this row, relative to the first visited key tile
-      const int lo = key_lo(p, qi) - w.kofs;
-      const int hi = key_hi(p, qi, w.Lk) - w.kofs;
+      // visible keys of this row, relative to the first key of this thread's
+      // half of the first visited key tile
+      const int lo = key_lo(p, qi) - w.kofs - h * HB;
+      const int hi = key_hi(p, qi, w.Lk) - w.kofs - h * HB;
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
         const uint32_t gj = g + j;
@@ -334,8 +484,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // phase gj-1 or gj.
         auto wait_o = [&]() { return wait_bar(&bars->pv_done, (gj - 1) & 1u, abort_flag); };
         const bool need_mask = j * BN < w.max_lo || (j + 1) * BN > w.min_hi;
-        if (!softmax_tile<BN, D, BF16>(tS0 + buf * BN, tO, j, sl2, need_mask, lo - j * BN,
-                                       hi - j * BN, m, l, wait_o)) {
+        if (!softmax_half<HB, DC, BF16>(tS0 + buf * BN, tP0 + buf * BN, tO, j, sl2, need_mask,
+                                        lo - j * BN, hi - j * BN, m, l, xs, wait_o)) {
           ok = false;
           break;
         }
@@ -354,12 +504,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       ptx::tc_fence_after();
+      // the row's sum over both halves (the same float in both threads)
+      float l_other;
+      if (!xs.swap(l, l_other)) {
+        ok = false;
+        break;
+      }
+      l += l_other;
       if (w.part < 0)
-        epilogue_row<D, BF16>(tO, m, l, sink_log2(p, w.hu), row_valid, orow_ptr, p.lse + orow,
-                              &bars->o_free, lane);
+        epilogue_row<DC, BF16>(tO, m, l, sink_log2(p, w.hu), row_valid, orow_ptr + h * DC,
+                               p.lse + orow, &bars->o_free, lane, h == 0);
       else
-        epilogue_part<D>(tO, m, l, row_valid, p.part_o + ((size_t)w.part * p.part_rows + orow) * D,
-                         p.part_lse + (size_t)w.part * p.part_rows + orow, &bars->o_free, lane);
+        epilogue_part<DC>(tO, m, l, row_valid,
+                          p.part_o + ((size_t)w.part * p.part_rows + orow) * D + h * DC,
+                          p.part_lse + (size_t)w.part * p.part_rows + orow, &bars->o_free, lane,
+                          h == 0);
     }
   }
 
