@@ -59,8 +59,8 @@ def test_split_single_kernel_odd_group(D, dtype):
 
 
 def test_split_single_kernel_wide_head_large_logits():
-    # D = 256 (64-key tiles in the kernel, pieces in 128-key tiles), std of the
-    # scaled scores about 9
+    # D = 256 (the single-tile kernel: K/V tiles in two column slices, two
+    # softmax halves per row), std of the scaled scores about 9
     case = workloads.make_case([5, 64, 30], [3000, 1500, 257], 2, 2, 256, "fp16", False,
                                seed=1040, sigma_q=3.0, sigma_k=3.0)
     full_check(case, num_splits=6)
