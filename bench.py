@@ -147,10 +147,13 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-# Device-code sources of each direction's kernels (the host code does not
-# change a kernel's traffic).
+# Device-code sources of each kernel family (the host code does not change a
+# kernel's traffic): all forward kernels, the pair kernel and the single-tile
+# kernel alone, the merge of split key ranges, the backward.
 KERNEL_SOURCES = {
     "fwd": ("sm100_ptx.cuh", "fwd_common.cuh", "fwd_pair.cuh", "fwd_single.cuh"),
+    "pair": ("sm100_ptx.cuh", "fwd_common.cuh", "fwd_pair.cuh"),
+    "single": ("sm100_ptx.cuh", "fwd_common.cuh", "fwd_single.cuh"),
     "combine": ("fwd_common.cuh", "fwd_combine.cuh"),
     "bwd": ("sm100_ptx.cuh", "fwd_common.cuh", "bwd_common.cuh", "bwd_dq.cuh", "bwd_dkdv.cuh"),
 }
@@ -169,13 +172,15 @@ def kernel_hash(read=None, kind: str = "fwd") -> str:
 
 def traffic_for(workload: str):
     """DRAM bytes per launch from the committed ncu summary, only if it was
-    taken on the current kernel source."""
+    taken on the current source of the kernel family the entry names
+    (``kernel_kind``, a key of KERNEL_SOURCES)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         ent = d.get(workload)
-        kind = "bwd" if workload.endswith(":bwd") else "fwd"
+        default = "bwd" if workload.endswith(":bwd") else "fwd"
+        kind = ent.get("kernel_kind", default) if ent else default
         if ent and ent.get("kernel_hash") == kernel_hash(kind=kind):
             return ent.get("bytes_per_launch")
     except Exception:

@@ -343,35 +343,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tc_fence_after();
         return true;
       };
-      auto release_tile = [&](const uint32_t (&s_in)[SPLIT]) {
-#pragma unroll
-        for (int i = 0; i < SPLIT; ++i) ptx::mma_commit(&bars->empty[s_in[i]]);
-      };
-      // S[buf] = Q K^T over D in steps of 16 (K-major A and B, 128B swizzle);
-      // step kk reads slice kk / (DS / 16) of the K tile
+      // S[buf] = Q K^T over D in steps of 16 (K-major A and B, 128B swizzle),
+      // slice by slice; each slice's ring slot is released (commit) as soon
+      // as the MMAs issued so far, which include all that read it, complete
       auto issue_s = [&](uint32_t buf, const uint32_t (&ks)[SPLIT]) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int ki = kk % (DS / 16);        // step inside the slice
-          const uint32_t off = (ki % 4) * 32u;  // 16 elements = 32 bytes inside a swizzle row
-          const uint32_t kbase = sKV_addr + ks[kk / (DS / 16)] * KV_BYTES;
-          uint64_t a = ptx::sdesc_sw128(sQ_addr + (kk / 4) * (BM * 128) + off, 16, 1024);
-          uint64_t bdesc = ptx::sdesc_sw128(kbase + (ki / 4) * (BN * 128) + off, 16, 1024);
-          ptx::mma_ss(tmem + buf * BN, a, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+        for (int i = 0; i < SPLIT; ++i) {
+          const uint32_t kbase = sKV_addr + ks[i] * KV_BYTES;
+#pragma unroll
+          for (int ki = 0; ki < DS / 16; ++ki) {
+            const int kk = i * (DS / 16) + ki;    // step along D
+            const uint32_t off = (ki % 4) * 32u;  // 16 elements = 32 bytes inside a swizzle row
+            uint64_t a = ptx::sdesc_sw128(sQ_addr + (kk / 4) * (BM * 128) + off, 16, 1024);
+            uint64_t bdesc = ptx::sdesc_sw128(kbase + (ki / 4) * (BN * 128) + off, 16, 1024);
+            ptx::mma_ss(tmem + buf * BN, a, bdesc, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          if (i == SPLIT - 1) ptx::mma_commit(&bars->s_full[buf]);
+          ptx::mma_commit(&bars->empty[ks[i]]);
         }
       };
       // O += P V over the BN keys in steps of 16 (P from TMEM, V MN-major);
-      // slice i of V feeds O's columns [i * DS, (i + 1) * DS)
+      // slice i of V feeds O's columns [i * DS, (i + 1) * DS) and its slot is
+      // released right after its MMAs
       auto issue_pv = [&](uint32_t buf, const uint32_t (&vs)[SPLIT], bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
+        for (int i = 0; i < SPLIT; ++i) {
+          const uint32_t vbase = sKV_addr + vs[i] * KV_BYTES;
 #pragma unroll
-          for (int i = 0; i < SPLIT; ++i) {
-            const uint32_t vbase = sKV_addr + vs[i] * KV_BYTES;
+          for (int kk = 0; kk < BN / 16; ++kk) {
             uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
             ptx::mma_ts(tmem + O_COL + i * DS, tmem + buf * BN + P_COL + kk * 8, bdesc, IDESC_PV,
                         (acc || kk > 0) ? 1u : 0u);
           }
+          ptx::mma_commit(&bars->empty[vs[i]]);
         }
       };
       while (ok) {
@@ -392,8 +396,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!(ok = take_tile(ks))) break;
           const uint32_t buf = (g + jj) & 1u;
           issue_s(buf, ks);
-          ptx::mma_commit(&bars->s_full[buf]);
-          release_tile(ks);
           if (jj == n - 1) ptx::mma_commit(&bars->q_empty);
         }
         for (int j = 0; ok && j < n; ++j) {
@@ -408,15 +410,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t vs[SPLIT];
           if (!(ok = take_tile(vs))) break;
           issue_pv(buf, vs, j > 0);
-          release_tile(vs);
           ptx::mma_commit(&bars->pv_done);
           if (j == n - 1) ptx::mma_commit(&bars->o_ready);
           if (j + 2 < n) {
             uint32_t ks[SPLIT];
             if (!(ok = take_tile(ks))) break;
             issue_s(buf, ks);
-            ptx::mma_commit(&bars->s_full[buf]);
-            release_tile(ks);
             if (j + 2 == n - 1) ptx::mma_commit(&bars->q_empty);
           }
         }
