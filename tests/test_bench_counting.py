@@ -61,3 +61,33 @@ def test_named_masked_workloads():
     used = workloads.seqused_k("shortq_used")
     _, lk = workloads.seqlens("shortq_used")
     assert len(used) == 32 and all(k // 2 <= u <= k for u, k in zip(used, lk))
+
+
+def test_traffic_entries_follow_their_kernel_family(tmp_path, monkeypatch):
+    # an entry counts only while the sources of the family it names hash to
+    # the value it was captured on; an edit to another family leaves it valid
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "traffic.json").write_text(
+        '{"a": {"kernel_kind": "pair", "kernel_hash": "P1", "bytes_per_launch": 10},'
+        ' "b": {"kernel_kind": "single", "kernel_hash": "S0", "bytes_per_launch": 20},'
+        ' "c": {"kernel_hash": "F1", "bytes_per_launch": 30},'
+        ' "c:bwd": {"kernel_hash": "B1", "bytes_per_launch": 40}}')
+    hashes = {"pair": "P1", "single": "S1", "fwd": "F1", "bwd": "B1"}
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_hash", lambda read=None, kind="fwd": hashes[kind])
+    assert bench.traffic_for("a") == 10
+    assert bench.traffic_for("b") is None       # single-kernel source changed since
+    assert bench.traffic_for("c") == 30         # no family named: all forward kernels
+    assert bench.traffic_for("c:bwd") == 40     # backward by the key's suffix
+    assert bench.traffic_for("missing") is None
+
+
+def test_committed_traffic_entries_name_known_families():
+    import json
+    import os
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        d = json.load(f)
+    for key, ent in d.items():
+        assert ent["kernel_kind"] in bench.KERNEL_SOURCES, key
+        assert len(ent["kernel_hash"]) == 16 and ent["bytes_per_launch"] > 0, key
