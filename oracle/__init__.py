@@ -6,10 +6,12 @@ library in ``flash_attention_fwd_b200`` and never imports it.
 
 Two independent implementations live here:
 
-* ``varlen_attn_oracle.c`` (loaded through ctypes): the CPU forward loop of
-  boostr 0.2.0, src/ops/cpu/attention/varlen_attention.rs
-  (``varlen_attention_fwd``), restated in double precision and threaded over
-  (sequence, head) work items.
+* ``varlen_attn_oracle.c`` (loaded through ctypes): the packed attention
+  forward defined by the boostr 0.2.0 source page
+  src/ops/cpu/attention/varlen_attention.rs (``varlen_attention_fwd``),
+  written from the definition in double precision (visible keys gathered
+  first, the LSE as a separate log-sum-exp, O as the exp(s - LSE)-weighted
+  sum of values) and threaded over (sequence, head) work items.
 * ``brute.py``: a dense NumPy restatement of the same definition that builds
   the full [Tq, Tk] score matrix with a block-diagonal (and causal) mask.
   Used only on tiny inputs to pin the C oracle.
@@ -202,7 +204,7 @@ def run_case_rows(case, rows, nthreads=None, **mask):
 
 def varlen_attn_bwd(dout, q, k, v, out, lse, cu_q, cu_k, H, Hkv, D, causal, scale, dtype,
                     nthreads=None, lib=None):
-    """fp64 backward of the page's loop.  dout/q [Tq,H,D] and k/v [Tk,Hkv,D]
+    """fp64 gradient of the forward (the page's varlen_attention_bwd).  dout/q [Tq,H,D] and k/v [Tk,Hkv,D]
     are bf16/fp16 tensors; out [Tq,H,D] and lse [Tq,H] any float tensor or
     array (widened to double).  Returns (dq [Tq,H,D], dk [Tk,Hkv,D],
     dv [Tk,Hkv,D]) float64."""

@@ -5,20 +5,22 @@
  * load this file: only the tests, the package's smoke check and the bench's
  * CPU-baseline leg use it.  It shares no code with the CUDA library.
  *
- * What it computes follows the CPU forward loop of boostr 0.2.0,
- * src/ops/cpu/attention/varlen_attention.rs (VarLenAttentionOps::
- * varlen_attention_fwd), step for step, with every f32 replaced by double:
+ * What it computes is the packed attention forward defined by the boostr
+ * 0.2.0 source page src/ops/cpu/attention/varlen_attention.rs
+ * (VarLenAttentionOps::varlen_attention_fwd), written here from that
+ * definition in double precision rather than in the shape of the page's
+ * loop.  For sequence b, query head h and sequence-local query qi:
  *
- *   for each sequence b, query head h, query qi in [0, Lq_b):
- *     kv_h = h / (H / Hkv)                           (GQA head map)
- *     for each key ki in [0, Lk_b):
- *       masked when causal and qi < ki                (sequence-local indices)
- *       s_ki = (sum_d Q[cu_q[b]+qi, h, d] * K[cu_k[b]+ki, kv_h, d]) * scale
- *     m = max of the unmasked s_ki
- *     e_ki = exp(s_ki - m)        (masked keys give exp(-inf) = 0)
- *     l = sum of e_ki
- *     O[cu_q[b]+qi, h, :] = sum_ki (e_ki / l) * V[cu_k[b]+ki, kv_h, :]
- *     LSE[cu_q[b]+qi, h]  = m + ln(l)
+ *   kv_h = h / (H / Hkv)                                  (GQA head map)
+ *   V(qi) = { ki in [0, Lk_b) : not (causal and qi < ki) }  (visible keys)
+ *   s_ki  = scale * <Q[cu_q[b]+qi, h, :], K[cu_k[b]+ki, kv_h, :]>  for ki in V(qi)
+ *   LSE   = log-sum-exp of { s_ki : ki in V(qi) }          (natural log)
+ *   O[cu_q[b]+qi, h, :] = sum over ki in V(qi) of exp(s_ki - LSE) * V[cu_k[b]+ki, kv_h, :]
+ *
+ * The visible keys are gathered first, the LSE comes from a separate
+ * max-shifted log-sum-exp reduction, and the weights exp(s - LSE) are the
+ * softmax over V(qi).  A row with an empty V(qi) gets O = 0 and LSE = -inf
+ * (the page's result for a sequence without keys).
  *
  * Layouts are the page's packed ones: Q/O [Tq, H, D], K/V [Tk, Hkv, D],
  * LSE [Tq, H], all row-major.  The scale is an explicit argument; a value
@@ -27,51 +29,44 @@
  * Extension (the `_ext` entry points): the sliding window and used-key count
  * that PyTorch pull request #176015 lists in the varlen forward schema
  * (window_size_left, window_size_right, seqused_k), read with the page's
- * sequence-local indices: key ki is also hidden when ki >= seqused_k[b]
+ * sequence-local indices: key ki also leaves V(qi) when ki >= seqused_k[b]
  * (clipped to [0, Lk_b]), when left >= 0 and ki < qi - left, or when
- * right >= 0 and ki > qi + right.  A row with no visible key gets O = 0 and
- * LSE = -inf, what the page's loop gives for a sequence without keys.
+ * right >= 0 and ki > qi + right.
  *
  * Attention sinks (the `sinks` argument of the `_ext` entry points; the
  * FLOAT32 per-head "sinks" input of the Ascend sparse shared-KV attention
  * page, which gives no formula): sinks[h] is one more logit, already in score
- * units (not multiplied by the scale), that joins the softmax of every row of
- * query head h but has no value row.  So m = max(max_ki s_ki, sinks[h]),
- * l = sum_ki exp(s_ki - m) + exp(sinks[h] - m), O = sum_ki exp(s_ki - m) / l
- * * V_ki, LSE = m + ln(l); a row without visible keys then gets O = 0 and
- * LSE = sinks[h].
+ * units (not multiplied by the scale), with no value row.  It is one more
+ * term of the log-sum-exp, LSE = ln(sum_ki exp(s_ki) + exp(sinks[h])), and
+ * the value sum keeps the weights exp(s_ki - LSE); a row with an empty V(qi)
+ * then gets O = 0 and LSE = sinks[h].
  *
- * Backward (oracle_varlen_attn_bwd): the CPU backward loop of the same page
- * (VarLenAttentionOps::varlen_attention_bwd), step for step in double
- * precision.  Given dO, Q, K, V, the forward output O and LSE:
+ * Backward (oracle_varlen_attn_bwd): the gradient of the forward as the
+ * same page's VarLenAttentionOps::varlen_attention_bwd defines it, in double
+ * precision, given dO, Q, K, V, the forward output O and LSE.  Per query row
+ * (b, h, qi), over its visible keys ki:
  *
- *   for each sequence b, query head h (kv_h = h / (H / Hkv)), query qi:
- *     delta = sum_d dO[qi, h, d] * O[qi, h, d]
- *     for each visible key ki (causal: skip qi < ki):
- *       s  = scale * <Q[qi, h], K[ki, kv_h]>
- *       p  = exp(s - LSE[qi, h])                 (the softmax weight)
- *       dp = <V[ki, kv_h], dO[qi, h]>
- *       ds = p * (dp - delta)
- *       dQ[qi, h]     += scale * ds * K[ki, kv_h]
- *       dK[ki, kv_h]  += scale * ds * Q[qi, h]
- *       dV[ki, kv_h]  += p * dO[qi, h]
+ *   P_ki  = exp(s_ki - LSE[qi, h])          (the softmax weights)
+ *   dP_ki = <dO[qi, h], V[ki, kv_h]>
+ *   delta = <dO[qi, h], O[qi, h]>
+ *   dS_ki = P_ki (dP_ki - delta)
+ *   dQ[qi, h]    = scale * sum_ki dS_ki K[ki, kv_h]
+ *   dK[ki, kv_h] += scale * dS_ki Q[qi, h]      (summed over the group's heads)
+ *   dV[ki, kv_h] += P_ki dO[qi, h]
  *
- * dK and dV sum over the H / Hkv query heads of their key/value head.  The
- * scale is the page's 1/sqrt(D) unless given (as in the forward).  dO is
- * 16-bit like Q/K/V; O and LSE are given in double (the caller widens the
- * stored bf16/fp16 O and float32 LSE exactly, or passes exact values).  Work items are (b, kv_h): each owns the dK/dV rows
- * of that key/value head of sequence b and the dQ rows of its query heads,
- * and runs the loop above serially, so the result does not depend on the
- * thread count.
+ * The row's vectors P, dP and dS are formed first; the three gradient sums
+ * follow.  dO is 16-bit like Q/K/V; O and LSE are given in double (the caller
+ * widens the stored bf16/fp16 O and float32 LSE exactly, or passes exact
+ * values).  Work items are (b, kv_h): each owns the dK/dV rows of that
+ * key/value head of sequence b and the dQ rows of its query heads, and runs
+ * its rows in a fixed order, so the result does not depend on the thread
+ * count.
  *
  * Inputs are bf16 or fp16 bit patterns; they are widened exactly to double
- * before any arithmetic.  The widening of a key/value head of one sequence
- * is done once per (b, h) work item; that is a format conversion, not a
- * change to the order of the attention arithmetic.
- *
- * Work items (b, h) are spread over POSIX threads; each output row is
- * computed by one thread with the serial loop above, so the result does not
- * depend on the thread count.
+ * before any arithmetic (a format conversion, once per (b, kv_h) item for
+ * K and V).  Forward work items (b, h), or single requested rows, are spread
+ * over POSIX threads; each output row is computed by one thread, so the
+ * result does not depend on the thread count.
  */
 #include <math.h>
 #include <pthread.h>
@@ -159,45 +154,52 @@ static int key_hidden(const OracleCtx *c, int qi, int ki) {
     return 0;
 }
 
-/* One query row: the page's two-pass softmax, in double precision.
- * kd/vd hold the widened keys/values of head kv_h of sequence b, [Lk][D]. */
-static void oracle_attend_row(const OracleCtx *c, const double *qrow, int qi, int Lk,
-                              const double *kd, const double *vd, double *scores, double sink,
-                              double *out_row, double *lse_out) {
+/* Indices of the keys of V(qi) among the first Lk keys of the sequence, in
+ * increasing order, into idx; returns how many there are. */
+static int visible_keys(const OracleCtx *c, int qi, int Lk, int *idx) {
+    int n = 0;
+    for (int ki = 0; ki < Lk; ++ki)
+        if (!key_hidden(c, qi, ki)) idx[n++] = ki;
+    return n;
+}
+
+static double dot_d(const double *a, const double *b, int D) {
+    double acc = 0.0;
+    for (int d = 0; d < D; ++d) acc += a[d] * b[d];
+    return acc;
+}
+
+/* ln(exp(extra) + sum_i exp(x[i])), shifted by the largest term; -inf for
+ * an empty sum (n = 0 and extra = -inf). */
+static double log_sum_exp(const double *x, int n, double extra) {
+    double m = extra;
+    for (int i = 0; i < n; ++i)
+        if (x[i] > m) m = x[i];
+    if (m == -INFINITY) return -INFINITY;
+    double acc = exp(extra - m);
+    for (int i = 0; i < n; ++i) acc += exp(x[i] - m);
+    return m + log(acc);
+}
+
+/* One output row from the definition: the scores of the visible keys, their
+ * log-sum-exp (with the head's sink logit as one more term), and the value
+ * rows weighted by exp(s - LSE).  kd/vd hold the widened keys/values of head
+ * kv_h of sequence b, [Lk][D]; idx and s are scratch of Lk entries. */
+static void oracle_row(const OracleCtx *c, const double *qrow, int qi, int Lk, const double *kd,
+                       const double *vd, int *idx, double *s, double sink, double *out_row,
+                       double *lse_out) {
     const int D = c->D;
-    double max_score = -INFINITY;
-    for (int ki = 0; ki < Lk; ++ki) {
-        if (key_hidden(c, qi, ki)) {
-            scores[ki] = -INFINITY;
-            continue;
-        }
-        double dot = 0.0;
-        const double *krow = kd + (size_t)ki * D;
-        for (int d = 0; d < D; ++d) dot += qrow[d] * krow[d];
-        double s = dot * c->scale;
-        if (s > max_score) max_score = s;
-        scores[ki] = s;
-    }
-    if (sink > max_score) max_score = sink; /* the sink logit takes part in the max */
-    if (max_score == -INFINITY) { /* no visible key and no sink */
-        for (int d = 0; d < D; ++d) out_row[d] = 0.0;
-        *lse_out = -INFINITY;
-        return;
-    }
-    double sum_exp = 0.0;
-    for (int ki = 0; ki < Lk; ++ki) {
-        double e = exp(scores[ki] - max_score);
-        sum_exp += e;
-        scores[ki] = e;
-    }
-    sum_exp += exp(sink - max_score); /* ... and in the normalisation (0 without a sink) */
+    const int n = visible_keys(c, qi, Lk, idx);
+    for (int i = 0; i < n; ++i) s[i] = c->scale * dot_d(qrow, kd + (size_t)idx[i] * D, D);
+    const double lse = log_sum_exp(s, n, sink);
     for (int d = 0; d < D; ++d) out_row[d] = 0.0;
-    for (int ki = 0; ki < Lk; ++ki) {
-        double weight = scores[ki] / sum_exp;
-        const double *vrow = vd + (size_t)ki * D;
-        for (int d = 0; d < D; ++d) out_row[d] += weight * vrow[d];
+    *lse_out = lse;
+    if (lse == -INFINITY) return;
+    for (int i = 0; i < n; ++i) {
+        const double w = exp(s[i] - lse);
+        const double *vrow = vd + (size_t)idx[i] * D;
+        for (int d = 0; d < D; ++d) out_row[d] += w * vrow[d];
     }
-    *lse_out = max_score + log(sum_exp);
 }
 
 static void widen_kv(const OracleCtx *c, int b, int kv_h, double *kd, double *vd) {
@@ -235,10 +237,11 @@ static void *full_worker(void *arg) {
     double *kd = (double *)malloc(kvn * sizeof(double));
     double *vd = (double *)malloc(kvn * sizeof(double));
     double *scores = (double *)malloc((size_t)(mk > 0 ? mk : 1) * sizeof(double));
+    int *idx = (int *)malloc((size_t)(mk > 0 ? mk : 1) * sizeof(int));
     double *qd = (double *)malloc((size_t)D * sizeof(double));
-    if (!kd || !vd || !scores || !qd) {
+    if (!kd || !vd || !scores || !idx || !qd) {
         __atomic_store_n(&c->status, -1, __ATOMIC_RELAXED);
-        free(kd); free(vd); free(scores); free(qd);
+        free(kd); free(vd); free(scores); free(idx); free(qd);
         return NULL;
     }
     for (;;) {
@@ -253,12 +256,11 @@ static void *full_worker(void *arg) {
         for (int qi = 0; qi < Lq; ++qi) {
             int64_t tok = (int64_t)q0 + qi;
             widen_q(c, tok, h, qd);
-            oracle_attend_row(c, qd, qi, Lk, kd, vd, scores, head_sink(c, h),
-                              c->out + ((size_t)tok * H + h) * D,
-                              c->lse + (size_t)tok * H + h);
+            oracle_row(c, qd, qi, Lk, kd, vd, idx, scores, head_sink(c, h),
+                       c->out + ((size_t)tok * H + h) * D, c->lse + (size_t)tok * H + h);
         }
     }
-    free(kd); free(vd); free(scores); free(qd);
+    free(kd); free(vd); free(scores); free(idx); free(qd);
     return NULL;
 }
 
@@ -282,11 +284,12 @@ static void *rows_worker(void *arg) {
     double *kd = (double *)malloc(kvn * sizeof(double));
     double *vd = (double *)malloc(kvn * sizeof(double));
     double *scores = (double *)malloc((size_t)(mk > 0 ? mk : 1) * sizeof(double));
+    int *idx = (int *)malloc((size_t)(mk > 0 ? mk : 1) * sizeof(int));
     double *qd = (double *)malloc((size_t)D * sizeof(double));
     int cached_b = -1, cached_kvh = -1;
-    if (!kd || !vd || !scores || !qd) {
+    if (!kd || !vd || !scores || !idx || !qd) {
         __atomic_store_n(&c->status, -1, __ATOMIC_RELAXED);
-        free(kd); free(vd); free(scores); free(qd);
+        free(kd); free(vd); free(scores); free(idx); free(qd);
         return NULL;
     }
     for (;;) {
@@ -304,10 +307,10 @@ static void *rows_worker(void *arg) {
             cached_kvh = kv_h;
         }
         widen_q(c, tok, h, qd);
-        oracle_attend_row(c, qd, qi, Lk, kd, vd, scores, head_sink(c, h),
-                          c->out_rows + (size_t)i * D, c->lse_rows + i);
+        oracle_row(c, qd, qi, Lk, kd, vd, idx, scores, head_sink(c, h),
+                   c->out_rows + (size_t)i * D, c->lse_rows + i);
     }
-    free(kd); free(vd); free(scores); free(qd);
+    free(kd); free(vd); free(scores); free(idx); free(qd);
     return NULL;
 }
 
@@ -409,46 +412,87 @@ typedef struct {
     int status;
 } OracleBwdCtx;
 
-static double bwd_elem(const OracleBwdCtx *c, const uint16_t *t, size_t off) {
-    return oracle_decode16(t[off], c->dtype);
+/* Keys of the sequence visible to query qi (the causal rule only), in
+ * increasing order, into idx; returns how many there are. */
+static int bwd_visible_keys(const OracleBwdCtx *c, int qi, int Lk, int *idx) {
+    int n = 0;
+    for (int ki = 0; ki < Lk; ++ki) {
+        if (c->causal && qi < ki) continue;
+        idx[n++] = ki;
+    }
+    return n;
+}
+
+static void bwd_widen(const OracleBwdCtx *c, const uint16_t *t, size_t off, int D, double *dst) {
+    for (int d = 0; d < D; ++d) dst[d] = oracle_decode16(t[off + d], c->dtype);
 }
 
 static void *bwd_worker(void *arg) {
     OracleBwdCtx *c = (OracleBwdCtx *)arg;
     const int D = c->D, H = c->H, Hkv = c->Hkv, G = c->H / c->Hkv;
+    int mk = 0;
+    for (int b = 0; b < c->B; ++b)
+        if (c->cu_k[b + 1] - c->cu_k[b] > mk) mk = c->cu_k[b + 1] - c->cu_k[b];
+    const size_t nk = (size_t)(mk > 0 ? mk : 1);
+    double *kd = (double *)malloc(nk * D * sizeof(double));
+    double *vd = (double *)malloc(nk * D * sizeof(double));
+    double *p = (double *)malloc(nk * sizeof(double));
+    double *dp = (double *)malloc(nk * sizeof(double));
+    double *ds = (double *)malloc(nk * sizeof(double));
+    int *idx = (int *)malloc(nk * sizeof(int));
+    double *qd = (double *)malloc((size_t)D * sizeof(double));
+    double *dod = (double *)malloc((size_t)D * sizeof(double));
+    if (!kd || !vd || !p || !dp || !ds || !idx || !qd || !dod) {
+        __atomic_store_n(&c->status, -1, __ATOMIC_RELAXED);
+        free(kd); free(vd); free(p); free(dp); free(ds); free(idx); free(qd); free(dod);
+        return NULL;
+    }
     for (;;) {
         int64_t item = __atomic_fetch_add(&c->next_item, 1, __ATOMIC_RELAXED);
         if (item >= c->n_items) break;
         int b = (int)(item / Hkv), kv_h = (int)(item % Hkv);
         int q0 = c->cu_q[b], Lq = c->cu_q[b + 1] - c->cu_q[b];
         int k0 = c->cu_k[b], Lk = c->cu_k[b + 1] - c->cu_k[b];
+        for (int ki = 0; ki < Lk; ++ki) {
+            size_t koff = ((size_t)(k0 + ki) * Hkv + kv_h) * D;
+            bwd_widen(c, c->k, koff, D, kd + (size_t)ki * D);
+            bwd_widen(c, c->v, koff, D, vd + (size_t)ki * D);
+        }
         for (int h = kv_h * G; h < (kv_h + 1) * G; ++h) {
             for (int qi = 0; qi < Lq; ++qi) {
-                size_t qoff = ((size_t)(q0 + qi) * H + h) * D;
-                double lse = c->lse[(size_t)(q0 + qi) * H + h];
-                double delta = 0.0;
-                for (int d = 0; d < D; ++d)
-                    delta += bwd_elem(c, c->dout, qoff + d) * c->o[qoff + d];
-                for (int ki = 0; ki < Lk; ++ki) {
-                    if (c->causal && qi < ki) continue;
-                    size_t koff = ((size_t)(k0 + ki) * Hkv + kv_h) * D;
-                    double dot = 0.0;
-                    for (int d = 0; d < D; ++d)
-                        dot += bwd_elem(c, c->q, qoff + d) * bwd_elem(c, c->k, koff + d);
-                    double prob = exp(dot * c->scale - lse);
-                    double dp = 0.0;
-                    for (int d = 0; d < D; ++d)
-                        dp += bwd_elem(c, c->v, koff + d) * bwd_elem(c, c->dout, qoff + d);
-                    double ds = prob * (dp - delta);
+                const size_t qoff = ((size_t)(q0 + qi) * H + h) * D;
+                const double lse = c->lse[(size_t)(q0 + qi) * H + h];
+                bwd_widen(c, c->q, qoff, D, qd);
+                bwd_widen(c, c->dout, qoff, D, dod);
+                const double delta = dot_d(dod, c->o + qoff, D);
+                const int n = bwd_visible_keys(c, qi, Lk, idx);
+                /* the row's softmax weights, dP and dS over its visible keys */
+                for (int i = 0; i < n; ++i) {
+                    const double *krow = kd + (size_t)idx[i] * D;
+                    const double *vrow = vd + (size_t)idx[i] * D;
+                    p[i] = exp(c->scale * dot_d(qd, krow, D) - lse);
+                    dp[i] = dot_d(dod, vrow, D);
+                }
+                for (int i = 0; i < n; ++i) ds[i] = p[i] * (dp[i] - delta);
+                /* dQ of the row: one weighted sum of key rows */
+                for (int d = 0; d < D; ++d) {
+                    double acc = 0.0;
+                    for (int i = 0; i < n; ++i) acc += ds[i] * kd[(size_t)idx[i] * D + d];
+                    c->dq[qoff + d] = c->scale * acc;
+                }
+                /* the row's contributions to dK and dV of its visible keys */
+                for (int i = 0; i < n; ++i) {
+                    double *dk_row = c->dk + ((size_t)(k0 + idx[i]) * Hkv + kv_h) * D;
+                    double *dv_row = c->dv + ((size_t)(k0 + idx[i]) * Hkv + kv_h) * D;
                     for (int d = 0; d < D; ++d) {
-                        c->dq[qoff + d] += c->scale * ds * bwd_elem(c, c->k, koff + d);
-                        c->dk[koff + d] += c->scale * ds * bwd_elem(c, c->q, qoff + d);
-                        c->dv[koff + d] += prob * bwd_elem(c, c->dout, qoff + d);
+                        dk_row[d] += c->scale * ds[i] * qd[d];
+                        dv_row[d] += p[i] * dod[d];
                     }
                 }
             }
         }
     }
+    free(kd); free(vd); free(p); free(dp); free(ds); free(idx); free(qd); free(dod);
     return NULL;
 }
 

@@ -1,5 +1,6 @@
-"""Pins of the oracle's backward (the CPU backward loop of boostr 0.2.0,
-src/ops/cpu/attention/varlen_attention.rs, varlen_attention_bwd, in fp64).
+"""Pins of the oracle's backward (the gradient that the boostr 0.2.0 source
+page src/ops/cpu/attention/varlen_attention.rs defines in varlen_attention_bwd,
+in fp64).
 
 The references here do not share its arithmetic: PyTorch autograd through an
 independent dense fp64 forward (block-diagonal + causal mask), central finite
@@ -154,18 +155,14 @@ def test_dv_rows_sum_to_dout_sums():
 
 
 MUTANTS = {
-    "delta_dropped": ("                double ds = prob * (dp - delta);",
-                      "                double ds = prob * dp;"),
-    "dq_without_scale": ("                        c->dq[qoff + d] += c->scale * ds * ",
-                         "                        c->dq[qoff + d] += ds * "),
-    "dk_uses_k": ("c->dk[koff + d] += c->scale * ds * bwd_elem(c, c->q, qoff + d);",
-                  "c->dk[koff + d] += c->scale * ds * bwd_elem(c, c->k, koff + d);"),
-    "dv_uses_ds": ("                        c->dv[koff + d] += prob * ",
-                   "                        c->dv[koff + d] += ds * "),
-    "causal_ignored": ("                    if (c->causal && qi < ki) continue;",
-                       "                    if (0) continue;"),
-    "lse_not_subtracted": ("double prob = exp(dot * c->scale - lse);",
-                           "double prob = exp(dot * c->scale);"),
+    "delta_dropped": ("ds[i] = p[i] * (dp[i] - delta);", "ds[i] = p[i] * dp[i];"),
+    "dq_without_scale": ("c->dq[qoff + d] = c->scale * acc;", "c->dq[qoff + d] = acc;"),
+    "dk_uses_k": ("dk_row[d] += c->scale * ds[i] * qd[d];",
+                  "dk_row[d] += c->scale * ds[i] * kd[(size_t)idx[i] * D + d];"),
+    "dv_uses_ds": ("dv_row[d] += p[i] * dod[d];", "dv_row[d] += ds[i] * dod[d];"),
+    "causal_ignored": ("if (c->causal && qi < ki) continue;", "if (0) continue;"),
+    "lse_not_subtracted": ("p[i] = exp(c->scale * dot_d(qd, krow, D) - lse);",
+                           "p[i] = exp(c->scale * dot_d(qd, krow, D));"),
 }
 
 

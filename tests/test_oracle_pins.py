@@ -1,8 +1,8 @@
 """Pins of the fp64 oracle against facts that do not come from the oracle.
 
-The oracle restates the CPU forward loop of boostr 0.2.0,
-src/ops/cpu/attention/varlen_attention.rs (``varlen_attention_fwd``).  These
-tests tie it to: exact format decoding, the dense brute-force definition, a
+The oracle computes the packed attention forward defined by the boostr 0.2.0
+source page src/ops/cpu/attention/varlen_attention.rs
+(``varlen_attention_fwd``).  These tests tie it to: exact format decoding, the dense brute-force definition, a
 library softmax, closed forms (single key, equal scores, two keys), the
 causal rule (one-hot values), packing/permutation/GQA invariances, convexity,
 the log-sum-exp definition and the empty cases.  ``test_planted_mistakes``
@@ -265,9 +265,9 @@ def test_empty_key_set_and_empty_query():
 MUTANTS = {
     "causal_off_by_one": ("if (c->causal && qi < ki) return 1;", "if (c->causal && qi <= ki) return 1;"),
     "gqa_map_modulo": ("int kv_h = h / G;\n        int q0", "int kv_h = h % G;\n        int q0"),
-    "dropped_scale": ("double s = dot * c->scale;", "double s = dot;"),
-    "lse_without_max": ("*lse_out = max_score + log(sum_exp);", "*lse_out = log(sum_exp);"),
-    "unnormalised_weights": ("double weight = scores[ki] / sum_exp;", "double weight = scores[ki];"),
+    "dropped_scale": ("s[i] = c->scale * dot_d(qrow,", "s[i] = dot_d(qrow,"),
+    "lse_without_max": ("return m + log(acc);", "return log(acc);"),
+    "unnormalised_weights": ("const double w = exp(s[i] - lse);", "const double w = exp(s[i]);"),
     "k_v_swapped": ("kd[(size_t)ki * D + d] = oracle_decode16(c->k[off + d], c->dtype);",
                     "kd[(size_t)ki * D + d] = oracle_decode16(c->v[off + d], c->dtype);"),
     "fp16_bias_wrong": ("expo - 25", "expo - 24"),

@@ -111,9 +111,8 @@ def test_rows_mode_with_sinks():
 
 
 MUTANTS = {
-    "sink_left_out_of_sum": ("    sum_exp += exp(sink - max_score);", "    (void)0;"),
-    "sink_left_out_of_max": ("    if (sink > max_score) max_score = sink;",
-                             "    if (0) max_score = sink;"),
+    "sink_left_out_of_sum": ("    double acc = exp(extra - m);", "    double acc = 0.0;"),
+    "sink_left_out_of_max": ("    double m = extra;", "    double m = -INFINITY;"),
     "sink_scaled": ("    return c->sinks ? c->sinks[h] : -INFINITY;",
                     "    return c->sinks ? c->sinks[h] * c->scale : -INFINITY;"),
     "sink_of_wrong_head": ("    return c->sinks ? c->sinks[h] : -INFINITY;",
