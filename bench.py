@@ -11,7 +11,12 @@ TFLOP/s with FLOPs = 4 * D * (unmasked query-key pairs summed over heads).
 
 Prints ONE JSON line on rank 0.  With N > 1 (launched by torchrun) every rank
 runs its own batch of the workload (weak scaling, no collective on the data
-path); the time is the max over ranks.
+path); with ``--shard kv_heads|sequences|auto`` the ranks instead split ONE
+batch (strong scaling): by key/value-head groups (each rank holds contiguous
+head slices, the tensor-parallel layout) or by sequences balanced by
+unmasked pairs, as ``varlen_attn_plan_shards`` plans it.  The forward has no
+exchange step, so no collective touches the data path either way; the time
+is the max over ranks.
 """
 from __future__ import annotations
 
@@ -310,9 +315,32 @@ def max_over_ranks(values, dist, device):
     return [float(x) for x in t.tolist()]
 
 
+def sum_over_ranks(values, dist, device):
+    """Element-wise sum of per-rank counts (every rank calls it)."""
+    import torch
+    t = torch.tensor([int(v) for v in values], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [int(x) for x in t.tolist()]
+
+
 def whole_job_tflops(world: int, flops_per_rank_step: int, ms_per_step: float) -> float:
     """Aggregate throughput: every rank processes one batch per step."""
     return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
+def shard_for_rank(case, args, rank: int, world: int):
+    """Strong scaling (``--shard``): the rank's part of the one batch, and the
+    plan.  Weak scaling: the whole batch, no plan."""
+    if args.shard == "none" or world == 1:
+        return case, None
+    import flash_attention_fwd_b200 as fa
+    m = case.mask
+    plan = fa.plan_shards(case.cu_q.tolist(), case.cu_k.tolist(), case.H, case.Hkv, world,
+                          args.shard, causal=case.causal,
+                          window_size_left=m.get("window_left", -1),
+                          window_size_right=m.get("window_right", -1),
+                          seqused_k=m.get("seqused_k"))
+    return workloads.shard_case(case, plan, rank), plan
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -334,8 +362,11 @@ def run_gpu(args, rank: int, world: int):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    case = workloads.make_workload(args.workload)
+    full_case = workloads.make_workload(args.workload)
+    case, plan = shard_for_rank(full_case, args, rank, world)
     flops = step_flops(case)
+    args.job_flops = step_flops(full_case) if plan else world * flops
+    args.plan = plan
     wl = workloads.WORKLOADS[args.workload]
     table_t = None
     if wl.page_size:
@@ -430,9 +461,10 @@ def run_gpu(args, rank: int, world: int):
 
     if dist:
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
+        h2d, d2h = sum_over_ranks([h2d, d2h], dist, dev)
         dist.barrier()
-    emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk,
-         launches_per_step=2 if ws is not None else 1)
+    emit(args, rank, world, full_case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk,
+         launches_per_step=2 if ws is not None else 1, rank_case=case)
     if dist:
         dist.destroy_process_group()
 
@@ -513,11 +545,29 @@ def hbm_line(case, avg_launch_ms: float, peaks: dict, peak_src: str, traffic_key
             "peak_source": "%s copy bandwidth" % peak_src}
 
 
+def parallelism_note(world: int, plan) -> str:
+    if plan is None:
+        return "dp%d (one independent batch per GPU)" % world
+    if plan["mode"] == "kv_heads":
+        return ("one batch split over %d GPUs by key/value-head groups %s (contiguous head "
+                "slices per GPU; no collective)" % (world, plan["kv_heads"]))
+    return ("one batch split over %d GPUs by sequences, balanced by unmasked pairs %s "
+            "(no collective)" % (world, plan["pairs"]))
+
+
 def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk,
-         metric=METRIC, cpu_fn=None, launches_per_step=1, traffic_key=None):
+         metric=METRIC, cpu_fn=None, launches_per_step=1, traffic_key=None, rank_case=None):
+    """One JSON line on rank 0.  ``case`` is the whole batch, ``flops`` and
+    ``per_launch`` are rank 0's (its shard's, with --shard); the whole-job
+    value divides the job's FLOPs per step (args.job_flops: every rank's
+    batch, or the one batch that the ranks split) by the max-over-ranks time.
+    h2d / d2h are whole-job bytes per step."""
     if rank == 0:
         ms = total_ms / args.steps
-        value = whole_job_tflops(world, flops, ms)
+        job_flops = getattr(args, "job_flops", None) or world * flops
+        plan = getattr(args, "plan", None)
+        value = job_flops / (ms * 1e-3) / 1e12
+        rcase = rank_case if rank_case is not None else case
         peaks, peak_src = load_peaks()
         peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
         peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -535,7 +585,8 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
         line = {
             "metric": metric, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if plan else "weak",
+            "vs_baseline": None,
             "dtype": case.dtype, "data": "synthetic (seeded N(0,1) Q/K/V, seeded lengths)",
             "config": {
                 "workload": workloads.WORKLOADS[args.workload].description,
@@ -548,20 +599,21 @@ def emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h,
                 "sinks": "sinks" in case.mask,
                 "num_splits": getattr(args, "num_splits", 1),
                 "workspace_bytes": getattr(args, "workspace_bytes", 0),
-                "l2": getattr(args, "l2", l2_note(case)),
-                "parallelism": "dp%d (one independent batch per GPU)" % world},
+                "l2": getattr(args, "l2", l2_note(rcase)),
+                "parallelism": parallelism_note(world, plan),
+                "job_flops_per_step": job_flops},
             "pct_of_peak": round(100.0 * achieved / peak, 2),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic_for(traffic_key or args.workload),
                          "peak_source": "%s burst bf16 (sustained %.1f -> frac %.4f)"
                                         % (peak_src, peak_sus, achieved / peak_sus)},
-            "hbm": hbm_line(case, avg_launch_ms, peaks, peak_src, traffic_key or args.workload,
+            "hbm": hbm_line(rcase, avg_launch_ms, peaks, peak_src, traffic_key or args.workload,
                             flops),
             "launch_ms": {"min": round(min(per_launch), 4),
                           "median": round(statistics.median(per_launch), 4),
                           "max": round(max(per_launch), 4)},
-            "e2e": {"value": round(whole_job_tflops(world, flops, e2e_ms), 3), "unit": UNIT,
+            "e2e": {"value": round(job_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 3),
                     "schedule": "every step copies all its inputs from pinned host memory and "
@@ -700,6 +752,7 @@ def run_gpu_bwd(args, rank: int, world: int):
                                max(2, min(args.steps, 6)), stream, dist)
     if dist:
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
+        h2d, d2h = sum_over_ranks([h2d, d2h], dist, dev)
         dist.barrier()
     emit(args, rank, world, case, flops, total_ms, per_launch, e2e_ms, h2d, d2h, clk,
          metric=METRIC_BWD, cpu_fn=lambda: time_oracle_bwd(case, args.cpu_seconds),
@@ -802,9 +855,14 @@ def main(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--shard", default="none", choices=["none", "auto", "kv_heads", "sequences"],
+                    help="N > 1: split one batch over the GPUs (strong scaling) instead of one "
+                         "batch per GPU (weak scaling, the default)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.pass_ == "bwd" and args.shard != "none":
+        ap.error("--shard applies to the forward")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
     if args.impl == "reference":

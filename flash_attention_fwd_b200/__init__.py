@@ -49,6 +49,7 @@ EXPORTED_SYMBOLS = (
     "varlen_attn_bwd_workspace_size",
     "varlen_attn_bwd_v1",
     "varlen_attn_bwd_noalloc",
+    "varlen_attn_plan_shards",
 )
 
 _lock = threading.Lock()
@@ -98,6 +99,9 @@ def _bind(lib):
     lib.varlen_attn_bwd_v1.restype = i32
     lib.varlen_attn_bwd_noalloc.argtypes = lib.varlen_attn_bwd_v1.argtypes[:22] + [P]
     lib.varlen_attn_bwd_noalloc.restype = i32
+    lib.varlen_attn_plan_shards.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, P,
+                                            P, P, P]
+    lib.varlen_attn_plan_shards.restype = i32
     return lib
 
 
@@ -438,3 +442,41 @@ def varlen_attn_bwd_noalloc(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor
             total_k, int(max_seqlen_q), int(max_seqlen_k), H, Hkv, D, int(bool(causal)),
             0.0 if scale is None else float(scale), DTYPE_CODES[q.dtype], V(addr(dq)),
             V(addr(dk)), V(addr(dv)), V(stream.cuda_stream))
+
+
+SHARD_AUTO, SHARD_KV_HEADS, SHARD_SEQUENCES = 0, 1, 2
+SHARD_MODES = {"auto": SHARD_AUTO, "kv_heads": SHARD_KV_HEADS, "sequences": SHARD_SEQUENCES}
+
+
+def plan_shards(cu_seqlens_q, cu_seqlens_k, num_heads: int, num_kv_heads: int, world: int,
+                mode: str = "auto", causal: bool = False, window_size_left: int = -1,
+                window_size_right: int = -1, seqused_k=None) -> dict:
+    """Split of one packed batch over ``world`` GPUs with no exchange
+    (varlen_attn_plan_shards, a host-only call).  cu_seqlens_q/k: host
+    sequences of B+1 ints; ``mode`` "auto", "kv_heads" or "sequences".
+    Returns {"mode", "seq_rank" (B ints, -1 = every rank), "kv_heads"
+    (per rank (lo, hi)), "pairs" (per rank)}."""
+    import numpy as np
+    cq = np.ascontiguousarray(np.asarray(cu_seqlens_q, dtype=np.int32))
+    ck = np.ascontiguousarray(np.asarray(cu_seqlens_k, dtype=np.int32))
+    B = cq.shape[0] - 1
+    if ck.shape[0] != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B+1 entries")
+    used = None if seqused_k is None else np.ascontiguousarray(np.asarray(seqused_k,
+                                                                          dtype=np.int32))
+    seq_rank = np.zeros(max(B, 1), dtype=np.int32)
+    lo = np.zeros(world, dtype=np.int32)
+    hi = np.zeros(world, dtype=np.int32)
+    pairs = np.zeros(world, dtype=np.int64)
+    P = ctypes.c_void_p
+    rc = load_library(build_if_missing=False).varlen_attn_plan_shards(
+        P(cq.ctypes.data), P(ck.ctypes.data), P(used.ctypes.data if used is not None else 0),
+        int(B), int(num_heads), int(num_kv_heads), int(bool(causal)), int(window_size_left),
+        int(window_size_right), int(world), int(SHARD_MODES[mode]), P(seq_rank.ctypes.data),
+        P(lo.ctypes.data), P(hi.ctypes.data), P(pairs.ctypes.data))
+    if rc < 0:
+        raise VarlenAttnError(rc, strerror(rc))
+    return {"mode": {SHARD_KV_HEADS: "kv_heads", SHARD_SEQUENCES: "sequences"}[rc],
+            "seq_rank": [int(x) for x in seq_rank[:B]],
+            "kv_heads": [(int(a), int(b)) for a, b in zip(lo, hi)],
+            "pairs": [int(x) for x in pairs]}

@@ -16,7 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libvarlen_attn.so")
-SOURCES = [os.path.join(CSRC, "varlen_attn_fwd.cu")]
+SOURCES = [os.path.join(CSRC, "varlen_attn_fwd.cu"), os.path.join(CSRC, "shard_plan.cpp")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
     os.path.join(INCLUDE, "varlen_attn.h")]
 

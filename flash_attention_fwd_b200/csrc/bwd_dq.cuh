@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t rs = 0, rph = 0, q_count = 0;
     bool ok = true;
     KVProducer<BN, D, NSLOT> kv;
-    kv.init(sKV, bars->full, bars->empty, abort_flag);
+    kv.init(sKV, bars->full, bars->empty, nullptr, abort_flag);
     for (;;) {
       WorkItem w;
       const bool have = sched.next(w, p);

@@ -19,13 +19,9 @@ namespace vattn {
 template <class Kernel>
 static int launch_bwd_kernel(Kernel kernel, size_t smem, int threads, const CUtensorMap &t0,
                              const CUtensorMap &t1, const CUtensorMap &t2, const CUtensorMap &t3,
-                             const BwdParams &bp, int grid, cudaStream_t stream, bool &attr_set) {
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return VARLEN_ERR_LAUNCH;
-    attr_set = true;
-  }
+                             const BwdParams &bp, int grid, cudaStream_t stream, DeviceInfo &dev,
+                             int slot) {
+  if (const int rc = prepare_kernel(kernel, smem, dev, slot)) return rc;
   kernel<<<grid, threads, smem, stream>>>(t0, t1, t2, t3, bp);
   return cudaGetLastError() == cudaSuccess ? VARLEN_OK : VARLEN_ERR_LAUNCH;
 }
@@ -40,11 +36,10 @@ static int launch_bwd(const CUtensorMap (&m_dq)[4], const CUtensorMap (&m_kv)[4]
   int rc = VARLEN_OK;
   if (run_dq)
     rc = launch_bwd_kernel(bwd_dq::dq_kernel<D, BF16>, smem_q, bwd_dq::NUM_THREADS, m_dq[0],
-                           m_dq[1], m_dq[2], m_dq[3], bp, grid_q, s, dev.attr_set[slot]);
+                           m_dq[1], m_dq[2], m_dq[3], bp, grid_q, s, dev, slot);
   if (rc == VARLEN_OK && run_dkdv)
     rc = launch_bwd_kernel(bwd_dkdv::dkdv_kernel<D, BF16>, smem_k, bwd_dkdv::NUM_THREADS,
-                           m_kv[0], m_kv[1], m_kv[2], m_kv[3], bp, grid_k, s,
-                           dev.attr_set[slot + 1]);
+                           m_kv[0], m_kv[1], m_kv[2], m_kv[3], bp, grid_k, s, dev, slot + 1);
   return rc;
 }
 
@@ -105,20 +100,9 @@ extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k
     return VARLEN_ERR_WORKSPACE;
   if (batch == 0 || (total_q == 0 && total_k == 0)) return VARLEN_OK;
 
-  int dev_id = 0;
-  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= 64)
-    return VARLEN_ERR_LAUNCH;
-  DeviceInfo &dev = g_dev[dev_id];
-  if (dev.sms == 0) {
-    int sms = 0, mj = 0, mn = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id) != cudaSuccess ||
-        cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, dev_id) != cudaSuccess ||
-        cudaDeviceGetAttribute(&mn, cudaDevAttrComputeCapabilityMinor, dev_id) != cudaSuccess)
-      return VARLEN_ERR_LAUNCH;
-    dev.major = mj;
-    dev.minor = mn;
-    dev.sms = sms;
-  }
+  DeviceInfo *devp = nullptr;
+  if (const int rc = device_state(devp)) return rc;
+  DeviceInfo &dev = *devp;
   if (dev.major != 10 || dev.minor != 0) return VARLEN_ERR_ARCH;
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return VARLEN_ERR_LAUNCH;
@@ -198,15 +182,16 @@ extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k
 // [total_q, H]) in a fixed file-scope device array instead of a caller
 // workspace.  NOALLOC_SCRATCH_BYTES bounds total_q * H * 4 (16 MiB: 4,194,304
 // (token, head) rows, e.g. 65,536 tokens x 64 heads).  The array's device
-// address is looked up once per device, on the first call, and cached.
-// Nothing in the scratch has to start at zero: every delta the dK/dV pass
-// reads is written by the dQ pass of the same call.  All calls on a device
-// share the array, so calls that overlap in time (other streams, other host
-// threads) race on it.
+// address is looked up with cudaGetSymbolAddress on the first call in each
+// CUDA context (with the device current) and kept with the device's other
+// per-context state, so a device reset leads to a fresh lookup.  Nothing in
+// the scratch has to start at zero: every delta the dK/dV pass reads is
+// written by the dQ pass of the same call.  All calls on a device share the
+// array, so calls that overlap in time (other streams, other host threads)
+// race on it.
 namespace vattn {
 constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_bwd_scratch[NOALLOC_SCRATCH_BYTES];
-static void *g_bwd_scratch_addr[64];
 }  // namespace vattn
 
 extern "C" int varlen_attn_bwd_noalloc(const void *dout, const void *q, const void *k,
@@ -225,17 +210,21 @@ extern "C" int varlen_attn_bwd_noalloc(const void *dout, const void *q, const vo
   if (varlen_attn_bwd_workspace_size(total_q, num_heads) > NOALLOC_SCRATCH_BYTES)
     return VARLEN_ERR_WORKSPACE;
   if (batch == 0 || (total_q == 0 && total_k == 0)) return VARLEN_OK;
-  int dev_id = 0;
-  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= 64)
-    return VARLEN_ERR_LAUNCH;
-  if (!g_bwd_scratch_addr[dev_id]) {
-    void *addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_bwd_scratch) != cudaSuccess || !addr)
-      return VARLEN_ERR_LAUNCH;
-    g_bwd_scratch_addr[dev_id] = addr;
+  DeviceInfo *devp = nullptr;
+  if ((rc = device_state(devp)) != VARLEN_OK) return rc;
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(devp->mu);
+    if (!devp->bwd_scratch) {
+      void *addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, g_bwd_scratch) != cudaSuccess || !addr)
+        return VARLEN_ERR_LAUNCH;
+      devp->bwd_scratch = addr;
+    }
+    scratch = devp->bwd_scratch;
   }
   return varlen_attn_bwd_v1(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q,
                             total_k, max_seqlen_q, max_seqlen_k, num_heads, num_kv_heads,
-                            head_dim, causal, scale, dtype, dq, dk, dv,
-                            g_bwd_scratch_addr[dev_id], NOALLOC_SCRATCH_BYTES, stream);
+                            head_dim, causal, scale, dtype, dq, dk, dv, scratch,
+                            NOALLOC_SCRATCH_BYTES, stream);
 }

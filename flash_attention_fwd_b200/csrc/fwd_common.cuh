@@ -399,6 +399,20 @@ struct Scheduler {
   }
 };
 
+// Keys of the item's last visited key tile (of BN keys) that lie inside the
+// sequence's used keys (at least 1); the tile's other rows hold whatever
+// follows them in the buffer (the next sequence, unused cache slots, the rest
+// of a page).  The PV product of that tile runs over the 16-key steps that
+// hold used keys only, so just the rows from the last used key to the end of
+// its 16-key step need clearing (none when the count is a multiple of 16).
+template <int BN>
+__device__ __forceinline__ int last_tile_keys(const WorkItem &w) {
+  return min(BN, w.Lk - (w.kofs + (w.n_kv - 1) * BN));
+}
+__device__ __forceinline__ bool tail_needs_fix(int keys) { return (keys & 15) != 0; }
+// 16-key steps of a PV product over a tile with `keys` used keys
+__device__ __forceinline__ int pv_steps(int keys) { return (keys + 15) >> 4; }
+
 // Work items travel from the scheduling (producer) warp to the other roles
 // through a small ring in shared memory.  An item with hu < 0 ends the list.
 constexpr int ITEM_RING = 4;
@@ -457,28 +471,75 @@ __device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
 // With SPLIT > 1 a slot holds one D-wide column slice of a key tile (the
 // tensor's head dim is SPLIT * D) and a tile takes SPLIT consecutive slots,
 // slice 0 first.
+//
+// Rows past the used keys.  The last key tile of an item may run past the
+// sequence's used keys (into the next sequence's rows, the unused slots of a
+// KV cache, or the rest of a page).  Their scores are masked, so P is 0
+// there, but 0 times a non-finite value is NaN.  The PV product of that tile
+// skips the 16-key steps past the used keys; once the last V tile has landed,
+// the warp overwrites the remaining rows of the last used step (from the last
+// used key to the step's end, at most 15) with zeros and then arrives on
+// `vfix`, which the MMA warp waits for before that tile's PV product.  The
+// fix is deferred until the next item's first K tile and Q tile are queued,
+// so that the wait for the V tile to land does not hold up the next item's
+// loads (and the slots it needs never wait on the fix).
 template <int BN, int D, int NSLOT, int SPLIT = 1>
 struct KVProducer {
   static constexpr int DB = D / 64;
   static constexpr uint32_t KV_BYTES = BN * D * 2;
   uint8_t *sKV;
-  uint64_t *full, *empty;
+  uint64_t *full, *empty, *vfix;
   volatile int *abort_flag;
   uint64_t pol;
   uint32_t slot, phase;
   uint32_t fills[NSLOT];
   int lane;
+  // pending tail fix: first ring slot and phase of the last V tile, and the
+  // number of its rows that hold used keys (BN or a multiple of 16: nothing
+  // to fix)
+  uint32_t fix_slot, fix_phase;
+  int fix_keys;
 
-  __device__ void init(uint8_t *s, uint64_t *f, uint64_t *e, volatile int *abort) {
+  __device__ void init(uint8_t *s, uint64_t *f, uint64_t *e, uint64_t *vf,
+                       volatile int *abort) {
     sKV = s;
     full = f;
     empty = e;
+    vfix = vf;
     abort_flag = abort;
     pol = ptx::policy_evict_last();
     slot = 0;
     phase = 0;
     for (int i = 0; i < NSLOT; ++i) fills[i] = 0;
     lane = threadIdx.x & 31;
+    fix_keys = BN;
+  }
+  // Whole warp: zero the rows [fix_keys, round_up(fix_keys, 16)) of the
+  // pending last V tile once it has landed, then signal vfix.  False when the
+  // wait gave up.
+  __device__ bool fix_tail() {
+    if (!tail_needs_fix(fix_keys)) return true;
+    const int keys = fix_keys;
+    fix_keys = BN;
+    uint32_t s = fix_slot, ph = fix_phase;
+#pragma unroll
+    for (int i = 0; i < SPLIT; ++i) {
+      if (!__all_sync(0xffffffffu, wait_bar(&full[s], ph, abort_flag))) return false;
+      const int per_block = (16 - (keys & 15)) * 8;  // 16-byte chunks of one column block
+      for (int c = lane; c < DB * per_block; c += 32) {
+        const int db = c / per_block;
+        uint4 *dst = reinterpret_cast<uint4 *>(sKV + s * KV_BYTES + db * (BN * 128) + keys * 128);
+        dst[c - db * per_block] = make_uint4(0u, 0u, 0u, 0u);
+      }
+      if (++s == NSLOT) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    ptx::fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(vfix);
+    return true;
   }
   __device__ void advance() {
     ++fills[slot];
@@ -550,24 +611,41 @@ struct KVProducer {
       if (!load_paged(tm, kv_h, my_row, ch, s * D)) return false;
     return true;
   }
+  // Records the ring position of the item's last V tile (about to be
+  // loaded) when some of its rows lie past the used keys.
+  __device__ void note_tail(const WorkItem &w) {
+    fix_keys = last_tile_keys<BN>(w);
+    fix_slot = slot;
+    fix_phase = phase;
+  }
   // Whole warp: the K/V tiles of one item in the order the MMA warp consumes
   // them (K0, K1, V0, K2, V1, K3, ..., V(n-1)), with the item's Q tile(s) after
   // K0 through load_q (called by lane 0, returns false when a wait gave up).
+  // The previous item's pending tail fix runs right after the Q load.
   template <class LoadQ>
   __device__ bool load_item(const KParams &p, const WorkItem &w, int kv_h, const CUtensorMap *tm_k,
                             const CUtensorMap *tm_v, LoadQ &&load_q) {
     const int n = w.n_kv;
     if (p.page_table == nullptr) {
       bool ok = true;
+      if (lane == 0) ok = tile_packed(tm_k, kv_h, w.k0) && load_q();
+      ok = __shfl_sync(0xffffffffu, ok, 0) && fix_tail();
       if (lane == 0) {
-        ok = tile_packed(tm_k, kv_h, w.k0) && load_q();
         if (ok && n >= 2) ok = tile_packed(tm_k, kv_h, w.k0 + BN);
         for (int j = 0; ok && j < n; ++j) {
+          if (j == n - 1) note_tail(w);
           ok = tile_packed(tm_v, kv_h, w.k0 + j * BN);
           if (ok && j + 2 < n) ok = tile_packed(tm_k, kv_h, w.k0 + (j + 2) * BN);
         }
       }
-      return __shfl_sync(0xffffffffu, ok, 0);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      fix_keys = __shfl_sync(0xffffffffu, fix_keys, 0);
+      fix_slot = __shfl_sync(0xffffffffu, fix_slot, 0);
+      fix_phase = __shfl_sync(0xffffffffu, fix_phase, 0);
+      // lane 0 advanced the ring for the whole warp
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      phase = __shfl_sync(0xffffffffu, phase, 0);
+      return ok;
     }
     const int ch = p.page_chunk;
     int r0 = chunk_row(p, w, w.kofs), r1 = 0;
@@ -575,7 +653,7 @@ struct KVProducer {
     if (ok) {
       bool q = true;
       if (lane == 0) q = load_q();
-      ok = __shfl_sync(0xffffffffu, q, 0);
+      ok = __shfl_sync(0xffffffffu, q, 0) && fix_tail();
     }
     if (ok && n >= 2) {
       r1 = chunk_row(p, w, w.kofs + BN);
@@ -584,6 +662,7 @@ struct KVProducer {
     for (int j = 0; ok && j < n; ++j) {
       // look up K(j+2) before waiting for V(j)'s slot, so that the two overlap
       const int rn = (j + 2 < n) ? chunk_row(p, w, w.kofs + (j + 2) * BN) : 0;
+      if (j == n - 1) note_tail(w);
       ok = tile_paged(tm_v, kv_h, (j & 1) ? r1 : r0, ch);
       if (ok && j + 2 < n) {
         if (j & 1)
@@ -647,51 +726,6 @@ __device__ __forceinline__ void tmem_st<64>(uint32_t taddr, const uint32_t (&r)[
   ptx::tmem_st_x64(taddr, r);
 }
 
-// ---------------------------------------------------------------------------
-// Software 2^x for the two lanes of a packed pair, used for a share of the
-// softmax exponentials so that the MUFU pipe is not the only unit computing
-// them.  Range reduction in the manner of Cody and Waite: x = n + f with
-// n = rint(x) (adding 1.5 * 2^23 rounds to the nearest integer) and
-// f in [-1/2, 1/2]; 2^f from a polynomial whose coefficients were fitted by a
-// Remez exchange on the relative error over [-1/2, 1/2] (degree 3: max
-// relative error 7.5e-5, below half a bf16 ulp; degree 4: 2.6e-6, below half
-// an fp16 ulp); 2^n is then added into the exponent field.  Inputs are
-// clamped below at -126 so that the exponent stays in range; the result there
-// (about 1e-38) stands in for exp of a masked (-inf) score.
-template <int DEG>
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  float x0, x1;
-  ptx::f2_unpack(x2, x0, x1);
-  const uint64_t x = ptx::f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t magic = ptx::f2_pack(12582912.f, 12582912.f);
-  const uint64_t t = ptx::f2_add(x, magic);
-  const uint64_t f = ptx::f2_sub(x, ptx::f2_sub(t, magic));
-  uint64_t p;
-  if constexpr (DEG == 3) {
-    p = ptx::f2_fma(f, ptx::f2_pack(0.0551716685295105f, 0.0551716685295105f),
-                    ptx::f2_pack(0.2426111251115799f, 0.2426111251115799f));
-    p = ptx::f2_fma(p, f, ptx::f2_pack(0.6932609677314758f, 0.6932609677314758f));
-    p = ptx::f2_fma(p, f, ptx::f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  } else {
-    p = ptx::f2_fma(f, ptx::f2_pack(0.009570102207362652f, 0.009570102207362652f),
-                    ptx::f2_pack(0.05591785907745361f, 0.05591785907745361f));
-    p = ptx::f2_fma(p, f, ptx::f2_pack(0.240247443318367f, 0.240247443318367f));
-    p = ptx::f2_fma(p, f, ptx::f2_pack(0.6931217908859253f, 0.6931217908859253f));
-    p = ptx::f2_fma(p, f, ptx::f2_pack(0.9999992847442627f, 0.9999992847442627f));
-  }
-  uint32_t t0 = (uint32_t)t, t1 = (uint32_t)(t >> 32);
-  uint32_t p0 = (uint32_t)p, p1 = (uint32_t)(p >> 32);
-  p0 += t0 << 23;  // the low bits of t hold n (two's complement)
-  p1 += t1 << 23;
-  return (uint64_t)p0 | ((uint64_t)p1 << 32);
-}
-
-// Share of the exponential pairs computed by exp2_poly2: one pair in every
-// SOFTMAX_POLY_EVERY (0 = all on the MUFU).
-#ifndef SOFTMAX_POLY_EVERY
-#define SOFTMAX_POLY_EVERY 0
-#endif
-
 // Running-max update of one row for key tile j, mx = the tile's row max in
 // log2 units (-inf when every key of the tile is hidden from the row).  m
 // stays -inf until the row has seen a visible key; the first finite max then
@@ -708,106 +742,6 @@ __device__ __forceinline__ void update_max(int j, float mx, float &m, float &alp
 // Offset added to the scaled scores before exp2: -m, or 0 while m = -inf (the
 // row has no visible key yet, every score is -inf and exp2 gives 0).
 __device__ __forceinline__ float exp_offset(float m) { return m == -INFINITY ? 0.f : -m; }
-
-// ---------------------------------------------------------------------------
-// Softmax of one S tile held in TMEM (one row per thread), written back as P
-// (bf16/fp16) over the first BN/2 columns of the same TMEM region.
-//
-// Running state per row: m = max of the scaled scores seen so far in log2
-// units (possibly stale by up to RESCALE_THRESHOLD), l = sum of exp2(x - m).
-// When a tile raises the max by more than the threshold, O (TMEM, D columns)
-// is multiplied by exp2(m_old - m_new) in place; before that `wait_o()` is
-// called by the whole warp and must guarantee that no PV MMA into O is in
-// flight.  P is written in 32-column chunks and O is rescaled after P, so
-// that the full S row, the packed P and an O chunk are never live together.
-// The row sum adds the rounded P values (what the PV MMA sees), so the
-// numerator and the denominator of O / l carry the same rounding.
-// Returns false when that wait gave up.
-template <int BN, int D, bool BF16, class WaitO>
-__device__ __forceinline__ bool softmax_tile(uint32_t tS, uint32_t tO, int j, float sl2,
-                                             bool need_mask, int lo, int hi, float &m, float &l,
-                                             WaitO &&wait_o) {
-  constexpr int POLY = SOFTMAX_POLY_EVERY;
-  constexpr int DEG = BF16 ? 3 : 4;
-  uint32_t sr[BN];
-  tmem_ld_wait<BN>(tS, sr);
-  float s[BN];
-#pragma unroll
-  for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
-  if (need_mask) {
-#pragma unroll
-    for (int c = 0; c < BN; ++c)
-      if (c < lo || c >= hi) s[c] = -INFINITY;
-  }
-  // Row max: four independent chains of three-input maxima.
-  float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-  for (int c = 4; c + 8 <= BN; c += 8) {
-    mx0 = ptx::fmax3(mx0, s[c], s[c + 1]);
-    mx1 = ptx::fmax3(mx1, s[c + 2], s[c + 3]);
-    mx2 = ptx::fmax3(mx2, s[c + 4], s[c + 5]);
-    mx3 = ptx::fmax3(mx3, s[c + 6], s[c + 7]);
-  }
-  mx0 = ptx::fmax3(mx0, s[BN - 4], s[BN - 3]);
-  mx1 = ptx::fmax3(mx1, s[BN - 2], s[BN - 1]);
-  const float mx = fmaxf(ptx::fmax3(mx0, mx1, mx2), mx3) * sl2;
-  float alpha = 1.f;
-  bool need = false;
-  update_max(j, mx, m, alpha, need);
-  const uint64_t sl2_2 = ptx::f2_pack(sl2, sl2);
-  const float negm = exp_offset(m);
-  const uint64_t negm_2 = ptx::f2_pack(negm, negm);
-  float sa = 0.f, sb = 0.f, sc = 0.f, sd = 0.f;
-#pragma unroll
-  for (int c0 = 0; c0 < BN; c0 += 32) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int c = c0 + 2 * i;
-      const uint64_t x2 = ptx::f2_fma(ptx::f2_pack(s[c], s[c + 1]), sl2_2, negm_2);
-      float p0, p1;
-      if (POLY > 0 && (i % (POLY > 0 ? POLY : 1)) == POLY - 1) {
-        ptx::f2_unpack(exp2_poly2<DEG>(x2), p0, p1);
-      } else {
-        float x0, x1;
-        ptx::f2_unpack(x2, x0, x1);
-        p0 = ptx::ex2_approx(x0);
-        p1 = ptx::ex2_approx(x1);
-      }
-      pk[i] = pack2<BF16>(p0, p1);
-      if (i & 1) {
-        sc = ptx::add_lo16<BF16>(pk[i], sc);
-        sd = ptx::add_hi16<BF16>(pk[i], sd);
-      } else {
-        sa = ptx::add_lo16<BF16>(pk[i], sa);
-        sb = ptx::add_hi16<BF16>(pk[i], sb);
-      }
-    }
-    ptx::tmem_st_x16(tS + c0 / 2, pk);
-  }
-  l = l * alpha + ((sa + sb) + (sc + sd));
-  if (__any_sync(0xffffffffu, need)) {
-    if (!__all_sync(0xffffffffu, wait_o())) return false;
-    ptx::tc_fence_after();
-    const uint64_t a2 = ptx::f2_pack(alpha, alpha);
-#pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      tmem_ld_wait<32>(tO + c0, o);
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        float o0, o1;
-        ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(__uint_as_float(o[c]), __uint_as_float(o[c + 1])), a2),
-                       o0, o1);
-        o[c] = __float_as_uint(o0);
-        o[c + 1] = __float_as_uint(o1);
-      }
-      tmem_st<32>(tO + c0, o);
-    }
-  }
-  ptx::tmem_st_wait();
-  return true;
-}
 
 // Epilogue of one row: O / l -> out (bf16/fp16, 16-byte stores), LSE -> lse.
 // A sink logit (sink_l2 > -inf, log2 units) joins the normalisation: with

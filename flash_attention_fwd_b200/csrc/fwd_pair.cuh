@@ -27,14 +27,11 @@
  * O_B (D columns each).  The MMA warp alternates between the tiles: after
  * S_A(0), S_B(0), for each key tile j it issues PV_A(j), S_A(j+1), PV_B(j),
  * S_B(j+1), so softmax A runs while the tensor cores work for tile B and vice
- * versa.  P_T(j) is handed over in PAIR_P_CHUNKS pieces and PV_T(j) is issued
- * piece by piece.  (A build option, PAIR_S_SPLIT, also computes the upper half
- * of S_T(j+1) — keys 64..127 into columns 64..127, which P does not use — as
- * soon as the softmax has read S_T(j); it measured slower and is off.)
- * Because S_T(j) (its lower half with the split) is issued after PV_T(j-1)
- * and its tcgen05.commit tracks every earlier MMA of the issuing thread, the
- * arrival of S_T(j) proves that PV_T(j-1) completed: the softmax may rescale
- * O_T in place, before its first P piece, without a further wait.
+ * versa.  P_T(j) is handed over in two pieces of 64 keys and PV_T(j) is
+ * issued piece by piece.  Because S_T(j) is issued after PV_T(j-1) and its
+ * tcgen05.commit tracks every earlier MMA of the issuing thread, the arrival
+ * of S_T(j) proves that PV_T(j-1) completed: the softmax may rescale O_T in
+ * place, before its first P piece, without a further wait.
  */
 #pragma once
 #include "fwd_common.cuh"
@@ -51,18 +48,9 @@ constexpr uint32_t REG_LOW = 120;
 constexpr uint32_t REG_HIGH = 192;
 static_assert(128 * REG_LOW + 256 * REG_HIGH == NUM_THREADS * REG_LAUNCH, "register split");
 constexpr int BN = 128;
-// P is handed to the MMA warp in NCHUNK pieces of BN / NCHUNK keys; with
-// S_SPLIT the upper half of S(j+1) is computed while the softmax runs.
-#ifndef PAIR_P_CHUNKS
-#define PAIR_P_CHUNKS 2
-#endif
-#ifndef PAIR_S_SPLIT
-#define PAIR_S_SPLIT 0
-#endif
-constexpr int NCHUNK = PAIR_P_CHUNKS;
+// P is handed to the MMA warp in NCHUNK pieces of BN / NCHUNK keys.
+constexpr int NCHUNK = 2;
 constexpr int CHUNK_KEYS = BN / NCHUNK;
-constexpr bool S_SPLIT = PAIR_S_SPLIT != 0;
-static_assert(NCHUNK == 1 || NCHUNK == 2 || NCHUNK == 4, "P chunks");
 
 template <int D>
 struct Cfg;
@@ -79,9 +67,10 @@ struct Barriers {
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t q_full, q_empty;
-  uint64_t s_full[2], s_loaded[2];  // per query tile (A, B)
+  uint64_t s_full[2];  // per query tile (A, B)
   uint64_t p_chunk[2][NCHUNK];
   uint64_t o_ready[2], o_free[2];
+  uint64_t v_fix;  // the last V tile's rows past the used keys are zeroed
   uint64_t drain;
   ItemRing ring;
   uint32_t tmem_base;
@@ -93,18 +82,16 @@ constexpr size_t smem_bytes() {
   return (size_t)2 * BM * D * 2 + (size_t)Cfg<D>::NSLOT * BN * D * 2 + sizeof(Barriers) + 1024;
 }
 
-// Softmax of one 128-key S tile with fine-grained hand-offs: `loaded()` once
-// S is in registers, `chunk_ready(c)` once P columns [16c, 16c+16) (keys
-// 32c..32c+31) are in TMEM.  O is rescaled (when the running max jumps) before
-// the first chunk is signalled.
-template <int D, bool BF16, class Loaded, class ChunkReady>
+// Softmax of one 128-key S tile with fine-grained hand-offs: `chunk_ready(c)`
+// once the packed P of keys [CHUNK_KEYS c, CHUNK_KEYS (c + 1)) (columns
+// [CHUNK_KEYS c / 2, CHUNK_KEYS (c + 1) / 2)) is in TMEM.  O is rescaled (when
+// the running max jumps) before the first chunk is signalled.
+template <int D, bool BF16, class ChunkReady>
 __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, int j, float sl2,
                                                      bool need_mask, int lo, int hi, float &m,
-                                                     float &l, Loaded &&loaded,
-                                                     ChunkReady &&chunk_ready) {
+                                                     float &l, ChunkReady &&chunk_ready) {
   uint32_t sr[BN];
   tmem_ld_wait<BN>(tS, sr);
-  loaded();
   float s[BN];
 #pragma unroll
   for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
@@ -272,7 +259,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr uint32_t O_COL0 = 2 * BN;
   static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
   constexpr uint32_t IDESC_S_FULL = ptx::idesc_f16(BM, BN, BF16, false);
-  constexpr uint32_t IDESC_S_HALF = ptx::idesc_f16(BM, BN / 2, BF16, false);
   constexpr uint32_t IDESC_PV = ptx::idesc_f16(BM, D, BF16, true);
 
   extern __shared__ uint8_t smem_raw[];
@@ -299,11 +285,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::mbar_init(&bars->q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars->s_full[i], 1);
-      ptx::mbar_init(&bars->s_loaded[i], 4);
       for (int c = 0; c < NCHUNK; ++c) ptx::mbar_init(&bars->p_chunk[i][c], 4);
       ptx::mbar_init(&bars->o_ready[i], 1);
       ptx::mbar_init(&bars->o_free[i], 4);
     }
+    ptx::mbar_init(&bars->v_fix, 1);
     ptx::mbar_init(&bars->drain, 1);
     for (int i = 0; i < ITEM_RING; ++i) {
       ptx::mbar_init(&bars->ring.full[i], 1);
@@ -344,7 +330,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t rs = 0, rph = 0, q_count = 0;
       bool ok = true;
       KVProducer<BN, D, NSLOT> kv;
-      kv.init(sKV, bars->full, bars->empty, abort_flag);
+      kv.init(sKV, bars->full, bars->empty, &bars->v_fix, abort_flag);
       // Q tiles of an item (lane 0): packed, tile t = the next (BM >> pack)
       // tokens of all query heads of kv_h; otherwise tile t = head 2u + t
       auto load_q = [&](const WorkItem &w) -> bool {
@@ -390,10 +376,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           rph ^= 1u;
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!have || !ok) break;
+        if (!ok) break;
+        if (!have) {
+          kv.fix_tail();
+          break;
+        }
         if (w.n_kv > 0) {
           const int kv_h = pack ? w.hu : (2 * w.hu) / p.group;
           ok = kv.load_item(p, w, kv_h, &tm_k, &tm_v, [&]() { return load_q(w); });
+        } else {
+          ok = kv.fix_tail();
         }
         if (!ok) break;
       }
@@ -405,7 +397,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == MMA_WARP && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       uint32_t rs = 0, rph = 0;
-      uint32_t slot = 0, phase = 0, g = 0, items = 0;
+      uint32_t slot = 0, phase = 0, g = 0, items = 0, nfix = 0;
       bool ok = true;
       const uint32_t sQ_addr = ptx::smem_u32(sQ);
       const uint32_t sKV_addr = ptx::smem_u32(sKV);
@@ -433,12 +425,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       };
       // O_t += P_t V for keys [c * CHUNK_KEYS, (c + 1) * CHUNK_KEYS) (P from
-      // TMEM, V MN-major), in steps of 16 keys
-      auto issue_pv_chunk = [&](int t, uint32_t vslot, int c, bool acc) {
+      // TMEM, V MN-major), in steps of 16 keys; steps from `steps` on (past
+      // the used keys of the item's last tile) are skipped.  Step 0 always
+      // runs, so the first product of an item still initialises O.
+      auto issue_pv_chunk = [&](int t, uint32_t vslot, int c, bool acc, int steps) {
         const uint32_t vbase = sKV_addr + vslot * KV_BYTES;
         constexpr int KS = CHUNK_KEYS / 16;
 #pragma unroll
         for (int kk = KS * c; kk < KS * c + KS; ++kk) {
+          if (kk >= steps) break;
           uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
           ptx::mma_ts(tmem + O_COL0 + t * D, tmem + t * BN + kk * 8, bdesc, IDESC_PV,
                       (acc || kk > KS * c) ? 1u : 0u);
@@ -455,6 +450,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (w.hu < 0) break;
         const int n = w.n_kv;
         if (n == 0) continue;
+        const int tail_keys = last_tile_keys<BN>(w);
         if (!(ok = wait_bar(&bars->q_full, items & 1u, abort_flag))) break;
         ptx::tc_fence_after();
         uint32_t ks;
@@ -472,18 +468,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t ks_next = 0, vs = 0;
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            if (S_SPLIT) {
-              // upper half of S_t(j+1) while the softmax works on S_t(j)
-              if (!(ok = wait_bar(&bars->s_loaded[t], par, abort_flag))) break;
-              ptx::tc_fence_after();
-              if (more) {
-                if (t == 0 && !(ok = take_slot(ks_next))) break;
-                issue_s(t, ks_next, BN / 2, IDESC_S_HALF);
-              }
-            } else if (more && t == 0 && !(ok = take_slot(ks_next))) {
-              break;
-            }
+            if (more && t == 0 && !(ok = take_slot(ks_next))) break;
             if (t == 0 && !(ok = take_slot(vs))) break;
+            if (t == 0 && j == n - 1 && tail_needs_fix(tail_keys)) {
+              // the producer has zeroed the rows past the used keys
+              if (!(ok = wait_bar(&bars->v_fix, nfix & 1u, abort_flag))) break;
+              ++nfix;
+              ptx::tc_fence_after();
+            }
             if (j == 0 && items > 0) {
               if (!(ok = wait_bar(&bars->o_free[t], (items - 1) & 1u, abort_flag))) break;
               ptx::tc_fence_after();
@@ -492,15 +484,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = 0; c < NCHUNK; ++c) {
               if (!(ok = wait_bar(&bars->p_chunk[t][c], par, abort_flag))) break;
               ptx::tc_fence_after();
-              issue_pv_chunk(t, vs, c, j > 0 || c > 0);
+              issue_pv_chunk(t, vs, c, j > 0 || c > 0, j == n - 1 ? pv_steps(tail_keys) : BN / 16);
             }
             if (!ok) break;
             if (j == n - 1) ptx::mma_commit(&bars->o_ready[t]);
             if (t == NT - 1) ptx::mma_commit(&bars->empty[vs]);
             if (more) {
-              // lower half of S_t(j+1): columns 0..63 that P_t(j) occupied
-              // (the whole of S_t(j+1) without the split)
-              issue_s(t, ks_next, 0, S_SPLIT ? IDESC_S_HALF : IDESC_S_FULL);
+              issue_s(t, ks_next, 0, IDESC_S_FULL);
               ptx::mma_commit(&bars->s_full[t]);
               if (t == NT - 1) {
                 ptx::mma_commit(&bars->empty[ks_next]);
@@ -584,12 +574,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           softmax_tile_rep<D, BF16>(tS, tO, copy, j, sl2, need_mask, lo - j * BN, hi - j * BN, m,
                                     l, [&](int c) { arrive(&bars->p_chunk[t][c]); });
         else
-          softmax_tile_chunked<D, BF16>(
-              tS, tO, j, sl2, need_mask, lo - j * BN, hi - j * BN, m, l,
-              [&]() {
-                if (S_SPLIT) arrive(&bars->s_loaded[t]);
-              },
-              [&](int c) { arrive(&bars->p_chunk[t][c]); });
+          softmax_tile_chunked<D, BF16>(tS, tO, j, sl2, need_mask, lo - j * BN, hi - j * BN, m,
+                                        l, [&](int c) { arrive(&bars->p_chunk[t][c]); });
       }
       if (!ok) break;
       g += n;

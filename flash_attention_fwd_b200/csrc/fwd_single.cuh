@@ -64,6 +64,7 @@ struct Barriers {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2];
   uint64_t pv_done, o_ready, o_free, drain;
+  uint64_t v_fix;  // the last V tile's rows past the used keys are zeroed
   uint64_t xf[4], xr[4];  // row-pair exchange, per TMEM lane quarter: value written / read
   float xch[2][BM];       // exchanged value of row r from column half h
   ItemRing ring;
@@ -111,9 +112,13 @@ struct RowSwap {
 // Softmax of one key tile over this thread's half of its columns (HB keys,
 // S at tS, packed P to tP, O columns [0, DC) at tO) for one row; the row's
 // max over the whole tile comes from the swap with the other half.  Running
-// state and rescaling as in softmax_tile: m (log2 units, possibly stale by up
-// to RESCALE_THRESHOLD) is the same in both halves, l is this half's sum of
-// the rounded P values.  Returns false when a wait gave up.
+// state: m = the row's running max of the scaled scores in log2 units (the
+// same in both halves; possibly stale by up to RESCALE_THRESHOLD), l = this
+// half's sum of the rounded P values (what the PV product sees, so O / l
+// carries one rounding).  When a tile raises m by more than the threshold, O
+// (TMEM, this half's DC columns) is multiplied by exp2(m_old - m_new) in
+// place, after `wait_o()` (called by the whole warp) has guaranteed that no
+// PV product into O is in flight.  Returns false when a wait gave up.
 template <int HB, int DC, bool BF16, class WaitO>
 __device__ __forceinline__ bool softmax_half(uint32_t tS, uint32_t tP, uint32_t tO, int j,
                                              float sl2, bool need_mask, int lo, int hi, float &m,
@@ -252,6 +257,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&bars->xr[i], 2);
     }
     ptx::mbar_init(&bars->drain, 1);
+    ptx::mbar_init(&bars->v_fix, 1);
     for (int i = 0; i < ITEM_RING; ++i) {
       ptx::mbar_init(&bars->ring.full[i], 1);
       ptx::mbar_init(&bars->ring.empty[i], RING_CONSUMERS);
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t rs = 0, rph = 0, q_count = 0;
       bool ok = true;
       KVProducer<BN, DS, NSLOT, SPLIT> kv;
-      kv.init(sKV, bars->full, bars->empty, abort_flag);
+      kv.init(sKV, bars->full, bars->empty, &bars->v_fix, abort_flag);
       // Q tile of an item (lane 0)
       auto load_q = [&](const WorkItem &w) -> bool {
         if (!wait_bar(&bars->q_empty, (q_count & 1u) ^ 1u, abort_flag)) return false;
@@ -310,9 +316,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           rph ^= 1u;
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!have || !ok) break;
+        if (!ok) break;
+        if (!have) {
+          kv.fix_tail();
+          break;
+        }
         if (w.n_kv > 0)
           ok = kv.load_item(p, w, w.hu / p.group, &tm_k, &tm_v, [&]() { return load_q(w); });
+        else
+          ok = kv.fix_tail();
         if (!ok) break;
       }
       if (lane == 0) {
@@ -325,7 +337,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t rs = 0, rph = 0;
-      uint32_t slot = 0, phase = 0, g = 0, items = 0;
+      uint32_t slot = 0, phase = 0, g = 0, items = 0, nfix = 0;
       bool ok = true;
       const uint32_t sQ_addr = ptx::smem_u32(sQ);
       const uint32_t sKV_addr = ptx::smem_u32(sKV);
@@ -364,13 +376,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       // O += P V over the BN keys in steps of 16 (P from TMEM, V MN-major);
       // slice i of V feeds O's columns [i * DS, (i + 1) * DS) and its slot is
-      // released right after its MMAs
-      auto issue_pv = [&](uint32_t buf, const uint32_t (&vs)[SPLIT], bool acc) {
+      // released right after its MMAs.  Steps from `steps` on (past the used
+      // keys of the item's last tile) are skipped; step 0 always runs.
+      auto issue_pv = [&](uint32_t buf, const uint32_t (&vs)[SPLIT], bool acc, int steps) {
 #pragma unroll
         for (int i = 0; i < SPLIT; ++i) {
           const uint32_t vbase = sKV_addr + vs[i] * KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
+            if (kk >= steps) break;
             uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
             ptx::mma_ts(tmem + O_COL + i * DS, tmem + buf * BN + P_COL + kk * 8, bdesc, IDESC_PV,
                         (acc || kk > 0) ? 1u : 0u);
@@ -409,7 +423,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           uint32_t vs[SPLIT];
           if (!(ok = take_tile(vs))) break;
-          issue_pv(buf, vs, j > 0);
+          const int keys = j == n - 1 ? last_tile_keys<BN>(w) : BN;
+          if (tail_needs_fix(keys)) {
+            // the producer has zeroed the rows past the used keys
+            if (!(ok = wait_bar(&bars->v_fix, nfix & 1u, abort_flag))) break;
+            ++nfix;
+            ptx::tc_fence_after();
+          }
+          issue_pv(buf, vs, j > 0, pv_steps(keys));
           ptx::mma_commit(&bars->pv_done);
           if (j == n - 1) ptx::mma_commit(&bars->o_ready);
           if (j + 2 < n) {

@@ -29,17 +29,14 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "fwd_combine.cuh"
 #include "fwd_common.cuh"
 #include "fwd_pair.cuh"
 #include "fwd_single.cuh"
 #include "varlen_attn.h"
-
-// GQA packing in the pair kernel: 0 = never, 1 = whenever H / Hkv is a power
-// of two, 2 = when the query sequences are short (see use_packing below).
-#ifndef PAIR_PACK_POLICY
-#define PAIR_PACK_POLICY 2
-#endif
 
 namespace vattn {
 
@@ -49,20 +46,39 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
+// A driver API entry point through the runtime (the library does not link
+// libcuda directly); nullptr when the driver does not provide it.
+static void *driver_entry(const char *name) {
+  void *ptr = nullptr;
+  cudaDriverEntryPointQueryResult qres;
+  if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+      qres == cudaDriverEntryPointSuccess)
+    return ptr;
+  return nullptr;
+}
+
+// Function-local statics: initialised once, thread-safely (C++11).
 static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult qres;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
-            cudaSuccess &&
-        qres == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+  static const EncodeTiledFn fn =
+      reinterpret_cast<EncodeTiledFn>(driver_entry("cuTensorMapEncodeTiled"));
   return fn;
+}
+
+// Unique id of the calling thread's current CUDA context (0 when none is
+// current yet, or the driver cannot tell).  Ids are never reused within a
+// process, so a device reset, which destroys the context, changes the id.
+static unsigned long long current_context_id() {
+  static const CtxGetCurrentFn get_cur =
+      reinterpret_cast<CtxGetCurrentFn>(driver_entry("cuCtxGetCurrent"));
+  static const CtxGetIdFn get_id = reinterpret_cast<CtxGetIdFn>(driver_entry("cuCtxGetId"));
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
 }
 
 // [rows, heads, D] row-major 16-bit tensor; box = 64 elements x box_heads
@@ -81,32 +97,81 @@ static bool encode_qkv_map(EncodeTiledFn enc, CUtensorMap *map, const void *base
   return r == CUDA_SUCCESS;
 }
 
+// Per-device state kept across calls: the SM count and compute capability,
+// which kernels have had their shared-memory limit raised, and the address
+// of the no-allocation backward's scratch array.  All of it belongs to one
+// CUDA context (function attributes and symbol addresses do not survive a
+// device reset), so it is tied to the context's unique id and set up again
+// when the calling thread's context differs.  Calls from several host
+// threads are safe: the set-up runs under the device's mutex.
+constexpr int MAX_DEVICES = 64;
+constexpr int KERNEL_SLOTS = 24;  // forward 0..9, backward 10..17, replicated rows 18..21
 struct DeviceInfo {
-  int sms = 0;
-  int major = 0, minor = 0;
-  bool attr_set[24] = {};
+  std::mutex mu;
+  std::atomic<unsigned long long> ctx_id;  // context the state below belongs to (0: none)
+  int sms, major, minor;                   // written under mu before ctx_id is published
+  std::atomic<bool> attr_set[KERNEL_SLOTS];
+  void *bwd_scratch;                       // under mu
 };
-static DeviceInfo g_dev[64];
+static DeviceInfo g_dev[MAX_DEVICES];  // static storage: zero-initialised
 
-// min_regs: the kernel rebalances registers between its warpgroups with
-// setmaxnreg and relies on the CTA having been launched with at least this
-// many registers per thread; a build that reports fewer is never launched
-// (the increase would wait for registers that do not exist).
+// The calling thread's device, its state brought up to date for the current
+// context.
+static int device_state(DeviceInfo *&dev_out) {
+  int dev_id = 0;
+  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= MAX_DEVICES)
+    return VARLEN_ERR_LAUNCH;
+  DeviceInfo &dev = g_dev[dev_id];
+  const unsigned long long id = current_context_id();
+  if (id == 0 || dev.ctx_id.load(std::memory_order_acquire) != id) {
+    std::lock_guard<std::mutex> lock(dev.mu);
+    if (id == 0 || dev.ctx_id.load(std::memory_order_relaxed) != id) {
+      int sms = 0, mj = 0, mn = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id) != cudaSuccess ||
+          cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, dev_id) != cudaSuccess ||
+          cudaDeviceGetAttribute(&mn, cudaDevAttrComputeCapabilityMinor, dev_id) != cudaSuccess)
+        return VARLEN_ERR_LAUNCH;
+      dev.sms = sms;
+      dev.major = mj;
+      dev.minor = mn;
+      for (int i = 0; i < KERNEL_SLOTS; ++i) dev.attr_set[i].store(false, std::memory_order_relaxed);
+      dev.bwd_scratch = nullptr;
+      dev.ctx_id.store(id, std::memory_order_release);
+    }
+  }
+  dev_out = &dev;
+  return VARLEN_OK;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per context.  min_regs:
+// the kernel rebalances registers between its warpgroups with setmaxnreg and
+// relies on the CTA having been launched with at least this many registers
+// per thread; a build that reports fewer is never launched (the increase
+// would wait for registers that do not exist).
+template <class Kernel>
+static int prepare_kernel(Kernel kernel, size_t smem, DeviceInfo &dev, int slot,
+                          int min_regs = 0) {
+  if (dev.attr_set[slot].load(std::memory_order_acquire)) return VARLEN_OK;
+  std::lock_guard<std::mutex> lock(dev.mu);
+  if (dev.attr_set[slot].load(std::memory_order_relaxed)) return VARLEN_OK;
+  if (min_regs > 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs < min_regs)
+      return VARLEN_ERR_LAUNCH;
+  }
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return VARLEN_ERR_LAUNCH;
+  dev.attr_set[slot].store(true, std::memory_order_release);
+  return VARLEN_OK;
+}
+
 template <class Kernel>
 static int launch_kernel(Kernel kernel, size_t smem, int threads, const CUtensorMap &tq,
                          const CUtensorMap &tk, const CUtensorMap &tv, const KParams &kp,
-                         int grid, cudaStream_t stream, bool &attr_set, int min_regs = 0) {
-  if (!attr_set) {
-    if (min_regs > 0) {
-      cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess || fa.numRegs < min_regs)
-        return VARLEN_ERR_LAUNCH;
-    }
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return VARLEN_ERR_LAUNCH;
-    attr_set = true;
-  }
+                         int grid, cudaStream_t stream, DeviceInfo &dev, int slot,
+                         int min_regs = 0) {
+  if (const int rc = prepare_kernel(kernel, smem, dev, slot, min_regs)) return rc;
   kernel<<<grid, threads, smem, stream>>>(tq, tk, tv, kp);
   return cudaGetLastError() == cudaSuccess ? VARLEN_OK : VARLEN_ERR_LAUNCH;
 }
@@ -117,7 +182,7 @@ static int launch_single(const CUtensorMap &tq, const CUtensorMap &tk, const CUt
   constexpr size_t smem = single::smem_bytes<D>();
   static_assert(smem <= 232448, "shared memory budget");
   return launch_kernel(single::fwd_kernel<D, BF16>, smem, single::NUM_THREADS, tq, tk, tv, kp,
-                       grid, s, dev.attr_set[slot]);
+                       grid, s, dev, slot);
 }
 
 template <int D, bool BF16>
@@ -129,9 +194,9 @@ static int launch_pair(const CUtensorMap &tq, const CUtensorMap &tk, const CUten
   // forward uses 0..9, the backward 10..17)
   if (kp.rep > 1)
     return launch_kernel(pair::fwd_kernel<D, BF16, true>, smem, pair::NUM_THREADS, tq, tk, tv, kp,
-                         grid, s, dev.attr_set[slot + 18], (int)pair::REG_LAUNCH);
+                         grid, s, dev, slot + 18, (int)pair::REG_LAUNCH);
   return launch_kernel(pair::fwd_kernel<D, BF16, false>, smem, pair::NUM_THREADS, tq, tk, tv, kp,
-                       grid, s, dev.attr_set[slot], (int)pair::REG_LAUNCH);
+                       grid, s, dev, slot, (int)pair::REG_LAUNCH);
 }
 
 static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -166,7 +231,7 @@ static FwdLayout fwd_layout(int max_seqlen_q, int num_heads, int num_kv_heads, i
   L.pack_log2 = 0;
   if (L.use_pair && (group & (group - 1)) == 0 && group <= BM) {
     const bool short_q = (long long)max_seqlen_q * 2 <= BM;
-    if (PAIR_PACK_POLICY == 1 || (PAIR_PACK_POLICY == 2 && short_q))
+    if (short_q)
       while ((1 << L.pack_log2) < group) ++L.pack_log2;
   }
   L.head_units = L.pack_log2 ? num_kv_heads : (L.use_pair ? num_heads / 2 : num_heads);
@@ -246,24 +311,6 @@ static size_t split_workspace_bytes(int64_t total_q, int num_heads, int D, int m
   return (size_t)max_parts * (size_t)total_q * (size_t)num_heads * (size_t)(D + 1) * 4u;
 }
 
-static int device_sms(DeviceInfo *&dev_out) {
-  int dev_id = 0;
-  if (cudaGetDevice(&dev_id) != cudaSuccess || dev_id < 0 || dev_id >= 64) return VARLEN_ERR_LAUNCH;
-  DeviceInfo &dev = g_dev[dev_id];
-  if (dev.sms == 0) {
-    int sms = 0, mj = 0, mn = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id) != cudaSuccess ||
-        cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, dev_id) != cudaSuccess ||
-        cudaDeviceGetAttribute(&mn, cudaDevAttrComputeCapabilityMinor, dev_id) != cudaSuccess)
-      return VARLEN_ERR_LAUNCH;
-    dev.major = mj;
-    dev.minor = mn;
-    dev.sms = sms;
-  }
-  dev_out = &dev;
-  return VARLEN_OK;
-}
-
 }  // namespace vattn
 
 using namespace vattn;
@@ -314,7 +361,7 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   if (batch == 0 || total_q == 0) return VARLEN_OK;
 
   DeviceInfo *devp = nullptr;
-  if (const int rc = device_sms(devp)) return rc;
+  if (const int rc = device_state(devp)) return rc;
   DeviceInfo &dev = *devp;
   if (dev.major != 10 || dev.minor != 0) return VARLEN_ERR_ARCH;
 
@@ -517,7 +564,7 @@ extern "C" int varlen_attn_fwd_num_splits(int batch, int64_t total_q, int64_t to
     return VARLEN_ERR_SHAPE;
   if (num_sms <= 0) {
     DeviceInfo *dev = nullptr;
-    if (const int rc = device_sms(dev)) return rc;
+    if (const int rc = device_state(dev)) return rc;
     num_sms = dev->sms;
   }
   const bool masked = causal || window_left >= 0 || window_right >= 0;
@@ -597,7 +644,7 @@ extern "C" int varlen_attn_device_status(unsigned int *status, int clear) {
   return VARLEN_OK;
 }
 
-extern "C" int varlen_attn_abi_version(void) { return 5; }
+extern "C" int varlen_attn_abi_version(void) { return 6; }
 
 // Backward entry points (same translation unit: one device status word).
 #include "bwd_host.cuh"

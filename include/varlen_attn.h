@@ -133,8 +133,8 @@ int varlen_attn_fwd(const void *q, const void *k, const void *v,
  *   window_left, window_right   as above (any int; negative = unbounded).
  *   seqused_k    NULL, or [batch] int32 device array (4-byte aligned); a
  *                negative entry counts as 0, an entry above Lk_b as Lk_b.
- *                Keys in [Lk_used(b), Lk_b) get weight exactly 0 but may be
- *                read, so they must hold finite values.
+ *                Keys in [Lk_used(b), Lk_b) take no part: their contents do
+ *                not matter (they may be uninitialised, NaN or infinite).
  *
  * Every other argument, the ownership and the error behaviour are those of
  * varlen_attn_fwd_v1.  A query that sees no key (possible with a window, a
@@ -178,7 +178,8 @@ int varlen_attn_fwd_v2(const void *q, const void *k, const void *v,
  * the table entries of pages holding used keys are read.  A table entry
  * outside [0, num_pages) is never dereferenced: its keys read as zeros and
  * bit 2 of the device status word is set.  The rows of a page past the used
- * keys may be read (weight exactly 0) and must hold finite values.
+ * keys, and pages no used key lives in, take no part: their contents do not
+ * matter (uninitialised, NaN or infinite values are fine).
  *
  * sinks        NULL, or a float32 device array [num_heads] (4-byte aligned):
  *              attention sinks, the FLOAT32 per-head "sinks" input of the
@@ -287,12 +288,17 @@ const char *varlen_attn_strerror(int code);
 
 /*
  * Device-side status word of the current device.  Every wait inside the
- * kernels is bounded; a wait that runs out (which does not happen in a
- * correct launch) ORs a bit into this word, the kernel drains its own
- * in-flight copies and returns instead of hanging.  Bits: 1 = pipeline wait
- * timed out; 2 = a page-table entry was outside [0, num_pages) (v3).  Reads
- * the word synchronously into *status (device-wide, shared by all launches of
- * this library on the device); clears it when clear != 0.  Returns VARLEN_OK or VARLEN_ERR_LAUNCH / VARLEN_ERR_NULL.
+ * kernels is bounded (2 s); a wait that runs out ORs a bit into this word,
+ * the kernel drains its own in-flight copies and returns instead of hanging.
+ * Bits: 1 = pipeline wait timed out; 2 = a page-table entry was outside
+ * [0, num_pages) (v3).  A launch that set a bit returned VARLEN_OK (the
+ * entry points do not wait for the kernels) and its outputs are not to be
+ * trusted: a caller that must detect this reads the word after synchronising
+ * with the launch.  A wait can run out without a fault, e.g. when a CTA is
+ * descheduled for more than the limit on a shared or time-sliced GPU.
+ * Reads the word synchronously into *status (device-wide, shared by all
+ * launches of this library on the device); clears it when clear != 0.
+ * Returns VARLEN_OK or VARLEN_ERR_LAUNCH / VARLEN_ERR_NULL.
  */
 int varlen_attn_device_status(unsigned int *status, int clear);
 
@@ -355,13 +361,13 @@ int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k, const voi
  * larger problems return VARLEN_ERR_WORKSPACE before anything is launched).
  * The pages have no counterpart: their backward allocates its buffers.
  *
- * The array's device address is looked up once per device on the first call
- * (cudaGetSymbolAddress), so the first call on each device must not be made
- * while the stream is being captured into a CUDA graph; later calls can be
- * captured.  Nothing in the scratch has to start at zero.  Every call on a
- * device uses the same array: calls that overlap in time (other streams or
- * host threads) race on it and give wrong gradients; serialise them.
- * Arguments, results and errors are otherwise those of varlen_attn_bwd_v1.
+ * The array's device address is looked up (cudaGetSymbolAddress) by the
+ * first call on each device, and again by the first call after the device's
+ * context has been reset; make that first call before any stream capture.
+ * Nothing in the scratch has to start at zero.  Every call on a device uses
+ * the same array: calls that overlap in time (other streams or host threads)
+ * race on it and give wrong gradients; serialise them.  Arguments, results
+ * and errors are otherwise those of varlen_attn_bwd_v1.
  */
 int varlen_attn_bwd_noalloc(const void *dout, const void *q, const void *k, const void *v,
                             const void *out, const float *lse,
@@ -372,7 +378,58 @@ int varlen_attn_bwd_noalloc(const void *dout, const void *q, const void *k, cons
                             int causal, float scale, varlen_dtype_t dtype,
                             void *dq, void *dk, void *dv, varlen_stream_t stream);
 
-/* Library ABI version: 5 for this header (v2, v3, v4 and the backward added; v1 unchanged). */
+/*
+ * varlen_attn_plan_shards — how to split one packed batch over `world` GPUs
+ * (one process each) with no exchange between them.  Host only: every
+ * pointer is a HOST pointer; nothing is launched or allocated on a device.
+ *
+ * The forward's units — a sequence and a key/value head with the query heads
+ * that map onto it (kv_h = h / (H / Hkv), the GQA head map of the boostr page
+ * cited above) — need nothing from one another, so a batch splits with no
+ * collective on the data path:
+ *
+ *   VARLEN_SHARD_KV_HEADS   rank r computes every sequence for key/value
+ *                heads [kv_head_lo[r], kv_head_hi[r]) and their query heads
+ *                [kv_head_lo[r] * G, kv_head_hi[r] * G) (G = H / Hkv): the
+ *                tensor-parallel layout, in which each rank holds contiguous
+ *                [T, heads_r, D] slices of q, k, v and out and calls the
+ *                forward on them with num_heads = heads_r * G and
+ *                num_kv_heads = heads_r.  The first Hkv mod world ranks take
+ *                one key/value head more.  Needs world <= num_kv_heads.
+ *   VARLEN_SHARD_SEQUENCES  rank r computes all heads of the sequences b with
+ *                seq_rank[b] == r (packed on that rank in their original
+ *                order): longest processing time first, by unmasked pairs.
+ *   VARLEN_SHARD_AUTO  whichever of the two has the smaller largest load
+ *                (key/value heads on a tie).
+ *
+ *   cu_seqlens_q, cu_seqlens_k  [batch + 1] int32 (host), non-decreasing
+ *   seqused_k    NULL or [batch] int32 (host): used keys per sequence (v2)
+ *   causal, window_left, window_right   the mask of the forward call (v2);
+ *                they only weigh the units
+ *   seq_rank     [batch] out: the rank of sequence b, -1 in the key/value
+ *                head split (every rank computes it)
+ *   kv_head_lo, kv_head_hi   [world] out: key/value heads of each rank
+ *                ([0, num_kv_heads) for every rank in the sequence split)
+ *   rank_pairs   [world] out: unmasked (query, key) pairs summed over the
+ *                query heads that rank r computes (the forward's FLOPs are
+ *                4 * head_dim * pairs)
+ *
+ * Returns the split used (VARLEN_SHARD_KV_HEADS or VARLEN_SHARD_SEQUENCES),
+ * or VARLEN_ERR_SHAPE (bad sizes, world < 1, mode unknown, a decreasing
+ * sequence table, world > num_kv_heads with VARLEN_SHARD_KV_HEADS) or
+ * VARLEN_ERR_NULL.
+ */
+#define VARLEN_SHARD_AUTO 0
+#define VARLEN_SHARD_KV_HEADS 1
+#define VARLEN_SHARD_SEQUENCES 2
+int varlen_attn_plan_shards(const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                            const int32_t *seqused_k, int batch, int num_heads, int num_kv_heads,
+                            int causal, int window_left, int window_right, int world, int mode,
+                            int32_t *seq_rank, int32_t *kv_head_lo, int32_t *kv_head_hi,
+                            int64_t *rank_pairs);
+
+/* Library ABI version: 6 for this header (v2, v3, v4, the backward and the
+ * shard planner added; v1 unchanged). */
 int varlen_attn_abi_version(void);
 
 #ifdef __cplusplus

@@ -28,7 +28,7 @@ def test_library_loads_and_exports_every_symbol():
     raw = ctypes.CDLL(fa.LIB_PATH)
     for name in header_functions():
         assert hasattr(raw, name), name
-    assert lib.varlen_attn_abi_version() == 5
+    assert lib.varlen_attn_abi_version() == 6
 
 
 def test_library_is_built_for_sm100a():

@@ -91,3 +91,25 @@ def test_committed_traffic_entries_name_known_families():
     for key, ent in d.items():
         assert ent["kernel_kind"] in bench.KERNEL_SOURCES, key
         assert len(ent["kernel_hash"]) == 16 and ent["bytes_per_launch"] > 0, key
+
+
+def test_strong_scaling_shards_add_up_to_the_batch():
+    # --shard: each rank's FLOPs (from its own shard) add up to the batch's,
+    # for both splits and with the window / used-key masks
+    import argparse
+    for name in ("gqa", "shortq_used", "long_swa"):
+        full = workloads.make_workload(name)
+        total = bench.step_flops(full)
+        for mode in ("kv_heads", "sequences"):
+            args = argparse.Namespace(shard=mode)
+            parts = []
+            for r in range(2):
+                sub, plan = bench.shard_for_rank(full, args, r, 2)
+                assert plan["mode"] == mode
+                parts.append(bench.step_flops(sub))
+                assert plan["pairs"][r] * 4 * full.D == parts[-1]
+            assert sum(parts) == total, (name, mode)
+    # one rank, or no --shard: the whole batch
+    full = workloads.make_workload("tiny")
+    sub, plan = bench.shard_for_rank(full, argparse.Namespace(shard="auto"), 0, 1)
+    assert plan is None and sub is full

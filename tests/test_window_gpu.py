@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import workloads
-from parity_helpers import check_close, full_check, require_gpu, run_gpu, sampled_check
+from parity_helpers import check_close, full_check, require_gpu, run_gpu, stratified_check
 
 pytestmark = pytest.mark.gpu
 
@@ -144,9 +144,12 @@ def test_full_seqused_equals_v1_bitwise():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-# --- a large case, sampled -------------------------------------------------------------
+# --- a large case, one oracle row per work item ---------------------------------------
 
-def test_long_prefill_sliding_window_sampled():
-    """The long ragged prefill workload with a 4096-key causal sliding window."""
-    case = workloads.make_workload("long")
-    sampled_check(case, n=600, mask=dict(window_left=4096))
+def test_long_prefill_sliding_window_stratified():
+    """The long ragged prefill workload with a 4096-key causal sliding window
+    (the bench's long_swa workload): one oracle row of every (sequence,
+    128-query tile, head)."""
+    case = workloads.make_workload("long_swa")
+    n = stratified_check(case, mask=case.mask)
+    assert n >= 33216

@@ -2,6 +2,7 @@
 import json
 import os
 
+import numpy as np
 import pytest
 import torch
 
@@ -42,3 +43,22 @@ def test_tensor_recipe_is_deterministic_and_cast():
     g = torch.Generator("cpu").manual_seed(7)
     q = (torch.randn((8, 4, 16), generator=g) * 3.0).to(torch.float16)
     assert torch.equal(q, a.q)
+
+
+def test_half_ulp_bounds_rounding_to_16_bit():
+    # the GPU tests' allowance for rounding the exact result to bf16 / fp16:
+    # every value lies within half_ulp of its rounded form, and the bound is
+    # tight (reached at midpoints between neighbours)
+    import torch
+    from parity_helpers import half_ulp
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.normal(0, 1, 20000), rng.normal(0, 50, 20000),
+                        rng.uniform(-1e-3, 1e-3, 5000)])
+    # float32 values, so that the cast to 16 bits is a single rounding
+    x = x.astype(np.float32).astype(np.float64)
+    for name, tdt in (("bf16", torch.bfloat16), ("fp16", torch.float16)):
+        r = torch.from_numpy(x).to(tdt).to(torch.float64).numpy()
+        assert np.all(np.abs(x - r) <= half_ulp(x, name))
+        one = np.array([1.0])
+        step = 2.0 ** -(7 if name == "bf16" else 10)
+        assert half_ulp(one, name)[0] == step / 2

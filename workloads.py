@@ -281,6 +281,42 @@ def sample_rows(case: Case, n: int, seed: int = 1234) -> np.ndarray:
     return arr
 
 
+def stratified_rows(case: Case, seed: int = 4321, tile: int = 128,
+                    per_tile: int = 1) -> np.ndarray:
+    """Seeded (token, head) rows of every (sequence, query tile of `tile`
+    rows, head): with per_tile = 1 one row, the tile's first, its last or a
+    random one, chosen at random; with per_tile > 1 the first and the last
+    row and per_tile - 2 random rows.  Plus the last query row of every
+    (sequence, head), whose visible keys reach the sequence's last key tile.
+    Duplicates are dropped.  Sorted by (head, token), so that rows sharing a
+    key/value head and a sequence are adjacent."""
+    rng = np.random.default_rng(seed)
+    cu = case.cu_q.tolist()
+    H = case.H
+    toks, heads = [], []
+    for b in range(case.B):
+        q0, L = cu[b], cu[b + 1] - cu[b]
+        if L <= 0:
+            continue
+        starts = np.arange(0, L, tile)
+        ends = np.minimum(starts + tile, L)
+        n_t = len(starts)
+        for i in range(per_tile):
+            kind = rng.integers(0, 3, (n_t, H)) if per_tile == 1 else np.full((n_t, H), min(i, 2))
+            rnd = starts[:, None] + (rng.random((n_t, H)) * (ends - starts)[:, None]).astype(
+                np.int64)
+            pick = np.where(kind == 0, starts[:, None],
+                            np.where(kind == 1, (ends - 1)[:, None], rnd))
+            toks.append((q0 + pick).reshape(-1))
+            heads.append(np.tile(np.arange(H), n_t))
+        toks.append(np.full(H, q0 + L - 1))
+        heads.append(np.arange(H))
+    if not toks:
+        return np.zeros((0, 2), dtype=np.int64)
+    rows = np.unique(np.stack([np.concatenate(heads), np.concatenate(toks)], axis=1), axis=0)
+    return np.ascontiguousarray(rows[:, ::-1]).astype(np.int64)
+
+
 # ----------------------------------------------------------------------------- paged K/V
 
 @dataclass
@@ -322,3 +358,70 @@ def to_paged(case: Case, page_size: int, seed: int = 0, spare_pages: int = 3,
             kc[pg, :hi - lo] = case.k[lo:hi]
             vc[pg, :hi - lo] = case.v[lo:hi]
     return PagedKV(kc, vc, table, list(case.lens_k), page_size)
+
+
+# ----------------------------------------------------------------------------- shards
+
+def shard_case(case: Case, plan: dict, rank: int) -> Case:
+    """The part of ``case`` that rank ``rank`` computes under ``plan`` (the
+    dict ``flash_attention_fwd_b200.plan_shards`` returns), laid out as that
+    rank would hold it: with the key/value-head split, contiguous head slices
+    [T, heads_r, D] of q, k, v (all sequences); with the sequence split, the
+    rank's sequences packed in their original order (all heads).  The mask
+    arguments (window, seqused_k, sinks) follow."""
+    G = case.H // case.Hkv
+    mask = dict(case.mask)
+    if plan["mode"] == "kv_heads":
+        lo, hi = plan["kv_heads"][rank]
+        q = case.q[:, lo * G:hi * G].contiguous()
+        k = case.k[:, lo:hi].contiguous()
+        v = case.v[:, lo:hi].contiguous()
+        if "sinks" in mask:
+            mask["sinks"] = list(mask["sinks"][lo * G:hi * G])
+        sub = Case(q, k, v, case.cu_q.clone(), case.cu_k.clone(), list(case.lens_q),
+                   list(case.lens_k), (hi - lo) * G, hi - lo, case.D, case.causal, case.dtype,
+                   case.scale, name="%s[kv heads %d:%d]" % (case.name, lo, hi), seed=case.seed)
+        sub.mask = mask
+        return sub
+    mine = [b for b, r in enumerate(plan["seq_rank"]) if r == rank]
+    cq, ck = case.cu_q.tolist(), case.cu_k.tolist()
+    q = torch.cat([case.q[cq[b]:cq[b + 1]] for b in mine]) if mine else case.q[:0]
+    k = torch.cat([case.k[ck[b]:ck[b + 1]] for b in mine]) if mine else case.k[:0]
+    v = torch.cat([case.v[ck[b]:ck[b + 1]] for b in mine]) if mine else case.v[:0]
+    lq = [case.lens_q[b] for b in mine]
+    lk = [case.lens_k[b] for b in mine]
+    if "seqused_k" in mask:
+        mask["seqused_k"] = [mask["seqused_k"][b] for b in mine]
+    sub = Case(q.contiguous(), k.contiguous(), v.contiguous(), cu_seqlens(lq), cu_seqlens(lk),
+               lq, lk, case.H, case.Hkv, case.D, case.causal, case.dtype, case.scale,
+               name="%s[%d sequences]" % (case.name, len(mine)), seed=case.seed)
+    sub.mask = mask
+    return sub
+
+
+def shard_rows(case: Case, plan: dict, rank: int):
+    """(token indices, query heads) of the full output that rank ``rank``'s
+    shard output covers, in the shard's own row and head order."""
+    G = case.H // case.Hkv
+    if plan["mode"] == "kv_heads":
+        lo, hi = plan["kv_heads"][rank]
+        return np.arange(case.Tq), np.arange(lo * G, hi * G)
+    cq = case.cu_q.tolist()
+    mine = [b for b, r in enumerate(plan["seq_rank"]) if r == rank]
+    toks = [np.arange(cq[b], cq[b + 1]) for b in mine]
+    return (np.concatenate(toks) if toks else np.zeros(0, dtype=np.int64)), np.arange(case.H)
+
+
+def unshard(case: Case, plan: dict, parts) -> tuple:
+    """Places the ranks' shard outputs ``parts`` (per rank (out [T_r, H_r, D],
+    lse [T_r, H_r]) NumPy arrays) back into full [Tq, H, D] / [Tq, H] arrays;
+    also returns how many ranks wrote each (token, head) row."""
+    out = np.zeros((case.Tq, case.H, case.D), dtype=np.float64)
+    lse = np.zeros((case.Tq, case.H), dtype=np.float64)
+    count = np.zeros((case.Tq, case.H), dtype=np.int64)
+    for r, (o, l) in enumerate(parts):
+        toks, heads = shard_rows(case, plan, r)
+        out[np.ix_(toks, heads)] = o
+        lse[np.ix_(toks, heads)] = l
+        count[np.ix_(toks, heads)] += 1
+    return out, lse, count
