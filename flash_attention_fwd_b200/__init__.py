@@ -50,6 +50,7 @@ EXPORTED_SYMBOLS = (
     "varlen_attn_bwd_v1",
     "varlen_attn_bwd_noalloc",
     "varlen_attn_plan_shards",
+    "varlen_attn_set_wait_limit",
 )
 
 _lock = threading.Lock()
@@ -102,6 +103,8 @@ def _bind(lib):
     lib.varlen_attn_plan_shards.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, P,
                                             P, P, P]
     lib.varlen_attn_plan_shards.restype = i32
+    lib.varlen_attn_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+    lib.varlen_attn_set_wait_limit.restype = i32
     return lib
 
 
@@ -135,6 +138,14 @@ def device_status(clear: bool = True) -> int:
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return int(val.value)
+
+
+def set_wait_limit(ns: int = 0) -> None:
+    """Testing hook (varlen_attn_set_wait_limit): the kernels' pipeline-wait
+    limit on the current device in ns; 0 restores the default (2 s)."""
+    rc = load_library().varlen_attn_set_wait_limit(int(ns))
+    if rc != VARLEN_OK:
+        raise VarlenAttnError(rc, strerror(rc))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -374,7 +385,7 @@ def varlen_attn_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: tor
                     ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
     """Gradients (dq, dk, dv) of the packed attention forward, given dO and
     the forward's out and lse.  Shapes and dtypes as in ``varlen_attn_fwd``
-    (head dim 64 or 128); outputs and the workspace (``bwd_workspace_size``
+    (head dim 64, 128 or 256); outputs and the workspace (``bwd_workspace_size``
     bytes, uint8 on the device) are allocated here when not given."""
     if q.dtype not in DTYPE_CODES or any(t.dtype != q.dtype for t in (k, v, dout, out)):
         raise TypeError("dout, q, k, v, out must share dtype bfloat16 or float16")

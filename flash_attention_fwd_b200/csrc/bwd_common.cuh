@@ -30,6 +30,7 @@ struct BwdParams {
   uint16_t *dq;            // [Tq, H, D]
   uint16_t *dk, *dv;       // [Tk, Hkv, D]
   float scale;             // softmax scale (dQ and dK carry it)
+  int v8;                  // dq, dk and dv start on 32-byte boundaries: 32-byte row stores
 };
 
 constexpr float LOG2E = 1.4426950408889634f;
@@ -73,11 +74,12 @@ __device__ __forceinline__ float row_delta(const uint16_t *dout_row, const uint1
 }
 
 // Writes D fp32 values read from TMEM (32-column chunks starting at taddr),
-// times `mul`, to a bf16 / fp16 row with 16-byte stores; when `valid` is
-// false the values are read (the TMEM load is collective) but not stored.
+// times `mul`, to a bf16 / fp16 row (32-byte stores when v8, else 16-byte);
+// when `valid` is false the values are read (the TMEM load is collective) but
+// not stored.
 template <int D, bool BF16>
 __device__ __forceinline__ void store_tmem_row(uint32_t taddr, float mul, bool valid,
-                                               uint16_t *row) {
+                                               uint16_t *row, bool v8) {
 #pragma unroll
   for (int c0 = 0; c0 < D; c0 += 32) {
     uint32_t v[32];
@@ -87,10 +89,7 @@ __device__ __forceinline__ void store_tmem_row(uint32_t taddr, float mul, bool v
 #pragma unroll
       for (int c = 0; c < 32; c += 2)
         pk[c / 2] = pack2<BF16>(__uint_as_float(v[c]) * mul, __uint_as_float(v[c + 1]) * mul);
-      uint4 *dst = reinterpret_cast<uint4 *>(row + c0);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+      store16w(row + c0, pk, v8);
     }
   }
 }

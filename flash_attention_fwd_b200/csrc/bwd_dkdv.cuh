@@ -1,6 +1,7 @@
 /*
  * bwd_dkdv.cuh — backward, dK/dV pass: one 128-key tile of one key/value
- * head per work item; the item streams every query tile (BQ = 64 queries)
+ * head per work item (at head dim 256: one column half of its dK / dV, see
+ * below); the item streams every query tile (BQ = 64 queries, 32 at D = 256)
  * of each of the head's H / Hkv query heads that sees the tile:
  *
  *   S^T  = K Q^T,  dP^T = V dO^T          tcgen05 (keys on the TMEM lanes)
@@ -22,10 +23,17 @@
  * double-buffered S^T / dP^T in TMEM and P^T / dS^T in shared memory — so one
  * computes while the tensor cores serve the other; warp 8 scheduler + TMA
  * producer, warp 9 TMEM owner + MMA issuer.  TMEM:
- * dV (D) | dK (D) | S^T[2] (BQ) | dP^T[2] (BQ).  Shared memory: K and V
+ * dV (DO) | dK (DO) | S^T[2] (BQ) | dP^T[2] (BQ).  Shared memory: K and V
  * tiles of the item and NST stages of (Q, dO) query tiles; a stage is held
  * from its load until the step's dV / dK products complete, so the depth is
  * what hides the load latency.
+ *
+ * Head dim 256: dK and dV of a 128-key tile would take all 512 TMEM columns,
+ * so an item computes one column half of them (DO = 128 output columns; the
+ * two halves of a key tile are two items, side by side in the schedule so
+ * that they share the K / V tiles in L2).  S^T and dP^T still contract over
+ * all 256 columns, so each half recomputes them.  K and V take 128 KB of
+ * shared memory, which leaves three stages of 32 queries.
  */
 #pragma once
 #include "bwd_common.cuh"
@@ -38,8 +46,18 @@ constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int RING_CONSUMERS = 1 + 8;
 constexpr int BK = 128;  // keys per item (TMEM lanes)
-constexpr int BQ = 64;   // queries per step
-constexpr int NST = 5;   // (Q, dO) stages
+// Queries per step BQ, (Q, dO) stages NST and output column halves NH per
+// head dim.
+template <int D>
+struct Cfg {
+  static constexpr int BQ = 64, NST = 5, NH = 1;
+};
+template <>
+struct Cfg<256> {
+  static constexpr int BQ = 32, NST = 3, NH = 2;
+};
+constexpr int MAX_STAGES = 5;
+constexpr int MAX_BQ = 64;
 
 struct KeyItem {
   int b;       // sequence; < 0 ends the list
@@ -51,6 +69,7 @@ struct KeyItem {
   int qt0;     // first query tile (BQ queries) that sees the key tile
   int nqt;     // query tiles per query head
   int nsteps;  // (query head, query tile) steps = (H / Hkv) * nqt
+  int half;    // column half of dK / dV (0 when NH = 1)
 };
 
 struct KeyRing {
@@ -59,13 +78,15 @@ struct KeyRing {
   uint64_t empty[ITEM_RING];
 };
 
-// Items are (sequence b, key tile kt, key/value head); an item's cost is its
-// number of query tiles per query head, nqt = ceil(Lq / BQ) - R kt with the
-// causal rule (R = BK / BQ: key tile kt is first seen by query tile R kt) and
-// ceil(Lq / BQ) without it.  Items are listed by cost level, highest first
-// ("longest processing time first", as in the forward scheduler), then by
-// sequence and head, and dealt to CTA i mod G with the direction reversed
-// every round.  The walk is warp-cooperative over 32 sequences at a time.
+// Items are (sequence b, key tile kt, key/value head[, column half]); an
+// item's cost is its number of query tiles per query head,
+// nqt = ceil(Lq / BQ) - R kt with the causal rule (R = BK / BQ: key tile kt is
+// first seen by query tile R kt) and ceil(Lq / BQ) without it.  Items are
+// listed by cost level, highest first ("longest processing time first", as
+// in the forward scheduler), then by sequence, head and half, and dealt to
+// CTA i mod G with the direction reversed every round.  The walk is
+// warp-cooperative over 32 sequences at a time.
+template <int BQ, int NH>
 struct KeyScheduler {
   static constexpr int R = BK / BQ;
   const int *cu_q, *cu_k;
@@ -116,7 +137,7 @@ struct KeyScheduler {
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       u += v;
     }
-    return u * Hkv;
+    return u * Hkv * NH;
   }
   __device__ void init(const KParams &p) {
     cu_q = p.cu_q;
@@ -163,8 +184,9 @@ struct KeyScheduler {
     }
     if (level < 0) return false;
     const long long local = idx - level_base;
-    const long long unit = local / Hkv;
-    w.kvh = (int)(local % Hkv);
+    const long long unit = local / (Hkv * NH);
+    w.kvh = (int)((local / NH) % Hkv);
+    w.half = (int)(local % NH);
     for (;;) {
       const int b = cur_b + lane;
       int qs = 0, lq = 0, ks = 0, lk = 0, u = 0;
@@ -211,21 +233,22 @@ struct KeyScheduler {
 
 struct Barriers {
   uint64_t kv_full, kv_empty;
-  uint64_t st_full[NST], st_empty[NST];
+  uint64_t st_full[MAX_STAGES], st_empty[MAX_STAGES];
   uint64_t s_full[2];    // S^T and dP^T of a step in TMEM buffer
   uint64_t pd_full[2];   // P^T and dS^T written to TMEM (one arrival per row warp)
   uint64_t acc_ready, acc_free;
   uint64_t lsd_full[2];  // [warpgroup]: a step's LSE / delta values written (one arrival per warp)
   uint64_t drain;
   KeyRing ring;
-  alignas(16) float lsd[2][2][BQ];  // [warpgroup]: LSE * log2e and delta of the step's queries
+  alignas(16) float lsd[2][2][MAX_BQ];  // [warpgroup]: LSE * log2e and delta of the step's queries
   uint32_t tmem_base;
-  int abort_flag;
+  AbortState abort;
 };
 
 template <int D>
 constexpr size_t smem_bytes() {
-  return (size_t)2 * BK * D * 2 + (size_t)NST * 2 * BQ * D * 2 + sizeof(Barriers) + 1024;
+  return (size_t)2 * BK * D * 2 + (size_t)Cfg<D>::NST * 2 * Cfg<D>::BQ * D * 2 +
+         sizeof(Barriers) + 1024;
 }
 
 template <int D, bool BF16>
@@ -233,14 +256,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const BwdParams bp) {
+  constexpr int BQ = Cfg<D>::BQ;
+  constexpr int NST = Cfg<D>::NST;
+  constexpr int NH = Cfg<D>::NH;
+  constexpr int DO = D / NH;  // dK / dV columns of an item
+  static_assert(NST <= MAX_STAGES && BQ <= MAX_BQ && BQ % 32 == 0, "stage layout");
   constexpr int DB = D / 64;
   constexpr uint32_t KV_BYTES = BK * D * 2;
   constexpr uint32_t QS_BYTES = BQ * D * 2;
-  constexpr uint32_t DV_COL = 0, DK_COL = D;
-  constexpr uint32_t ST_COL = 2 * D, DPT_COL = 2 * D + 2 * BQ;
+  constexpr uint32_t DV_COL = 0, DK_COL = DO;
+  constexpr uint32_t ST_COL = 2 * DO, DPT_COL = 2 * DO + 2 * BQ;
   static_assert(DPT_COL + 2 * BQ <= TMEM_COLS, "TMEM budget");
   constexpr uint32_t IDESC_ST = ptx::idesc_f16(BK, BQ, BF16, false);
-  constexpr uint32_t IDESC_ACC = ptx::idesc_f16(BK, D, BF16, true);
+  constexpr uint32_t IDESC_ACC = ptx::idesc_f16(BK, DO, BF16, true);
   const KParams &p = bp.kp;
 
   extern __shared__ uint8_t smem_raw[];
@@ -250,7 +278,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *sV = sK + KV_BYTES;
   uint8_t *sQs = sV + KV_BYTES;  // stage s: Q at sQs + s * 2 * QS_BYTES, dO after it
   Barriers *bars = reinterpret_cast<Barriers *>(sQs + NST * 2 * QS_BYTES);
-  volatile int *abort_flag = &bars->abort_flag;
+  AbortState *abort_flag = &bars->abort;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -275,7 +303,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&bars->ring.full[i], 1);
       ptx::mbar_init(&bars->ring.empty[i], RING_CONSUMERS);
     }
-    bars->abort_flag = 0;
+    bars->abort.init();
     ptx::mbar_init_fence();
   }
   if (warp == PRODUCER_WARP && lane == 0) {
@@ -295,7 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
-    KeyScheduler sched;
+    KeyScheduler<BQ, NH> sched;
     sched.init(p);
     uint32_t rs = 0, rph = 0, kv_count = 0, gs = 0;
     bool ok = true;
@@ -383,10 +411,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       // dV += P^T dO, dK += dS^T Q for global step gs: P^T / dS^T from TMEM
       // (bf16/fp16 pairs over the first BQ / 2 columns of S^T / dP^T), dO and
-      // Q MN-major from the stage, in steps of 16 queries
-      auto issue_acc = [&](uint32_t gs, bool acc) {
+      // Q MN-major from the stage (columns [half * DO, (half + 1) * DO): the
+      // column blocks from half * DO / 64 on), in steps of 16 queries
+      auto issue_acc = [&](uint32_t gs, bool acc, int half) {
         const uint32_t st = gs % NST;
-        const uint32_t qa = sQs_addr + st * 2 * QS_BYTES;
+        const uint32_t qa = sQs_addr + st * 2 * QS_BYTES + half * (DO / 64) * (BQ * 128);
         const uint32_t buf = gs & 1u;
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk) {
@@ -421,7 +450,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!(ok = wait_bar(&bars->acc_free, (items - 1) & 1u, abort_flag))) break;
             ptx::tc_fence_after();
           }
-          issue_acc(gs, s > 0);
+          issue_acc(gs, s > 0, w.half);
           ptx::mma_commit(&bars->st_empty[gs % NST]);
           if (s == n - 1) {
             ptx::mma_commit(&bars->acc_ready);
@@ -448,6 +477,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // LSE (log2 units) or delta of query c of step s: thread r < BQ loads LSE
     // of query r, thread BQ + c delta of query c
     auto load_lsd = [&](const KeyItem &w, int s) -> float {
+      if (r >= 2 * BQ) return 0.f;  // no value to publish
       const int c = r & (BQ - 1);
       const int h = w.kvh * p.group + s / w.nqt;
       const int qi = (w.qt0 + s % w.nqt) * BQ + c;
@@ -470,11 +500,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int n = w.nsteps;
       const int kk = w.kt * BK + r;  // sequence-local key
       const bool key_valid = kk < w.Lk;
-      const size_t drow = ((size_t)(w.k0 + r) * p.Hkv + w.kvh) * D;
-      // warpgroup 0 writes dV, warpgroup 1 dK
+      const size_t drow = ((size_t)(w.k0 + r) * p.Hkv + w.kvh) * D + w.half * DO;
+      // warpgroup 0 writes dV, warpgroup 1 dK (the item's column half)
       uint16_t *out_row = (t == 0 ? bp.dv : bp.dk) + drow;
       if (n == 0) {
-        if (key_valid) zero_row<D>(out_row);
+        if (key_valid) zero_row<DO>(out_row);
         continue;
       }
       const int s0 = (int)((t - g) & 1u);  // this warpgroup's first step of the item
@@ -493,7 +523,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // finished reading the previous values and the buffer can be reused.
         // (S^T(gs) also overwrote the previous step's P^T in TMEM only after
         // the dV / dK products that read it: the tensor core runs in order.)
-        bars->lsd[t][r / BQ][r & (BQ - 1)] = pre;
+        if (r < 2 * BQ) bars->lsd[t][r / BQ][r & (BQ - 1)] = pre;
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(&bars->lsd_full[t]);
         if (s + 2 < n) pre = load_lsd(w, s + 2);
@@ -509,17 +539,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float *lse2 = bars->lsd[t][0];
         const float *dl = bars->lsd[t][1];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int piece = 0; piece < BQ / 32; ++piece) {
           uint32_t sv[32], dpv[32];
-          tmem_ld_wait<32>(tST + half * 32, sv);
-          tmem_ld_wait<32>(tDPT + half * 32, dpv);
+          tmem_ld_wait<32>(tST + piece * 32, sv);
+          tmem_ld_wait<32>(tDPT + piece * 32, dpv);
           uint32_t ppk[16], dpk[16];
 #pragma unroll
           for (int c2 = 0; c2 < 32; c2 += 2) {
             float pr[2], ds[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int c = half * 32 + c2 + e;
+              const int c = piece * 32 + c2 + e;
               const float x = __uint_as_float(sv[c2 + e]) * sl2 - lse2[c];
               pr[e] = (key_valid && c >= cmin) ? ptx::ex2_approx(x) : 0.f;
               ds[e] = pr[e] * (__uint_as_float(dpv[c2 + e]) - dl[c]);
@@ -527,9 +557,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ppk[c2 / 2] = pack2<BF16>(pr[0], pr[1]);
             dpk[c2 / 2] = pack2<BF16>(ds[0], ds[1]);
           }
-          // columns [16 half, 16 half + 16): S^T / dP^T columns already read
-          tmem_st<16>(tST + half * 16, ppk);
-          tmem_st<16>(tDPT + half * 16, dpk);
+          // columns [16 piece, 16 piece + 16): S^T / dP^T columns already read
+          tmem_st<16>(tST + piece * 16, ppk);
+          tmem_st<16>(tDPT + piece * 16, dpk);
         }
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
@@ -542,8 +572,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ++items;
       if (!__all_sync(0xffffffffu, got)) break;
       ptx::tc_fence_after();
-      store_tmem_row<D, BF16>(tmem + lane_base + (t == 0 ? DV_COL : DK_COL),
-                              t == 0 ? 1.f : bp.scale, key_valid, out_row);
+      store_tmem_row<DO, BF16>(tmem + lane_base + (t == 0 ? DV_COL : DK_COL),
+                               t == 0 ? 1.f : bp.scale, key_valid, out_row, bp.v8 != 0);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->acc_free);

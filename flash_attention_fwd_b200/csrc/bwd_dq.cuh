@@ -1,6 +1,7 @@
 /*
  * bwd_dq.cuh — backward, dQ pass: one 128-row query tile (one query head) per
- * work item, streaming the sequence's visible key tiles of BN = 96 keys:
+ * work item, streaming the sequence's visible key tiles of BN keys (96 at
+ * head dims 64 and 128, 32 at 256):
  *
  *   S(j)  = Q K(j)^T                      tcgen05, into TMEM
  *   dP(j) = dO V(j)^T                     tcgen05, into TMEM
@@ -20,9 +21,11 @@
  * serve the other; warp 8 scheduler + TMA producer, warp 9 TMEM owner + MMA
  * issuer.  TMEM:
  * S[2] | dP[2] (BN columns each, double-buffered across key tiles) | dQ (D),
- * 4 * 96 + 128 = 512 columns at D = 128.  (The S and dP products take about
- * as long per instruction at N = 96 as at N = 64, so the wider tile does half
- * again as much work per instruction; N = 128 would not fit.)  The row
+ * 4 * 96 + 128 = 512 columns at D = 128, 4 * 32 + 256 = 384 at D = 256.
+ * (The S and dP products take about as long per instruction at N = 96 as at
+ * N = 64, so the wider tile does half again as much work per instruction;
+ * N = 128 would not fit.  At D = 256 shared memory, not TMEM, sets the
+ * 32-key tile.)  The row
  * threads read S and dP in 32-column pieces.  The K/V ring holds K(j) and
  * V(j) in turn; V(j) is released after dP(j), K(j) after dQ(j).
  */
@@ -36,12 +39,24 @@ constexpr int NUM_THREADS = 320;
 constexpr int PRODUCER_WARP = 8;
 constexpr int MMA_WARP = 9;
 constexpr int RING_CONSUMERS = 1 + 8;
-constexpr int BN = 96;
-constexpr int NSLOT = 6;
+// Key tile BN and K/V ring depth NSLOT per head dim.  At D = 256 the query
+// and dO tiles take 128 KB of shared memory and dQ 256 TMEM columns, which
+// leaves room for double-buffered S / dP of 32 keys and six 16 KB slots (the
+// ring must hold K and V of two tiles ahead: the prologue computes S / dP of
+// two tiles before the first dQ product releases a K tile).
+template <int D>
+struct Cfg {
+  static constexpr int BN = 96, NSLOT = 6;
+};
+template <>
+struct Cfg<256> {
+  static constexpr int BN = 32, NSLOT = 6;
+};
+constexpr int MAX_SLOTS = 6;
 
 struct Barriers {
-  uint64_t full[NSLOT];
-  uint64_t empty[NSLOT];
+  uint64_t full[MAX_SLOTS];
+  uint64_t empty[MAX_SLOTS];
   uint64_t q_full, q_empty;  // Q and dO tiles of the item
   uint64_t s_full[2];        // S(j) and dP(j) in TMEM buffer j & 1
   uint64_t ds_full[2];       // dS(j) written (one arrival per row warp)
@@ -49,12 +64,13 @@ struct Barriers {
   uint64_t drain;
   ItemRing ring;
   uint32_t tmem_base;
-  int abort_flag;
+  AbortState abort;
 };
 
 template <int D>
 constexpr size_t smem_bytes() {
-  return (size_t)2 * BM * D * 2 + (size_t)NSLOT * BN * D * 2 + sizeof(Barriers) + 1024;
+  return (size_t)2 * BM * D * 2 + (size_t)Cfg<D>::NSLOT * Cfg<D>::BN * D * 2 + sizeof(Barriers) +
+         1024;
 }
 
 template <int D, bool BF16>
@@ -62,6 +78,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const BwdParams bp) {
+  constexpr int BN = Cfg<D>::BN;
+  constexpr int NSLOT = Cfg<D>::NSLOT;
+  static_assert(NSLOT <= MAX_SLOTS && NSLOT >= 4, "K/V ring depth");
   constexpr int DB = D / 64;
   constexpr uint32_t Q_BYTES = BM * D * 2;
   constexpr uint32_t KV_BYTES = BN * D * 2;
@@ -79,7 +98,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *sDO = smem + Q_BYTES;
   uint8_t *sKV = smem + 2 * Q_BYTES;
   Barriers *bars = reinterpret_cast<Barriers *>(sKV + NSLOT * KV_BYTES);
-  volatile int *abort_flag = &bars->abort_flag;
+  AbortState *abort_flag = &bars->abort;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -102,7 +121,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&bars->ring.full[i], 1);
       ptx::mbar_init(&bars->ring.empty[i], RING_CONSUMERS);
     }
-    bars->abort_flag = 0;
+    bars->abort.init();
     ptx::mbar_init_fence();
   }
   if (warp == PRODUCER_WARP && lane == 0) {
@@ -342,7 +361,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ++items;
       if (!__all_sync(0xffffffffu, got)) break;
       ptx::tc_fence_after();
-      store_tmem_row<D / 2, BF16>(tDQ + t * (D / 2), bp.scale, row_valid, dq_half);
+      store_tmem_row<D / 2, BF16>(tDQ + t * (D / 2), bp.scale, row_valid, dq_half, bp.v8 != 0);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->dq_free);

@@ -65,7 +65,7 @@ static int bwd_check_args(const void *dout, const void *q, const void *k, const 
     return VARLEN_ERR_SHAPE;
   if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0)
     return VARLEN_ERR_SHAPE;
-  if (head_dim != 64 && head_dim != 128) return VARLEN_ERR_SHAPE;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return VARLEN_ERR_SHAPE;
   if (total_q >= (int64_t(1) << 31) || total_k >= (int64_t(1) << 31)) return VARLEN_ERR_SHAPE;
   if (num_heads > 65535) return VARLEN_ERR_SHAPE;
   if (batch > 0 && (!cu_seqlens_q || !cu_seqlens_k)) return VARLEN_ERR_NULL;
@@ -109,21 +109,24 @@ extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k
   const bool bf16 = dtype == VARLEN_BF16;
   const int D = head_dim;
 
-  // tensor maps: dQ pass (Q, dO tiles of 128 rows; K, V tiles of 64), dK/dV
-  // pass (Q, dO tiles of 64 rows; K, V tiles of 128)
+  // tensor maps: dQ pass (Q, dO tiles of 128 rows; K, V tiles of its key
+  // tile), dK/dV pass (Q, dO tiles of its query step; K, V tiles of 128)
+  const int dq_bn = D == 256 ? bwd_dq::Cfg<256>::BN : bwd_dq::Cfg<128>::BN;
+  const int kv_bq = D == 256 ? bwd_dkdv::Cfg<256>::BQ : bwd_dkdv::Cfg<128>::BQ;
+  const int kv_nh = D == 256 ? bwd_dkdv::Cfg<256>::NH : bwd_dkdv::Cfg<128>::NH;
   alignas(64) CUtensorMap m_dq[4], m_kv[4];
   memset(m_dq, 0, sizeof m_dq);
   memset(m_kv, 0, sizeof m_kv);
   if (total_q > 0) {
     if (!encode_qkv_map(enc, &m_dq[0], q, bf16, total_q, num_heads, D, BM) ||
         !encode_qkv_map(enc, &m_dq[1], dout, bf16, total_q, num_heads, D, BM) ||
-        !encode_qkv_map(enc, &m_kv[0], q, bf16, total_q, num_heads, D, bwd_dkdv::BQ) ||
-        !encode_qkv_map(enc, &m_kv[1], dout, bf16, total_q, num_heads, D, bwd_dkdv::BQ))
+        !encode_qkv_map(enc, &m_kv[0], q, bf16, total_q, num_heads, D, kv_bq) ||
+        !encode_qkv_map(enc, &m_kv[1], dout, bf16, total_q, num_heads, D, kv_bq))
       return VARLEN_ERR_LAUNCH;
   }
   if (total_k > 0) {
-    if (!encode_qkv_map(enc, &m_dq[2], k, bf16, total_k, num_kv_heads, D, bwd_dq::BN) ||
-        !encode_qkv_map(enc, &m_dq[3], v, bf16, total_k, num_kv_heads, D, bwd_dq::BN) ||
+    if (!encode_qkv_map(enc, &m_dq[2], k, bf16, total_k, num_kv_heads, D, dq_bn) ||
+        !encode_qkv_map(enc, &m_dq[3], v, bf16, total_k, num_kv_heads, D, dq_bn) ||
         !encode_qkv_map(enc, &m_kv[2], k, bf16, total_k, num_kv_heads, D, bwd_dkdv::BK) ||
         !encode_qkv_map(enc, &m_kv[3], v, bf16, total_k, num_kv_heads, D, bwd_dkdv::BK))
       return VARLEN_ERR_LAUNCH;
@@ -156,10 +159,11 @@ extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k
   bp.dk = static_cast<uint16_t *>(dk);
   bp.dv = static_cast<uint16_t *>(dv);
   bp.scale = sc;
+  bp.v8 = (aligned(dq, 32) && aligned(dk, 32) && aligned(dv, 32)) ? 1 : 0;
 
   long long items_q = (long long)batch * ((max_seqlen_q + BM - 1) / BM) * num_heads;
   long long items_k = (long long)batch * ((max_seqlen_k + bwd_dkdv::BK - 1) / bwd_dkdv::BK) *
-                      num_kv_heads;
+                      num_kv_heads * kv_nh;
   int grid_q = dev.sms, grid_k = dev.sms;
   if (items_q >= 1 && items_q < grid_q) grid_q = (int)items_q;
   if (items_k >= 1 && items_k < grid_k) grid_k = (int)items_k;
@@ -171,6 +175,11 @@ extern "C" int varlen_attn_bwd_v1(const void *dout, const void *q, const void *k
                                        10)
                 : launch_bwd<64, false>(m_dq, m_kv, bp, grid_q, grid_k, run_dq, run_dkdv, s,
                                         dev, 12);
+  if (D == 256)
+    return bf16 ? launch_bwd<256, true>(m_dq, m_kv, bp, grid_q, grid_k, run_dq, run_dkdv, s,
+                                        dev, 22)
+                : launch_bwd<256, false>(m_dq, m_kv, bp, grid_q, grid_k, run_dq, run_dkdv, s,
+                                         dev, 24);
   return bf16 ? launch_bwd<128, true>(m_dq, m_kv, bp, grid_q, grid_k, run_dq, run_dkdv, s, dev,
                                       14)
               : launch_bwd<128, false>(m_dq, m_kv, bp, grid_q, grid_k, run_dq, run_dkdv, s, dev,

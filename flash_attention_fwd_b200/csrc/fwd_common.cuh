@@ -31,6 +31,26 @@ constexpr unsigned STATUS_BAD_PAGE = 2u;  // a page-table entry outside [0, num_
 
 // Device-side status word (bit STATUS_TIMEOUT: a bounded wait gave up).
 __device__ unsigned int g_device_status = 0;
+// Limit of the pipeline waits (wait_bar) on this device: WAIT_TIMEOUT_NS,
+// unless a test lowers it (varlen_attn_set_wait_limit) so that the waits run
+// out and the kernels take their abort path.  Each CTA copies it into shared
+// memory at start (AbortState).  The end-of-kernel drains keep
+// WAIT_TIMEOUT_NS: they wait for work already issued.
+__device__ unsigned long long g_wait_limit_ns = WAIT_TIMEOUT_NS;
+
+// Per-CTA abort state in shared memory: the flag a role raises when one of
+// its waits runs out (every other pipeline wait then gives up too), and the
+// CTA's copy of the wait limit.
+struct AbortState {
+  unsigned long long limit_ns;
+  int flag;
+  __device__ void init() {
+    limit_ns = g_wait_limit_ns;
+    flag = 0;
+  }
+  __device__ bool raised() const { return *reinterpret_cast<const volatile int *>(&flag) != 0; }
+  __device__ void raise() { *reinterpret_cast<volatile int *>(&flag) = 1; }
+};
 
 struct KParams {
   const int *cu_q;
@@ -82,7 +102,25 @@ struct KParams {
   long long part_rows;  // total_q * H
   float *part_o;
   float *part_lse;
+  // out / part_o start on a 32-byte boundary (their rows then do too: a row
+  // is a multiple of 128 bytes), so rows are written in 32-byte stores, one
+  // whole sector each; otherwise in 16-byte stores
+  int out_v8, part_v8;
 };
+
+// 16 words (32 bf16 / fp16 values) to dst: two 32-byte stores when v8 (dst
+// 32-byte aligned), four 16-byte stores otherwise.
+__device__ __forceinline__ void store16w(void *dst, const uint32_t (&w)[16], bool v8) {
+  if (v8) {
+    ptx::st_global_v8(dst, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+    ptx::st_global_v8(static_cast<uint32_t *>(dst) + 8, w[8], w[9], w[10], w[11], w[12], w[13],
+                      w[14], w[15]);
+  } else {
+    uint4 *d = static_cast<uint4 *>(dst);
+#pragma unroll
+    for (int v4 = 0; v4 < 4; ++v4) d[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+  }
+}
 
 // Pieces of a key range of nk tiles: P pieces, the first r of base + 1 tiles
 // and the other P - r of base tiles (P = 1, base = nk when it is not split).
@@ -402,16 +440,11 @@ struct Scheduler {
 // Keys of the item's last visited key tile (of BN keys) that lie inside the
 // sequence's used keys (at least 1); the tile's other rows hold whatever
 // follows them in the buffer (the next sequence, unused cache slots, the rest
-// of a page).  The PV product of that tile runs over the 16-key steps that
-// hold used keys only, so just the rows from the last used key to the end of
-// its 16-key step need clearing (none when the count is a multiple of 16).
+// of a page).
 template <int BN>
 __device__ __forceinline__ int last_tile_keys(const WorkItem &w) {
   return min(BN, w.Lk - (w.kofs + (w.n_kv - 1) * BN));
 }
-__device__ __forceinline__ bool tail_needs_fix(int keys) { return (keys & 15) != 0; }
-// 16-key steps of a PV product over a tile with `keys` used keys
-__device__ __forceinline__ int pv_steps(int keys) { return (keys + 15) >> 4; }
 
 // Work items travel from the scheduling (producer) warp to the other roles
 // through a small ring in shared memory.  An item with hu < 0 ends the list.
@@ -423,15 +456,16 @@ struct ItemRing {
 };
 
 // Bounded wait; on timeout raises the CTA abort flag and the device status.
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+// The clock and the abort flag are looked at every 64 polls (about 2 us).
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, AbortState *abort_flag) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (ptx::globaltimer_ns() - t0 > WAIT_TIMEOUT_NS) {
-        *abort_flag = 1;
+      if (abort_flag->raised()) return false;
+      if (ptx::globaltimer_ns() - t0 > abort_flag->limit_ns) {
+        abort_flag->raise();
         atomicOr(&g_device_status, STATUS_TIMEOUT);
         return false;
       }
@@ -475,37 +509,39 @@ __device__ __forceinline__ bool drain_wait(uint64_t *bar, uint32_t parity) {
 // Rows past the used keys.  The last key tile of an item may run past the
 // sequence's used keys (into the next sequence's rows, the unused slots of a
 // KV cache, or the rest of a page).  Their scores are masked, so P is 0
-// there, but 0 times a non-finite value is NaN.  The PV product of that tile
-// skips the 16-key steps past the used keys; once the last V tile has landed,
-// the warp overwrites the remaining rows of the last used step (from the last
-// used key to the step's end, at most 15) with zeros and then arrives on
-// `vfix`, which the MMA warp waits for before that tile's PV product.  The
-// fix is deferred until the next item's first K tile and Q tile are queued,
-// so that the wait for the V tile to land does not hold up the next item's
-// loads (and the slots it needs never wait on the fix).
+// there, but 0 times a non-finite value is NaN.  So the copies of that V tile
+// complete on `tail` (an mbarrier of SPLIT arrivals) instead of the slot's
+// `full` barrier; once they have landed, the warp overwrites the rows past the
+// used keys with zeros, fences the writes for the async proxy and then
+// arrives on `full` itself, which is what the MMA warp waits for: the
+// consumers see an ordinary slot.  The fix is deferred until the next item's
+// first K tile is queued (so that the wait for the V tile to land overlaps
+// that load, and the slot it needs is never held by the fix), and it runs
+// before that item's Q tile, whose buffer frees only once the current item's
+// last S products complete.
 template <int BN, int D, int NSLOT, int SPLIT = 1>
 struct KVProducer {
   static constexpr int DB = D / 64;
   static constexpr uint32_t KV_BYTES = BN * D * 2;
   uint8_t *sKV;
-  uint64_t *full, *empty, *vfix;
-  volatile int *abort_flag;
+  uint64_t *full, *empty, *tail;
+  AbortState *abort_flag;
   uint64_t pol;
   uint32_t slot, phase;
   uint32_t fills[NSLOT];
   int lane;
-  // pending tail fix: first ring slot and phase of the last V tile, and the
-  // number of its rows that hold used keys (BN or a multiple of 16: nothing
-  // to fix)
-  uint32_t fix_slot, fix_phase;
+  // pending tail fix: first ring slot of the last V tile, the number of its
+  // rows that hold used keys (BN: nothing to fix), tail fills so far
+  uint32_t fix_slot;
   int fix_keys;
+  uint32_t tails;
 
-  __device__ void init(uint8_t *s, uint64_t *f, uint64_t *e, uint64_t *vf,
-                       volatile int *abort) {
+  __device__ void init(uint8_t *s, uint64_t *f, uint64_t *e, uint64_t *tl, AbortState *abort) {
     sKV = s;
     full = f;
     empty = e;
-    vfix = vf;
+    tail = tl;
+    tails = 0;
     abort_flag = abort;
     pol = ptx::policy_evict_last();
     slot = 0;
@@ -514,32 +550,51 @@ struct KVProducer {
     lane = threadIdx.x & 31;
     fix_keys = BN;
   }
-  // Whole warp: zero the rows [fix_keys, round_up(fix_keys, 16)) of the
-  // pending last V tile once it has landed, then signal vfix.  False when the
-  // wait gave up.
+  // Whole warp: once the pending last V tile has landed on `tail`, zero its
+  // rows [fix_keys, BN) in every slice and complete the slices' `full`
+  // barriers.  False when the wait gave up.
   __device__ bool fix_tail() {
-    if (!tail_needs_fix(fix_keys)) return true;
+    if (fix_keys >= BN) return true;
+    // on a wait that gave up the fix stays pending, for drain_tail
+    if (!__all_sync(0xffffffffu, wait_bar(tail, (tails - 1) & 1u, abort_flag))) return false;
     const int keys = fix_keys;
     fix_keys = BN;
-    uint32_t s = fix_slot, ph = fix_phase;
+    const int per_block = (BN - keys) * 8;  // 16-byte chunks of one column block
+    uint32_t s = fix_slot;
 #pragma unroll
     for (int i = 0; i < SPLIT; ++i) {
-      if (!__all_sync(0xffffffffu, wait_bar(&full[s], ph, abort_flag))) return false;
-      const int per_block = (16 - (keys & 15)) * 8;  // 16-byte chunks of one column block
-      for (int c = lane; c < DB * per_block; c += 32) {
-        const int db = c / per_block;
+#pragma unroll
+      for (int db = 0; db < DB; ++db) {
+        // rows [keys, BN) of a column block are one contiguous range
         uint4 *dst = reinterpret_cast<uint4 *>(sKV + s * KV_BYTES + db * (BN * 128) + keys * 128);
-        dst[c - db * per_block] = make_uint4(0u, 0u, 0u, 0u);
+        for (int c = lane; c < per_block; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
       }
-      if (++s == NSLOT) {
-        s = 0;
-        ph ^= 1u;
-      }
+      if (++s == NSLOT) s = 0;
     }
     ptx::fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(vfix);
+    if (lane == 0) {
+      s = fix_slot;
+#pragma unroll
+      for (int i = 0; i < SPLIT; ++i) {
+        ptx::mbar_arrive(&full[s]);
+        if (++s == NSLOT) s = 0;
+      }
+    }
     return true;
+  }
+  // lane 0, end of kernel: a tail tile whose fix never ran (the CTA gave up)
+  // still has copies in flight; wait for them, then complete its slots'
+  // `full` barriers so that the ring drain below sees every fill done.
+  __device__ void drain_tail() {
+    if (fix_keys >= BN) return;
+    drain_wait(tail, (tails - 1) & 1u);
+    uint32_t s = fix_slot;
+    for (int i = 0; i < SPLIT; ++i) {
+      ptx::mbar_arrive(&full[s]);
+      if (++s == NSLOT) s = 0;
+    }
+    fix_keys = BN;
   }
   __device__ void advance() {
     ++fills[slot];
@@ -549,22 +604,23 @@ struct KVProducer {
     }
   }
   // lane 0: key rows [row, row + BN) of a packed k/v (columns [col0, col0 + D)
-  // of the tensor; col0 a multiple of 64)
-  __device__ bool load_packed(const CUtensorMap *tm, int kv_h, int row, int col0 = 0) {
+  // of the tensor; col0 a multiple of 64), completing on `bar`
+  __device__ bool load_packed(const CUtensorMap *tm, int kv_h, int row, int col0 = 0,
+                              uint64_t *bar = nullptr) {
     if (!wait_bar(&empty[slot], phase ^ 1u, abort_flag)) return false;
     uint8_t *dst = sKV + slot * KV_BYTES;
-    ptx::mbar_arrive_expect_tx(&full[slot], KV_BYTES);
+    if (bar == nullptr) bar = &full[slot];
+    ptx::mbar_arrive_expect_tx(bar, KV_BYTES);
 #pragma unroll
     for (int db = 0; db < DB; ++db)
-      ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &full[slot], col0 + db * 64, kv_h, row,
-                            pol);
+      ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, bar, col0 + db * 64, kv_h, row, pol);
     advance();
     return true;
   }
-  __device__ bool tile_packed(const CUtensorMap *tm, int kv_h, int row) {
+  __device__ bool tile_packed(const CUtensorMap *tm, int kv_h, int row, uint64_t *bar = nullptr) {
 #pragma unroll
     for (int s = 0; s < SPLIT; ++s)
-      if (!load_packed(tm, kv_h, row, s * D)) return false;
+      if (!load_packed(tm, kv_h, row, s * D, bar)) return false;
     return true;
   }
   // paged: source row of box `lane` of the key tile that starts at key0
@@ -587,11 +643,13 @@ struct KVProducer {
   // Lane 0 waits for the slot and posts the byte count first, so the lanes'
   // copies (one warp instruction per column block) complete into a phase
   // that already expects them.
-  __device__ bool load_paged(const CUtensorMap *tm, int kv_h, int my_row, int ch, int col0 = 0) {
+  __device__ bool load_paged(const CUtensorMap *tm, int kv_h, int my_row, int ch, int col0 = 0,
+                             uint64_t *bar = nullptr) {
     bool ok = true;
+    if (bar == nullptr) bar = &full[slot];
     if (lane == 0) {
       ok = wait_bar(&empty[slot], phase ^ 1u, abort_flag);
-      if (ok) ptx::mbar_arrive_expect_tx(&full[slot], KV_BYTES);
+      if (ok) ptx::mbar_arrive_expect_tx(bar, KV_BYTES);
     }
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) return false;
@@ -599,61 +657,63 @@ struct KVProducer {
       uint8_t *dst = sKV + slot * KV_BYTES + lane * ch * 128;
 #pragma unroll
       for (int db = 0; db < DB; ++db)
-        ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, &full[slot], col0 + db * 64, kv_h,
-                              my_row, pol);
+        ptx::tma_load_3d_hint(dst + db * (BN * 128), tm, bar, col0 + db * 64, kv_h, my_row, pol);
     }
     advance();
     return true;
   }
-  __device__ bool tile_paged(const CUtensorMap *tm, int kv_h, int my_row, int ch) {
+  __device__ bool tile_paged(const CUtensorMap *tm, int kv_h, int my_row, int ch,
+                             uint64_t *bar = nullptr) {
 #pragma unroll
     for (int s = 0; s < SPLIT; ++s)
-      if (!load_paged(tm, kv_h, my_row, ch, s * D)) return false;
+      if (!load_paged(tm, kv_h, my_row, ch, s * D, bar)) return false;
     return true;
   }
-  // Records the ring position of the item's last V tile (about to be
-  // loaded) when some of its rows lie past the used keys.
-  __device__ void note_tail(const WorkItem &w) {
-    fix_keys = last_tile_keys<BN>(w);
+  // The item's last V tile, about to be loaded: when some of its rows lie
+  // past the used keys, records its ring position and returns the barrier
+  // its copies complete on (`tail`); otherwise its slot's own `full`.
+  __device__ uint64_t *note_tail(const WorkItem &w) {
+    const int keys = last_tile_keys<BN>(w);
+    if (keys >= BN) return nullptr;
+    fix_keys = keys;
     fix_slot = slot;
-    fix_phase = phase;
+    ++tails;
+    return tail;
   }
   // Whole warp: the K/V tiles of one item in the order the MMA warp consumes
   // them (K0, K1, V0, K2, V1, K3, ..., V(n-1)), with the item's Q tile(s) after
   // K0 through load_q (called by lane 0, returns false when a wait gave up).
-  // The previous item's pending tail fix runs right after the Q load.
+  // The previous item's pending tail fix runs between K0 and the Q load.
   template <class LoadQ>
   __device__ bool load_item(const KParams &p, const WorkItem &w, int kv_h, const CUtensorMap *tm_k,
                             const CUtensorMap *tm_v, LoadQ &&load_q) {
     const int n = w.n_kv;
     if (p.page_table == nullptr) {
       bool ok = true;
-      if (lane == 0) ok = tile_packed(tm_k, kv_h, w.k0) && load_q();
+      if (lane == 0) ok = tile_packed(tm_k, kv_h, w.k0);
       ok = __shfl_sync(0xffffffffu, ok, 0) && fix_tail();
       if (lane == 0) {
+        if (ok) ok = load_q();
         if (ok && n >= 2) ok = tile_packed(tm_k, kv_h, w.k0 + BN);
         for (int j = 0; ok && j < n; ++j) {
-          if (j == n - 1) note_tail(w);
-          ok = tile_packed(tm_v, kv_h, w.k0 + j * BN);
+          ok = tile_packed(tm_v, kv_h, w.k0 + j * BN, j == n - 1 ? note_tail(w) : nullptr);
           if (ok && j + 2 < n) ok = tile_packed(tm_k, kv_h, w.k0 + (j + 2) * BN);
         }
       }
+      // lane 0 issued the copies; the whole warp runs the fix
       ok = __shfl_sync(0xffffffffu, ok, 0);
       fix_keys = __shfl_sync(0xffffffffu, fix_keys, 0);
       fix_slot = __shfl_sync(0xffffffffu, fix_slot, 0);
-      fix_phase = __shfl_sync(0xffffffffu, fix_phase, 0);
-      // lane 0 advanced the ring for the whole warp
-      slot = __shfl_sync(0xffffffffu, slot, 0);
-      phase = __shfl_sync(0xffffffffu, phase, 0);
+      tails = __shfl_sync(0xffffffffu, tails, 0);
       return ok;
     }
     const int ch = p.page_chunk;
     int r0 = chunk_row(p, w, w.kofs), r1 = 0;
-    bool ok = tile_paged(tm_k, kv_h, r0, ch);
+    bool ok = tile_paged(tm_k, kv_h, r0, ch) && fix_tail();
     if (ok) {
       bool q = true;
       if (lane == 0) q = load_q();
-      ok = __shfl_sync(0xffffffffu, q, 0) && fix_tail();
+      ok = __shfl_sync(0xffffffffu, q, 0);
     }
     if (ok && n >= 2) {
       r1 = chunk_row(p, w, w.kofs + BN);
@@ -662,8 +722,7 @@ struct KVProducer {
     for (int j = 0; ok && j < n; ++j) {
       // look up K(j+2) before waiting for V(j)'s slot, so that the two overlap
       const int rn = (j + 2 < n) ? chunk_row(p, w, w.kofs + (j + 2) * BN) : 0;
-      if (j == n - 1) note_tail(w);
-      ok = tile_paged(tm_v, kv_h, (j & 1) ? r1 : r0, ch);
+      ok = tile_paged(tm_v, kv_h, (j & 1) ? r1 : r0, ch, j == n - 1 ? note_tail(w) : nullptr);
       if (ok && j + 2 < n) {
         if (j & 1)
           r1 = rn;
@@ -676,6 +735,7 @@ struct KVProducer {
   }
   // lane 0: every copy issued has landed (before the CTA exits)
   __device__ void drain() {
+    drain_tail();
     for (int i = 0; i < NSLOT; ++i)
       if (fills[i] > 0) drain_wait(&full[i], (fills[i] - 1) & 1u);
   }
@@ -755,7 +815,8 @@ __device__ __forceinline__ float exp_offset(float m) { return m == -INFINITY ? 0
 template <int D, bool BF16>
 __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, float sink_l2,
                                              bool row_valid, uint16_t *orow_ptr, float *lse_ptr,
-                                             uint64_t *o_free, int lane, bool write_lse = true) {
+                                             uint64_t *o_free, int lane, bool v8,
+                                             bool write_lse = true) {
   float o_scale = 1.f;
   if (sink_l2 != -INFINITY) {
     const float M = fmaxf(m, sink_l2);
@@ -779,10 +840,7 @@ __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, floa
 #pragma unroll
       for (int c = 0; c < 32; c += 2)
         pk[c / 2] = pack2<BF16>(__uint_as_float(o[c]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
-      uint4 *dst = reinterpret_cast<uint4 *>(orow_ptr + c0);
-#pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4)
-        dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+      store16w(orow_ptr + c0, pk, v8);
     }
   }
   if (row_valid && write_lse)
@@ -795,7 +853,7 @@ __device__ __forceinline__ void epilogue_row(uint32_t tO, float m, float l, floa
 template <int D>
 __device__ __forceinline__ void epilogue_part(uint32_t tO, float m, float l, bool row_valid,
                                               float *part_o_row, float *part_lse, uint64_t *o_free,
-                                              int lane, bool write_lse = true) {
+                                              int lane, bool v8, bool write_lse = true) {
   const bool any = l > 0.f;
   const float inv_l = any ? 1.f / l : 0.f;
 #pragma unroll
@@ -808,12 +866,13 @@ __device__ __forceinline__ void epilogue_part(uint32_t tO, float m, float l, boo
       if (lane == 0) ptx::mbar_arrive(o_free);
     }
     if (row_valid) {
-      float4 *dst = reinterpret_cast<float4 *>(part_o_row + c0);
+      uint32_t w[32];
 #pragma unroll
-      for (int v4 = 0; v4 < 8; ++v4)
-        dst[v4] = make_float4(__uint_as_float(o[4 * v4]) * inv_l, __uint_as_float(o[4 * v4 + 1]) * inv_l,
-                              __uint_as_float(o[4 * v4 + 2]) * inv_l,
-                              __uint_as_float(o[4 * v4 + 3]) * inv_l);
+      for (int c = 0; c < 32; ++c) w[c] = __float_as_uint(__uint_as_float(o[c]) * inv_l);
+      const uint32_t(&lo)[16] = *reinterpret_cast<const uint32_t(*)[16]>(&w[0]);
+      const uint32_t(&hi)[16] = *reinterpret_cast<const uint32_t(*)[16]>(&w[16]);
+      store16w(part_o_row + c0, lo, v8);
+      store16w(part_o_row + c0 + 16, hi, v8);
     }
   }
   if (row_valid && write_lse) *part_lse = any ? m + log2f(l) : -INFINITY;

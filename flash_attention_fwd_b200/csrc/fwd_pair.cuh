@@ -70,11 +70,11 @@ struct Barriers {
   uint64_t s_full[2];  // per query tile (A, B)
   uint64_t p_chunk[2][NCHUNK];
   uint64_t o_ready[2], o_free[2];
-  uint64_t v_fix;  // the last V tile's rows past the used keys are zeroed
+  uint64_t v_tail;  // an item's last V tile that runs past the used keys has landed
   uint64_t drain;
   ItemRing ring;
   uint32_t tmem_base;
-  int abort_flag;
+  AbortState abort;
 };
 
 template <int D>
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *sQ = smem;  // tile A at sQ, tile B at sQ + Q_BYTES
   uint8_t *sKV = smem + 2 * Q_BYTES;
   Barriers *bars = reinterpret_cast<Barriers *>(sKV + NSLOT * KV_BYTES);
-  volatile int *abort_flag = &bars->abort_flag;
+  AbortState *abort_flag = &bars->abort;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -289,13 +289,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&bars->o_ready[i], 1);
       ptx::mbar_init(&bars->o_free[i], 4);
     }
-    ptx::mbar_init(&bars->v_fix, 1);
+    ptx::mbar_init(&bars->v_tail, 1);
     ptx::mbar_init(&bars->drain, 1);
     for (int i = 0; i < ITEM_RING; ++i) {
       ptx::mbar_init(&bars->ring.full[i], 1);
       ptx::mbar_init(&bars->ring.empty[i], RING_CONSUMERS);
     }
-    bars->abort_flag = 0;
+    bars->abort.init();
     ptx::mbar_init_fence();
   }
   if (warp == PRODUCER_WARP && lane == 0) {
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t rs = 0, rph = 0, q_count = 0;
       bool ok = true;
       KVProducer<BN, D, NSLOT> kv;
-      kv.init(sKV, bars->full, bars->empty, &bars->v_fix, abort_flag);
+      kv.init(sKV, bars->full, bars->empty, &bars->v_tail, abort_flag);
       // Q tiles of an item (lane 0): packed, tile t = the next (BM >> pack)
       // tokens of all query heads of kv_h; otherwise tile t = head 2u + t
       auto load_q = [&](const WorkItem &w) -> bool {
@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == MMA_WARP && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       uint32_t rs = 0, rph = 0;
-      uint32_t slot = 0, phase = 0, g = 0, items = 0, nfix = 0;
+      uint32_t slot = 0, phase = 0, g = 0, items = 0;
       bool ok = true;
       const uint32_t sQ_addr = ptx::smem_u32(sQ);
       const uint32_t sKV_addr = ptx::smem_u32(sKV);
@@ -425,15 +425,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       };
       // O_t += P_t V for keys [c * CHUNK_KEYS, (c + 1) * CHUNK_KEYS) (P from
-      // TMEM, V MN-major), in steps of 16 keys; steps from `steps` on (past
-      // the used keys of the item's last tile) are skipped.  Step 0 always
-      // runs, so the first product of an item still initialises O.
-      auto issue_pv_chunk = [&](int t, uint32_t vslot, int c, bool acc, int steps) {
+      // TMEM, V MN-major), in steps of 16 keys
+      auto issue_pv_chunk = [&](int t, uint32_t vslot, int c, bool acc) {
         const uint32_t vbase = sKV_addr + vslot * KV_BYTES;
         constexpr int KS = CHUNK_KEYS / 16;
 #pragma unroll
         for (int kk = KS * c; kk < KS * c + KS; ++kk) {
-          if (kk >= steps) break;
           uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
           ptx::mma_ts(tmem + O_COL0 + t * D, tmem + t * BN + kk * 8, bdesc, IDESC_PV,
                       (acc || kk > KS * c) ? 1u : 0u);
@@ -450,7 +447,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (w.hu < 0) break;
         const int n = w.n_kv;
         if (n == 0) continue;
-        const int tail_keys = last_tile_keys<BN>(w);
         if (!(ok = wait_bar(&bars->q_full, items & 1u, abort_flag))) break;
         ptx::tc_fence_after();
         uint32_t ks;
@@ -470,12 +466,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int t = 0; t < NT; ++t) {
             if (more && t == 0 && !(ok = take_slot(ks_next))) break;
             if (t == 0 && !(ok = take_slot(vs))) break;
-            if (t == 0 && j == n - 1 && tail_needs_fix(tail_keys)) {
-              // the producer has zeroed the rows past the used keys
-              if (!(ok = wait_bar(&bars->v_fix, nfix & 1u, abort_flag))) break;
-              ++nfix;
-              ptx::tc_fence_after();
-            }
             if (j == 0 && items > 0) {
               if (!(ok = wait_bar(&bars->o_free[t], (items - 1) & 1u, abort_flag))) break;
               ptx::tc_fence_after();
@@ -484,7 +474,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int c = 0; c < NCHUNK; ++c) {
               if (!(ok = wait_bar(&bars->p_chunk[t][c], par, abort_flag))) break;
               ptx::tc_fence_after();
-              issue_pv_chunk(t, vs, c, j > 0 || c > 0, j == n - 1 ? pv_steps(tail_keys) : BN / 16);
+              issue_pv_chunk(t, vs, c, j > 0 || c > 0);
             }
             if (!ok) break;
             if (j == n - 1) ptx::mma_commit(&bars->o_ready[t]);
@@ -588,13 +578,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tc_fence_after();
       if (w.part < 0 && rep == 1) {
         epilogue_row<D, BF16>(tO, m, l, sink_log2(p, h), row_valid, orow_ptr, p.lse + orow,
-                              &bars->o_free[t], lane);
+                              &bars->o_free[t], lane, p.out_v8 != 0);
       } else {
         // a piece of the row: the key-range piece, and with replicated rows
         // the copy within it
         const size_t piece = (size_t)(w.part < 0 ? 0 : w.part) * rep + (rep > 1 ? copy : 0);
         epilogue_part<D>(tO, m, l, row_valid, p.part_o + (piece * p.part_rows + orow) * D,
-                         p.part_lse + piece * p.part_rows + orow, &bars->o_free[t], lane);
+                         p.part_lse + piece * p.part_rows + orow, &bars->o_free[t], lane,
+                         p.part_v8 != 0);
       }
     }
     end_of_kernel();

@@ -64,12 +64,12 @@ struct Barriers {
   uint64_t q_full, q_empty;
   uint64_t s_full[2], p_full[2];
   uint64_t pv_done, o_ready, o_free, drain;
-  uint64_t v_fix;  // the last V tile's rows past the used keys are zeroed
+  uint64_t v_tail;  // an item's last V tile that runs past the used keys has landed
   uint64_t xf[4], xr[4];  // row-pair exchange, per TMEM lane quarter: value written / read
   float xch[2][BM];       // exchanged value of row r from column half h
   ItemRing ring;
   uint32_t tmem_base;
-  int abort_flag;
+  AbortState abort;
 };
 
 // Exchange of one float between the two threads of a row (one per column
@@ -82,11 +82,11 @@ struct RowSwap {
   float *mine;
   const volatile float *other;
   uint64_t *xf, *xr;
-  volatile int *abort_flag;
+  AbortState *abort_flag;
   uint32_t n;
   int lane;
   __device__ void init(float *a, const float *b, uint64_t *f, uint64_t *rd, int ln,
-                       volatile int *abort) {
+                       AbortState *abort) {
     mine = a;
     other = b;
     xf = f;
@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *sQ = smem;
   uint8_t *sKV = smem + Q_BYTES;
   Barriers *bars = reinterpret_cast<Barriers *>(sKV + NSLOT * KV_BYTES);
-  volatile int *abort_flag = &bars->abort_flag;
+  AbortState *abort_flag = &bars->abort;
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -257,12 +257,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&bars->xr[i], 2);
     }
     ptx::mbar_init(&bars->drain, 1);
-    ptx::mbar_init(&bars->v_fix, 1);
+    ptx::mbar_init(&bars->v_tail, Cfg<D>::SPLIT);  // one arrival per V slice
     for (int i = 0; i < ITEM_RING; ++i) {
       ptx::mbar_init(&bars->ring.full[i], 1);
       ptx::mbar_init(&bars->ring.empty[i], RING_CONSUMERS);
     }
-    bars->abort_flag = 0;
+    bars->abort.init();
     ptx::mbar_init_fence();
   }
   if (warp == PRODUCER_WARP && lane == 0) {
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t rs = 0, rph = 0, q_count = 0;
       bool ok = true;
       KVProducer<BN, DS, NSLOT, SPLIT> kv;
-      kv.init(sKV, bars->full, bars->empty, &bars->v_fix, abort_flag);
+      kv.init(sKV, bars->full, bars->empty, &bars->v_tail, abort_flag);
       // Q tile of an item (lane 0)
       auto load_q = [&](const WorkItem &w) -> bool {
         if (!wait_bar(&bars->q_empty, (q_count & 1u) ^ 1u, abort_flag)) return false;
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t rs = 0, rph = 0;
-      uint32_t slot = 0, phase = 0, g = 0, items = 0, nfix = 0;
+      uint32_t slot = 0, phase = 0, g = 0, items = 0;
       bool ok = true;
       const uint32_t sQ_addr = ptx::smem_u32(sQ);
       const uint32_t sKV_addr = ptx::smem_u32(sKV);
@@ -376,15 +376,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       // O += P V over the BN keys in steps of 16 (P from TMEM, V MN-major);
       // slice i of V feeds O's columns [i * DS, (i + 1) * DS) and its slot is
-      // released right after its MMAs.  Steps from `steps` on (past the used
-      // keys of the item's last tile) are skipped; step 0 always runs.
-      auto issue_pv = [&](uint32_t buf, const uint32_t (&vs)[SPLIT], bool acc, int steps) {
+      // released right after its MMAs
+      auto issue_pv = [&](uint32_t buf, const uint32_t (&vs)[SPLIT], bool acc) {
 #pragma unroll
         for (int i = 0; i < SPLIT; ++i) {
           const uint32_t vbase = sKV_addr + vs[i] * KV_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BN / 16; ++kk) {
-            if (kk >= steps) break;
             uint64_t bdesc = ptx::sdesc_sw128(vbase + kk * (16 * 128), BN * 128, 1024);
             ptx::mma_ts(tmem + O_COL + i * DS, tmem + buf * BN + P_COL + kk * 8, bdesc, IDESC_PV,
                         (acc || kk > 0) ? 1u : 0u);
@@ -423,14 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           uint32_t vs[SPLIT];
           if (!(ok = take_tile(vs))) break;
-          const int keys = j == n - 1 ? last_tile_keys<BN>(w) : BN;
-          if (tail_needs_fix(keys)) {
-            // the producer has zeroed the rows past the used keys
-            if (!(ok = wait_bar(&bars->v_fix, nfix & 1u, abort_flag))) break;
-            ++nfix;
-            ptx::tc_fence_after();
-          }
-          issue_pv(buf, vs, j > 0, pv_steps(keys));
+          issue_pv(buf, vs, j > 0);
           ptx::mma_commit(&bars->pv_done);
           if (j == n - 1) ptx::mma_commit(&bars->o_ready);
           if (j + 2 < n) {
@@ -533,12 +524,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       l += l_other;
       if (w.part < 0)
         epilogue_row<DC, BF16>(tO, m, l, sink_log2(p, w.hu), row_valid, orow_ptr + h * DC,
-                               p.lse + orow, &bars->o_free, lane, h == 0);
+                               p.lse + orow, &bars->o_free, lane, p.out_v8 != 0, h == 0);
       else
         epilogue_part<DC>(tO, m, l, row_valid,
                           p.part_o + ((size_t)w.part * p.part_rows + orow) * D + h * DC,
                           p.part_lse + (size_t)w.part * p.part_rows + orow, &bars->o_free, lane,
-                          h == 0);
+                          p.part_v8 != 0, h == 0);
     }
   }
 

@@ -105,7 +105,7 @@ static bool encode_qkv_map(EncodeTiledFn enc, CUtensorMap *map, const void *base
 // when the calling thread's context differs.  Calls from several host
 // threads are safe: the set-up runs under the device's mutex.
 constexpr int MAX_DEVICES = 64;
-constexpr int KERNEL_SLOTS = 24;  // forward 0..9, backward 10..17, replicated rows 18..21
+constexpr int KERNEL_SLOTS = 26;  // forward 0..9, backward 10..17 and 22..25, replicated rows 18..21
 struct DeviceInfo {
   std::mutex mu;
   std::atomic<unsigned long long> ctx_id;  // context the state below belongs to (0: none)
@@ -443,6 +443,8 @@ static int fwd_impl(const void *q, const void *k, const void *v, const int32_t *
   kp.part_rows = (long long)total_q * num_heads;
   kp.part_o = nullptr;
   kp.part_lse = nullptr;
+  kp.out_v8 = aligned(out, 32) ? 1 : 0;
+  kp.part_v8 = aligned(workspace, 32) ? 1 : 0;
   if (kp.split_tiles > 0 || kp.rep > 1) {
     const int slots = kp.max_parts * kp.rep;
     const size_t need = split_workspace_bytes(total_q, num_heads, D, slots);
@@ -642,6 +644,12 @@ extern "C" int varlen_attn_device_status(unsigned int *status, int clear) {
       return VARLEN_ERR_LAUNCH;
   }
   return VARLEN_OK;
+}
+
+extern "C" int varlen_attn_set_wait_limit(unsigned long long ns) {
+  const unsigned long long v = ns ? ns : WAIT_TIMEOUT_NS;
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof v) == cudaSuccess ? VARLEN_OK
+                                                                           : VARLEN_ERR_LAUNCH;
 }
 
 extern "C" int varlen_attn_abi_version(void) { return 6; }

@@ -303,6 +303,19 @@ const char *varlen_attn_strerror(int code);
 int varlen_attn_device_status(unsigned int *status, int clear);
 
 /*
+ * Testing hook: the limit, in nanoseconds, of the kernels' pipeline waits on
+ * the current device (0 restores the default of 2 s).  With a limit far below
+ * a pipeline's ordinary waits (a microsecond), the kernels of the following
+ * launches give up those waits, set bit 1 of the status word, drain their own
+ * in-flight copies and tensor-core work and return; their outputs are then
+ * incomplete.  This is how the tests exercise that abort path without a
+ * fault.  The end-of-kernel drains keep their 2 s limit.  Synchronous with
+ * the host; not meant for production use.  Returns VARLEN_OK or
+ * VARLEN_ERR_LAUNCH.
+ */
+int varlen_attn_set_wait_limit(unsigned long long ns);
+
+/*
  * Backward of the packed attention forward (varlen_attn_fwd_v1's operation):
  * the CPU backward loop of boostr 0.2.0, src/ops/cpu/attention/
  * varlen_attention.rs (VarLenAttentionOps::varlen_attention_bwd).  For every
@@ -330,7 +343,7 @@ size_t varlen_attn_bwd_workspace_size(int64_t total_q, int num_heads);
  *   out, lse     the forward's outputs for these inputs (out dtype, lse float32)
  *   cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k, max_seqlen_q,
  *   max_seqlen_k, num_heads, num_kv_heads, causal, scale, dtype
- *                as in varlen_attn_fwd_v1; head_dim must be 64 or 128.
+ *                as in varlen_attn_fwd_v1 (head_dim 64, 128 or 256).
  *   dq           [total_q, H, D] dtype, written for rows [0, cu_seqlens_q[batch])
  *   dk, dv       [total_k, Hkv, D] dtype, written for rows [0, cu_seqlens_k[batch]);
  *                a key that no query sees gets zeros.

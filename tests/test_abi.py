@@ -196,7 +196,7 @@ BWD = dict(dout_ptr=0x11000, q_ptr=0x10000, k_ptr=0x20000, v_ptr=0x30000, out_pt
 
 
 @pytest.mark.parametrize("change,code", [
-    (dict(head_dim=256), -2),                # the backward covers D = 64, 128
+    (dict(head_dim=96), -2),                 # the backward covers D = 64, 128, 256
     (dict(num_heads=5), -2),
     (dict(dtype_code=3), -3),
     (dict(dout_ptr=0), -1),

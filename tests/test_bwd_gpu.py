@@ -1,5 +1,5 @@
 """GPU parity of the backward (varlen_attn_bwd_v1) against the fp64 oracle's
-restatement of the page's varlen_attention_bwd loop.
+backward (the gradient the page's varlen_attention_bwd defines).
 
 Both sides get the same inputs: Q, K, V, a seeded dO, and O / LSE taken from
 the oracle's forward and rounded to the storage types the GPU path reads
@@ -100,12 +100,35 @@ def check_bwd(case, dout_seed=0, what=None):
     return got
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 @pytest.mark.parametrize("causal", [True, False])
 def test_backward_ragged_tiles(D, dtype, causal):
     case = workloads.make_case(LENS, None, 4, 2, D, dtype, causal, seed=800 + D + causal)
     check_bwd(case, D + causal)
+
+
+@pytest.mark.parametrize("H,Hkv", [(8, 8), (6, 2), (3, 1)])
+def test_backward_head_dim_256_head_layouts(H, Hkv):
+    # head dim 256: 32-key tiles in the dQ pass, dK / dV in two column halves
+    case = workloads.make_case([200, 77, 130, 1], None, H, Hkv, 256, "bf16", True,
+                               seed=860 + H + Hkv)
+    check_bwd(case, 7 + H)
+
+
+def test_backward_head_dim_256_wide_logits_fp16():
+    # the wide-head configuration's shape and logit scale (Q, K ~ N(0, 3^2)),
+    # on two sequences of 1024 so that the fp64 oracle stays quick
+    case = workloads.make_case([1024, 1024], None, 4, 4, 256, "fp16", True, seed=870,
+                               sigma_q=3.0, sigma_k=3.0)
+    check_bwd(case, 11)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_head_dim_256_q_and_k_lengths_differ(causal):
+    case = workloads.make_case([70, 200, 5, 131], [250, 64, 1, 300], 4, 2, 256, "fp16", causal,
+                               seed=880 + causal)
+    check_bwd(case, 13)
 
 
 @pytest.mark.parametrize("H,Hkv", [(8, 2), (3, 1), (3, 3)])

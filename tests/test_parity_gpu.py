@@ -201,3 +201,56 @@ def test_sequence_table_past_the_buffers_is_clamped(splits):
         bad = dataclasses.replace(case, cu_q=cq, cu_k=ck)
         out, lse, _, _ = run_gpu(bad, max_q=max_q, max_k=2700, num_splits=splits)
         check_close(out, lse, ref_out, ref_lse, "table past the buffers")
+
+
+def _off16(shape, dtype, dev):
+    """A contiguous tensor whose data starts 16 bytes past a 32-byte boundary
+    (the entry points require 16-byte alignment only)."""
+    n = 1
+    for s in shape:
+        n *= s
+    e = torch.empty((), dtype=dtype).element_size()
+    buf = torch.empty(n + 64 // e, dtype=dtype, device=dev)
+    k = ((-buf.data_ptr()) % 32 + 16) % 32 // e
+    t = buf[k:k + n].view(shape)
+    assert t.data_ptr() % 32 == 16
+    return t
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_rows_written_with_16_byte_alignment(D):
+    # rows are stored 32 bytes at a time when the output starts on a 32-byte
+    # boundary, 16 bytes at a time otherwise: both give the same bits
+    import flash_attention_fwd_b200 as fa
+    case = workloads.make_case([300, 77, 129], None, 4, 2, D, "bf16", True, seed=1700 + D)
+    dev = torch.device("cuda", 0)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    cq, ck = case.cu_q.to(dev), case.cu_k.to(dev)
+    o32, l32 = fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, True)
+    o16 = _off16(q.shape, q.dtype, dev)
+    _, l16 = fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, True, out=o16)
+    torch.cuda.synchronize()
+    assert o32.data_ptr() % 32 == 0
+    assert torch.equal(o32.view(torch.int16), o16.view(torch.int16)) and torch.equal(l32, l16)
+    # key-range pieces in a workspace that starts 16 bytes past a 32-byte boundary
+    dec = workloads.make_case([1, 3, 2], [3000, 1700, 2500], 8, 2, D, "bf16", False, seed=1710)
+    q, k, v = dec.q.to(dev), dec.k.to(dev), dec.v.to(dev)
+    cq, ck = dec.cu_q.to(dev), dec.cu_k.to(dev)
+    nbytes = fa.fwd_workspace_size(dec.Tq, dec.H, dec.Hkv, D, dec.max_q, dec.max_k, 4)
+    ws = _off16((nbytes,), torch.uint8, dev)
+    a, la = fa.varlen_attn_fwd(q, k, v, cq, ck, dec.max_q, dec.max_k, num_splits=4)
+    b, lb = fa.varlen_attn_fwd(q, k, v, cq, ck, dec.max_q, dec.max_k, num_splits=4, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16)) and torch.equal(la, lb)
+    # the backward's gradients
+    g = torch.Generator("cpu").manual_seed(1720)
+    dout = torch.randn(case.q.shape, generator=g).to(case.q.dtype).to(dev)
+    args = [t.to(dev) for t in (case.q, case.k, case.v)]
+    grads = fa.varlen_attn_bwd(dout, *args, o32, l32, case.cu_q.to(dev), case.cu_k.to(dev),
+                               case.max_q, case.max_k, True)
+    offs = [_off16(t.shape, t.dtype, dev) for t in grads]
+    fa.varlen_attn_bwd(dout, *args, o32, l32, case.cu_q.to(dev), case.cu_k.to(dev),
+                       case.max_q, case.max_k, True, dq=offs[0], dk=offs[1], dv=offs[2])
+    torch.cuda.synchronize()
+    for x, y in zip(grads, offs):
+        assert torch.equal(x.view(torch.int16), y.view(torch.int16))
