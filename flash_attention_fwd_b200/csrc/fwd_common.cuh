@@ -371,6 +371,7 @@ struct Scheduler {
         const unsigned hit = __ballot_sync(0xffffffffu, cur_units + incl > unit);
         const int src = __ffs(hit) - 1;
         const int before = __shfl_sync(0xffffffffu, incl - u, src);
+        const int u_b = __shfl_sync(0xffffffffu, u, src);
         qs = __shfl_sync(0xffffffffu, qs, src);
         lq = __shfl_sync(0xffffffffu, lq, src);
         ks = __shfl_sync(0xffffffffu, ks, src);
@@ -378,12 +379,18 @@ struct Scheduler {
         cur_b += src;
         cur_units += before;
         w.b = cur_b;
-        const int k = (int)(unit - cur_units);
+        int k = (int)(unit - cur_units);
         const int nk = (lk + BM - 1) / BM;
         int qt, t0 = 0, nt = 0;
         w.part = -1;
         if (folded(lq, lk)) {
-          // folded unit: ranges k and nq - 1 - k, or the middle range alone
+          // folded unit: ranges k and nq - 1 - k, or the middle range alone.
+          // The sequence's u_b units x HU head units at this level are taken
+          // unit fastest: the units in flight then cover few (sequence, head)
+          // pairs, whose K/V stays in L2 while all their query ranges read it.
+          const long long o = local - (long long)cur_units * HU;
+          k = (int)(o % u_b);
+          w.hu = (int)(o / u_b);
           const int nq = (lq + U - 1) / U;
           if (level == nq + 1 && nq >= 2) {
             qt = k;
