@@ -140,6 +140,37 @@ def device_status(clear: bool = True) -> int:
     return int(val.value)
 
 
+# Opt-in check after every varlen_attn_fwd / varlen_attn_bwd call: when this
+# environment variable is set to anything but "" or "0", the call waits for
+# its stream and raises VarlenAttnError(VARLEN_ERR_DEVICE) if the device
+# status word is set (a bounded wait inside a kernel ran out, so that call's
+# results may be incomplete).  Off by default: the check synchronises.
+STATUS_CHECK_ENV = "VARLEN_ATTN_CHECK_STATUS"
+VARLEN_ERR_DEVICE = -6
+
+
+def status_check_enabled() -> bool:
+    return os.environ.get(STATUS_CHECK_ENV, "") not in ("", "0")
+
+
+def raise_on_status(word: int) -> None:
+    """Raises VarlenAttnError(VARLEN_ERR_DEVICE) when `word` (a device status
+    word) is non-zero."""
+    if word:
+        raise VarlenAttnError(VARLEN_ERR_DEVICE,
+                              "device status word 0x%x: a bounded wait inside a kernel ran out; "
+                              "the results of the calls since the last check may be incomplete"
+                              % word)
+
+
+def check_device_status(stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Waits for `stream` (default: the current stream), then reads and clears
+    the device status word of the current device and raises
+    VarlenAttnError(VARLEN_ERR_DEVICE) when it was set."""
+    (stream or torch.cuda.current_stream()).synchronize()
+    raise_on_status(device_status(clear=True))
+
+
 def set_wait_limit(ns: int = 0) -> None:
     """Testing hook (varlen_attn_set_wait_limit): the kernels' pipeline-wait
     limit on the current device in ns; 0 restores the default (2 s)."""
@@ -312,6 +343,8 @@ def varlen_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             stream.cuda_stream, int(window_size_left), int(window_size_right), addr(seqused_k),
             addr(page_table), stride, page_size, addr(sinks), splits,
             addr(workspace) if ws_bytes else 0, ws_bytes)
+        if rc == VARLEN_OK and status_check_enabled():
+            check_device_status(stream)
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return out, lse
@@ -422,6 +455,8 @@ def varlen_attn_bwd(dout: torch.Tensor, q: torch.Tensor, k: torch.Tensor, v: tor
             int(max_seqlen_k), H, Hkv, D, causal, 0.0 if scale is None else float(scale),
             DTYPE_CODES[q.dtype], addr(dq), addr(dk), addr(dv), addr(workspace),
             workspace.numel() * workspace.element_size(), stream.cuda_stream)
+        if rc == VARLEN_OK and status_check_enabled():
+            check_device_status(stream)
     if rc != VARLEN_OK:
         raise VarlenAttnError(rc, strerror(rc))
     return dq, dk, dv

@@ -241,3 +241,19 @@ def test_noalloc_backward_rejects_before_any_device_call():
         "dout_ptr", "q_ptr", "k_ptr", "v_ptr", "out_ptr", "lse_ptr", "cu_q_ptr", "cu_k_ptr")),
         0, 10, 10, 5, 5, 8, 2, 128, 1, 0.0, 0, V(0x61000), V(0x62000), V(0x63000), V(0))
     assert rc == 0
+
+
+def test_opt_in_status_check_helpers(monkeypatch):
+    """The binding's opt-in device status check: the switch and the error it
+    raises (no device needed)."""
+    import flash_attention_fwd_b200 as fa
+    monkeypatch.delenv(fa.STATUS_CHECK_ENV, raising=False)
+    assert not fa.status_check_enabled()
+    for val, on in (("", False), ("0", False), ("1", True), ("yes", True)):
+        monkeypatch.setenv(fa.STATUS_CHECK_ENV, val)
+        assert fa.status_check_enabled() == on
+    fa.raise_on_status(0)
+    with pytest.raises(fa.VarlenAttnError) as err:
+        fa.raise_on_status(1)
+    assert err.value.code == fa.VARLEN_ERR_DEVICE == -6
+    assert "0x1" in str(err.value)

@@ -101,3 +101,34 @@ def test_backward_abort_then_recover():
         assert err.max() <= 1.5e-2 * np.abs(ref).max(), name
         assert err.mean() <= 2.0 ** -8 * np.abs(ref).mean(), name
     assert fa.device_status(clear=True) == 0
+
+
+def test_opt_in_status_check_raises(monkeypatch):
+    """With VARLEN_ATTN_CHECK_STATUS set, the binding waits for each call and
+    raises VARLEN_ERR_DEVICE when a bounded wait ran out; a normal call does
+    not raise."""
+    import flash_attention_fwd_b200 as fa
+    lq, lk, H, Hkv, D, dt, causal = CASES[0]
+    case = workloads.make_case(lq, lk, H, Hkv, D, dt, causal, seed=4200)
+    dev = torch.device("cuda", 0)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    cq, ck = case.cu_q.to(dev), case.cu_k.to(dev)
+    long_q, long_k = (t.to(dev) for t in _with_empty_sequences(case))
+    monkeypatch.setenv(fa.STATUS_CHECK_ENV, "1")
+    fa.device_status(clear=True)
+    fa.varlen_attn_fwd(q, k, v, cq, ck, case.max_q, case.max_k, case.causal, num_splits=1)
+    torch.cuda.synchronize()
+    fa.set_wait_limit(SHORT_NS)
+    try:
+        with pytest.raises(fa.VarlenAttnError) as err:
+            fa.varlen_attn_fwd(q, k, v, long_q, long_k, case.max_q, case.max_k, case.causal,
+                               num_splits=1)
+        assert err.value.code == fa.VARLEN_ERR_DEVICE
+    finally:
+        torch.cuda.synchronize()
+        fa.set_wait_limit(0)
+    fa.device_status(clear=True)
+    # the check stays on: a normal call on fresh buffers passes it and matches
+    out, lse, _, _ = run_gpu(case)
+    ref_out, ref_lse = oracle.run_case(case)
+    check_close(out, lse, ref_out, ref_lse, "after the raised check")
