@@ -797,6 +797,16 @@ __device__ __forceinline__ void tmem_st<64>(uint32_t taddr, const uint32_t (&r)[
 // log2 units (-inf when every key of the tile is hidden from the row).  m
 // stays -inf until the row has seen a visible key; the first finite max then
 // "rescales" O and l by exp2(-inf) = 0, which is exact because both are 0.
+// s[c] = -inf for every column whose key offset c0 + c lies outside
+// [lo, hi), as one select per column: the bounds differ from row to row, and
+// an `if` per column made the warp take both paths of 128 branches.
+template <int N>
+__device__ __forceinline__ void mask_outside(float (&s)[N], int lo, int hi, int c0 = 0) {
+#pragma unroll
+  for (int c = 0; c < N; ++c)
+    s[c] = ptx::slct_f32(s[c], -INFINITY, min(c0 + c - lo, hi - 1 - (c0 + c)));
+}
+
 __device__ __forceinline__ void update_max(int j, float mx, float &m, float &alpha, bool &need) {
   if (j == 0) {
     m = mx;

@@ -95,11 +95,7 @@ __device__ __forceinline__ void softmax_tile_chunked(uint32_t tS, uint32_t tO, i
   float s[BN];
 #pragma unroll
   for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(sr[c]);
-  if (need_mask) {
-#pragma unroll
-    for (int c = 0; c < BN; ++c)
-      if (c < lo || c >= hi) s[c] = -INFINITY;
-  }
+  if (need_mask) mask_outside(s, lo, hi);
   float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
   for (int c = 4; c + 8 <= BN; c += 8) {
@@ -180,12 +176,7 @@ __device__ __forceinline__ void softmax_tile_rep(uint32_t tS, uint32_t tO, int c
   float s[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(sr[c]);
-  if (need_mask) {
-    const int k0 = 32 * copy;
-#pragma unroll
-    for (int c = 0; c < 32; ++c)
-      if (k0 + c < lo || k0 + c >= hi) s[c] = -INFINITY;
-  }
+  if (need_mask) mask_outside(s, lo, hi, 32 * copy);
   float mx0 = s[0], mx1 = s[1];
 #pragma unroll
   for (int c = 2; c < 32; c += 4) {

@@ -128,11 +128,7 @@ __device__ __forceinline__ bool softmax_half(uint32_t tS, uint32_t tP, uint32_t 
   float s[HB];
 #pragma unroll
   for (int c = 0; c < HB; ++c) s[c] = __uint_as_float(sr[c]);
-  if (need_mask) {
-#pragma unroll
-    for (int c = 0; c < HB; ++c)
-      if (c < lo || c >= hi) s[c] = -INFINITY;
-  }
+  if (need_mask) mask_outside(s, lo, hi);
   float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
   for (int c = 4; c + 8 <= HB; c += 8) {

@@ -281,6 +281,13 @@ __device__ __forceinline__ float add_hi16(uint32_t packed, float acc) {
   return d;
 }
 
+// c >= 0 ? a : b, as one select instruction.
+__device__ __forceinline__ float slct_f32(float a, float b, int c) {
+  float d;
+  asm("slct.f32.s32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "r"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
